@@ -1,0 +1,223 @@
+/*
+ * s6_oracle.c -- float64 CPU oracle for the S6 selective scan.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline leg do.  It shares no code, header, table or constant with the CUDA
+ * path.  It is deliberately plain: one channel at a time, one token at a time,
+ * one state coordinate at a time, every step in double precision, in the order
+ * the pages state the method.
+ *
+ * What it follows (page title, then section):
+ *  - "mamba, live" (soundlark.studio), "what is actually running": the block's
+ *    streaming form -- causal depthwise conv of width 4 + SiLU, dt = softplus(.),
+ *    A = -exp(A_log), h <- exp(dt*A)*h + (dt*B)*xc, y = <h, C> + D*xc, output
+ *    gated by SiLU(z).
+ *  - "the s6 cell" (soundlark.studio), "the recurrence": the same three lines
+ *    with the decay written as a power of two; Delta*A <= 0.
+ *  - "Carry context through a selective state" (tensorviz.dev), "Recorded
+ *    numerical example" and the model manifest's `steps` ("local", "select",
+ *    "state", "read"): exact diagonal zero-order hold,
+ *    B_bar = (exp(Delta*A) - 1) / A * B, the conv left-padded with zeros so it
+ *    reads the current and the K-1 earlier tokens, C reading the UPDATED state,
+ *    and D multiplying the conv output.
+ *
+ * Readings where the pages leave a step open:
+ *  - softplus is log(1 + e^v) exactly (no large-v identity switch); written as
+ *    max(v,0) + log1p(exp(-|v|)) so that it neither overflows nor cancels.
+ *  - the conv has a bias (nullable by passing 0).
+ *  - the scan starts from a zero state and a zero conv history unless a state
+ *    is passed in (the streaming step and the resume case).
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#define S6O_ABI_VERSION 1
+
+int s6o_abi_version(void) { return S6O_ABI_VERSION; }
+
+/* softplus(v) = log(1 + e^v) ("mamba, live": dt = softplus(dt_proj(.)) > 0). */
+double s6o_softplus(double v)
+{
+    double m = v > 0.0 ? v : 0.0;
+    return m + log1p(exp(-fabs(v)));
+}
+
+/* SiLU(v) = v * sigmoid(v) = v / (1 + e^-v). */
+double s6o_silu(double v)
+{
+    if (v >= 0.0)
+        return v / (1.0 + exp(-v));
+    /* same value, written so e^-v cannot overflow for very negative v */
+    double e = exp(v);
+    return v * e / (1.0 + e);
+}
+
+/* A = -exp(A_log) < 0 ("mamba, live"; "the s6 cell", "the recurrence"). */
+double s6o_A(double A_log) { return -exp(A_log); }
+
+/* Decay factor A_bar = exp(Delta * A). */
+double s6o_decay(double delta, double A_log) { return exp(delta * s6o_A(A_log)); }
+
+/* Input term multiplying B*u.
+ *  simplified (zoh = 0): Delta            ("mamba, live"; "the s6 cell")
+ *  exact ZOH  (zoh = 1): (exp(Delta*A) - 1) / A   (the TinyMamba example,
+ *              Mamba paper Eq. 4, as quoted on "Carry context ...").     */
+double s6o_write_gain(double delta, double A_log, int zoh)
+{
+    if (!zoh)
+        return delta;
+    double A = s6o_A(A_log);
+    return expm1(delta * A) / A;
+}
+
+/* h <- A_bar * h + write ("Decay the old state and add the current write"). */
+double s6o_update(double h, double a_bar, double write) { return a_bar * h + write; }
+
+/* Causal depthwise conv at one token:
+ *   pre = bias + sum_{k<K-1} w[k] * hist[k] + w[K-1] * x_t
+ * hist holds the K-1 previous pre-conv inputs, oldest first (zeros before the
+ * first token).  Returns the pre-activation; the caller applies SiLU.        */
+double s6o_conv_pre(int K, const double *w, double bias, const double *hist, double x_t)
+{
+    double acc = bias;
+    for (int k = 0; k < K - 1; ++k)
+        acc += w[k] * hist[k];
+    acc += w[K - 1] * x_t;
+    return acc;
+}
+
+/*
+ * One channel over L tokens.
+ *
+ *   x       [L]     pre-conv input when K > 0, else the scan input u itself
+ *   dt_raw  [L]     raw step size (before bias and softplus)
+ *   z       [L]     gate input, or NULL for no gate
+ *   Bm, Cm  [L*N]   per-token B_t and C_t rows of this channel's sequence
+ *   A_log   [N]     this channel's A_log row
+ *   D, dt_bias      this channel's skip weight and step-size bias
+ *   K               conv width (0 = no conv: x is u)
+ *   conv_w  [K]     taps, oldest first; conv_b the bias
+ *   hist    [K-1]   in: conv history (oldest first), or NULL for zeros;
+ *                   out (if hist_out != NULL): history after the last token
+ *   h       [N]     in: initial state, or NULL for zeros
+ *   y       [L]     out
+ *   h_out   [N]     out (may be NULL)
+ *   xc_out  [L]     out: the conv output u_t (may be NULL)
+ *   delta_out [L]   out: Delta_t (may be NULL)
+ */
+void s6o_scan_channel(int64_t L, int N, int K, int zoh,
+                      const double *x, const double *dt_raw, const double *z,
+                      const double *Bm, const double *Cm,
+                      const double *A_log, double D, double dt_bias,
+                      const double *conv_w, double conv_b,
+                      const double *hist_in, const double *h_in,
+                      double *y, double *h_out, double *hist_out,
+                      double *xc_out, double *delta_out)
+{
+    double hist[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    double h[64];
+    for (int n = 0; n < N; ++n)
+        h[n] = h_in ? h_in[n] : 0.0;
+    if (K > 1 && hist_in)
+        for (int k = 0; k < K - 1; ++k)
+            hist[k] = hist_in[k];
+
+    for (int64_t t = 0; t < L; ++t) {
+        /* conv + SiLU ("Gather local context before the scan") */
+        double u;
+        if (K > 0) {
+            double pre = s6o_conv_pre(K, conv_w, conv_b, hist, x[t]);
+            for (int k = 0; k + 1 < K - 1; ++k)
+                hist[k] = hist[k + 1];
+            if (K > 1)
+                hist[K - 2] = x[t];
+            u = s6o_silu(pre);
+        } else {
+            u = x[t];
+        }
+        /* Delta ("Choose dynamics from the current input") */
+        double delta = s6o_softplus(dt_raw[t] + dt_bias);
+        if (xc_out)
+            xc_out[t] = u;
+        if (delta_out)
+            delta_out[t] = delta;
+        /* state update and readout ("Decay the old state ...", "Read, gate ...") */
+        double acc = 0.0;
+        for (int n = 0; n < N; ++n) {
+            double a_bar = s6o_decay(delta, A_log[n]);
+            double write = s6o_write_gain(delta, A_log[n], zoh) * Bm[t * N + n] * u;
+            h[n] = s6o_update(h[n], a_bar, write);
+            acc += h[n] * Cm[t * N + n];
+        }
+        double out = acc + D * u;
+        if (z)
+            out *= s6o_silu(z[t]);
+        y[t] = out;
+    }
+    if (h_out)
+        for (int n = 0; n < N; ++n)
+            h_out[n] = h[n];
+    if (hist_out && K > 1)
+        for (int k = 0; k < K - 1; ++k)
+            hist_out[k] = hist[k];
+}
+
+/*
+ * Many independent channels in one call (no arithmetic beyond the loop above).
+ * Channel c reads its sequences at x + c*L etc., its B/C rows at
+ * Bm + bc_row[c]*L*N, its parameters at A_log + c*N, D[c], dt_bias[c],
+ * conv_w + c*K, conv_b[c].  Optional per-channel state in/out follows the same
+ * c-major layout.  NULL optional arrays mean "absent".
+ */
+void s6o_scan_channels(int64_t n_ch, int64_t L, int N, int K, int zoh,
+                       const double *x, const double *dt_raw, const double *z,
+                       const double *Bm, const double *Cm, const int64_t *bc_row,
+                       const double *A_log, const double *D, const double *dt_bias,
+                       const double *conv_w, const double *conv_b,
+                       const double *hist_in, const double *h_in,
+                       double *y, double *h_out, double *hist_out)
+{
+    int km1 = K > 1 ? K - 1 : 0;
+    for (int64_t c = 0; c < n_ch; ++c) {
+        s6o_scan_channel(L, N, K, zoh,
+                         x + c * L, dt_raw + c * L, z ? z + c * L : NULL,
+                         Bm + bc_row[c] * L * N, Cm + bc_row[c] * L * N,
+                         A_log + c * N, D[c], dt_bias ? dt_bias[c] : 0.0,
+                         K > 0 ? conv_w + c * K : NULL, (K > 0 && conv_b) ? conv_b[c] : 0.0,
+                         hist_in ? hist_in + c * km1 : NULL, h_in ? h_in + c * N : NULL,
+                         y + c * L, h_out ? h_out + c * N : NULL,
+                         hist_out ? hist_out + c * km1 : NULL, NULL, NULL);
+    }
+}
+
+/* Standalone conv + SiLU over many channels: xc[c*L + t]. */
+void s6o_conv_silu_channels(int64_t n_ch, int64_t L, int K, const double *x,
+                            const double *conv_w, const double *conv_b, double *xc)
+{
+    for (int64_t c = 0; c < n_ch; ++c) {
+        double hist[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int64_t t = 0; t < L; ++t) {
+            double pre = s6o_conv_pre(K, conv_w + c * K, conv_b ? conv_b[c] : 0.0, hist, x[c * L + t]);
+            for (int k = 0; k + 1 < K - 1; ++k)
+                hist[k] = hist[k + 1];
+            if (K > 1)
+                hist[K - 2] = x[c * L + t];
+            xc[c * L + t] = s6o_silu(pre);
+        }
+    }
+}
+
+/* Streaming state size of a block stack: channels x states x blocks
+ * ("mamba, live": 1,536 x 16 x 6 = 147,456; the TinyMamba example: 8 x 3 = 24). */
+int64_t s6o_ssm_state_values(int64_t d_inner, int64_t d_state, int64_t blocks)
+{
+    return d_inner * d_state * blocks;
+}
+
+/* Conv history values: K-1 past inputs per channel (TinyMamba: 8 x 2 = 16). */
+int64_t s6o_conv_history_values(int64_t d_inner, int64_t K, int64_t blocks)
+{
+    return d_inner * (K - 1) * blocks;
+}

@@ -1,0 +1,99 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a temporary copy of oracle/s6_oracle.c (on the
+CPU, never in the CUDA path), builds it, routes the oracle through it, and
+checks that at least one pin of test_oracle_pins.py now fails.
+"""
+import os
+import subprocess
+
+import pytest
+
+from oracle import s6_oracle as O
+import test_oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(O.__file__), "s6_oracle.c")
+
+ALL_PINS = [
+    P.test_recorded_decays_exact,
+    P.test_recorded_decays_in_unit_interval,
+    P.test_recorded_first_state_equals_first_write,
+    P.test_recorded_update_rule_exact,
+    P.test_recorded_changed_token_carries_through_decay_only,
+    P.test_state_sizes,
+    lambda: [P.test_softplus_against_libm(v) for v in (-7.0, -1e-3, 0.5, 21.0)],
+    P.test_softplus_zero_is_ln2,
+    lambda: [P.test_silu_against_libm(v) for v in (-10.0, 0.7, 5.0)],
+    P.test_A_is_negative_exp,
+    P.test_zoh_gain_tends_to_delta,
+    P.test_geometric_series_simplified,
+    P.test_zoh_matches_continuous_time_solution,
+    lambda: P.test_bruteforce_decayed_sum(False),
+    lambda: P.test_bruteforce_decayed_sum(True),
+    P.test_readout_uses_updated_state,
+    P.test_conv_onehot_taps_shift,
+    P.test_conv_against_numpy_convolve,
+    P.test_D_multiplies_conv_output_and_gate,
+    P.test_future_changes_leave_past_unchanged,
+    P.test_conv_window_width3,
+    lambda: P.test_streaming_equals_full_forward(True),
+]
+
+MUTATIONS = {
+    "decay_sign": ("return exp(delta * s6o_A(A_log));", "return exp(-delta * s6o_A(A_log));"),
+    "A_not_exp": ("double s6o_A(double A_log) { return -exp(A_log); }",
+                  "double s6o_A(double A_log) { return -A_log; }"),
+    "update_minus": ("return a_bar * h + write;", "return a_bar * h - write;"),
+    "update_no_decay": ("return a_bar * h + write;", "return h + write;"),
+    "zoh_missing_minus_one": ("return expm1(delta * A) / A;", "return exp(delta * A) / A;"),
+    "zoh_missing_div_A": ("return expm1(delta * A) / A;", "return -expm1(delta * A);"),
+    "zoh_as_simplified": ("    if (!zoh)\n        return delta;", "    if (zoh >= 0)\n        return delta;"),
+    "readout_old_state": ("            h[n] = s6o_update(h[n], a_bar, write);\n            acc += h[n] * Cm[t * N + n];",
+                          "            acc += h[n] * Cm[t * N + n];\n            h[n] = s6o_update(h[n], a_bar, write);"),
+    "C_index_transposed": ("acc += h[n] * Cm[t * N + n];", "acc += h[n] * Cm[n * N + t % N];"),
+    "B_is_C": ("* Bm[t * N + n] * u;", "* Cm[t * N + n] * u;"),
+    "D_on_preconv": ("double out = acc + D * u;", "double out = acc + D * x[t];"),
+    "no_gate_silu": ("out *= s6o_silu(z[t]);", "out *= z[t];"),
+    "no_dt_bias": ("s6o_softplus(dt_raw[t] + dt_bias);", "s6o_softplus(dt_raw[t]);"),
+    "softplus_drop_max": ("return m + log1p(exp(-fabs(v)));", "return log1p(exp(-fabs(v)));"),
+    "silu_is_sigmoid": ("return v / (1.0 + exp(-v));", "return 1.0 / (1.0 + exp(-v));"),
+    "conv_taps_reversed": ("acc += w[k] * hist[k];", "acc += w[K - 2 - k] * hist[k];"),
+    "conv_no_bias": ("double acc = bias;", "double acc = 0.0 * bias;"),
+    "conv_history_not_shifted": ("hist[k] = hist[k + 1];", "hist[k] = hist[k];"),
+    "state_count_wrong": ("return d_inner * d_state * blocks;", "return d_inner * d_state;"),
+}
+
+
+def _build_mutant(tmp_path, name):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, name
+    src = src.replace(old, new)
+    c = tmp_path / f"{name}.c"
+    so = tmp_path / f"lib_{name}.so"
+    c.write_text(src)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", str(so), str(c), "-lm"])
+    return str(so)
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(tmp_path, name):
+    so = _build_mutant(tmp_path, name)
+    failed = []
+    with O.use_library(so):
+        for pin in ALL_PINS:
+            try:
+                pin()
+            except AssertionError:
+                failed.append(pin)
+    assert failed, f"no pin caught mutation {name}"
+
+
+def test_unmutated_copy_passes_all(tmp_path):
+    c = tmp_path / "same.c"
+    so = tmp_path / "lib_same.so"
+    c.write_text(open(SRC).read())
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", str(so), str(c), "-lm"])
+    with O.use_library(str(so)):
+        for pin in ALL_PINS:
+            pin()
