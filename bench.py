@@ -1,0 +1,490 @@
+"""Throughput of the S6 selective scan on B200 -- one JSON line on rank 0.
+
+A step is one pass of the hot path over one batch: the fused causal conv4 +
+SiLU + selective scan + SiLU(z) gate + h_final of the long-sequence workload
+(Bt16 L8192 d1536 N16, bf16 I/O, float32 state, simplified dt*B write), i.e.
+one s6_conv_scan_fwd launch over 201M (b, t, channel) elements.  Inputs
+(1.2 GB per step) are larger than L2, so no flush is needed between steps.
+
+metric: Gelem/s = Bt*L*d_inner / time.  value: whole job (all ranks).
+Also reported: the roofline of the dominant kernel (MUFU ex2: N = 16
+exponentials per element; HBM alongside), the oracle on the host cores
+(cpu_baseline), the same metric end to end from pinned host buffers (e2e), and
+the other rows of the path -- the streaming-decode step and the standalone conv.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: torchrun ... bench.py --gpus N; each rank scans its own batch (weak
+scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import s6_inputs as SI  # noqa: E402
+
+METRIC = "selective-scan Gelem/s (B·L·d_inner) and % of HBM/MUFU-ex2 roofline"
+WORKLOAD = "long_seq"
+SMS = 148
+MUFU_PER_SM_CLK = 16  # ex2 results per SM per clock (special-function unit)
+HBM_FALLBACK_GBS = 6650.0
+
+
+def peaks():
+    p = {"hbm_gbs": HBM_FALLBACK_GBS, "sm_max_mhz": 1965.0, "source": "fallback"}
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        p.update(hbm_gbs=float(m["hbm_gbs"]), sm_max_mhz=float(m.get("sm_max_mhz", 1965.0)), source="measured")
+    return p
+
+
+def algorithmic_bytes_per_elem(cfg, gate=True):
+    """x, dt, z read + y written per element, B and C rows per token shared by d channels."""
+    s = 2 if cfg["io"] == "bf16" else 4
+    per = (3 if gate else 2) * s + s
+    return per + 2 * cfg["N"] * s / cfg["d"]
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons in the background."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.rows = []
+        self.proc = None
+        self.gpu = gpu_index
+        self.period = period_ms
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        self.t0 = time.time()
+        return self
+
+    def mark(self):
+        return time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples (nvidia-smi unavailable)"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        loaded = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded or sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows), "samples_under_load": len(loaded)}
+
+
+# ------------------------------------------------------------------ helpers
+def to_dev(a, device):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(a).to(device)
+
+
+def to_pinned(a):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(a)
+    return t.pin_memory()
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for f in ("s6_common.cuh", "s6_scan.cuh"):
+        with open(os.path.join(ROOT, "selective_state_space_19_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the scan kernel from the committed ncu summary, if it
+    was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "s6_conv_scan_long_seq.md")
+    if not os.path.exists(path):
+        return None, None
+    txt = open(path).read()
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    m_b = re.search(r"dram_bytes_per_full_launch:\s*([0-9.eE+]+)", txt)
+    if not (m_sha and m_b) or m_sha.group(1) != kernel_source_sha():
+        return None, (m_sha.group(1) if m_sha else None)
+    return float(m_b.group(1)), m_sha.group(1)
+
+
+# ------------------------------------------------------------------ oracle leg
+class OracleLeg:
+    """The float64 oracle timed on the host cores over a bounded sample of the
+    workload: n (b, channel) pairs, each over the whole sequence."""
+
+    def __init__(self, inp, zoh, threads=None):
+        self.inp, self.zoh = inp, zoh
+        self.cores = threads or os.cpu_count() or 1
+        self.rng = np.random.default_rng(99)
+
+    def run(self, n_ch, Lc=None):
+        from oracle import s6_oracle as O
+        inp = self.inp
+        Lc = Lc or inp["L"]
+        ch = np.stack([self.rng.integers(0, inp["Bt"], n_ch), self.rng.integers(0, inp["d"], n_ch)], axis=1)
+        sub = {k: inp[k][:, :Lc] for k in ("x", "dt", "z", "B", "C")}
+        t0 = time.perf_counter()
+        O.scan(sub["x"], sub["dt"], inp["A_log"], sub["B"], sub["C"], inp["D"], z=sub["z"], dt_bias=inp["dt_bias"],
+               zoh=self.zoh, conv_w=inp["conv_w"], conv_b=inp["conv_b"], channels=ch, threads=self.cores)
+        return n_ch * Lc / (time.perf_counter() - t0)
+
+    def size_for(self, budget_s):
+        """Channels per sample for about budget_s seconds of oracle work."""
+        L = self.inp["L"]
+        rate = self.run(self.cores, min(L, 1024))
+        n = int(rate * budget_s / L)
+        n = max(self.cores, min(self.inp["Bt"] * self.inp["d"], n))
+        return max(self.cores, (n // self.cores) * self.cores)
+
+    def describe(self, n_ch):
+        L = self.inp["L"]
+        return (f"{n_ch} (b, channel) pairs x all {L} tokens of {WORKLOAD} ({n_ch * L / 1e6:.1f}M elements; "
+                f"float64 C loop, {self.cores} threads)")
+
+
+def oracle_rate(inp, zoh, budget_s, threads=None):
+    leg = OracleLeg(inp, zoh, threads)
+    n = leg.size_for(budget_s)
+    return leg.run(n) / 1e9, leg.cores, leg.describe(n)
+
+
+# ------------------------------------------------------------------ rows
+def time_events(fn, iters, stream):
+    import torch
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(iters):
+        fn()
+    e.record(stream)
+    e.synchronize()
+    return s.elapsed_time(e) / iters
+
+
+def row_decode(device, stream, pk, steps=96, pool=8):
+    """Streaming decode: 256 sequences x 6 blocks x d1536 x N16 (147,456 state
+    values per sequence), one token per step per block, fp32 state, in place."""
+    import torch
+    import selective_state_space_19_b200 as S
+    Bt, d, N, K, blocks = 256, 1536, 16, 4, 6
+    params = [{k: to_dev(v, device) for k, v in SI.decode_params(b).items()} for b in range(blocks)]
+    h = [torch.zeros(Bt, d, N, device=device) for _ in range(blocks)]
+    cs = [torch.zeros(Bt, d, K - 1, device=device) for _ in range(blocks)]
+    toks = [[{k: to_dev(v, device) for k, v in SI.decode_tokens(s, b).items()} for b in range(blocks)]
+            for s in range(pool)]
+    ys = [torch.empty(Bt, d, device=device) for _ in range(blocks)]
+
+    def one_cycle():
+        for s in range(pool):
+            for b in range(blocks):
+                p, t = params[b], toks[s][b]
+                S.s6_step(t["x"], t["dt"], t["B"], t["C"], p["A_log"], p["D"], p["conv_w"], h[b], cs[b], z_t=t["z"],
+                          dt_bias=p["dt_bias"], conv_b=p["conv_b"], y_t=ys[b], stream=stream)
+
+    with torch.cuda.stream(stream):
+        one_cycle()  # warm-up outside capture
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            one_cycle()
+        g.replay()
+        torch.cuda.synchronize(device)
+        reps = max(1, steps // pool)
+        ms = time_events(g.replay, reps, stream)
+    n_tok = pool * blocks  # launches per replay
+    elems = n_tok * Bt * d
+    per_launch_ms = ms / n_tok
+    bytes_per = 2 * (N * 4) + 2 * (K - 1) * 4 + 4 * 4 + 2 * N * 4 / d  # h r+w, conv r+w, x/dt/z/y, B/C
+    gbs = elems * bytes_per / (ms * 1e-3) / 1e9
+    return {"workload": "decode: 256 seq x 6 blocks x d1536 x N16, K4, fp32, 1 token/step (CUDA graph of "
+                        f"{n_tok} launches, {pool}-step input pool cycled)",
+            "value": elems / (ms * 1e-3) / 1e9, "unit": "Gelem/s", "us_per_launch": per_launch_ms * 1e3,
+            "us_per_token_all_blocks": per_launch_ms * 1e3 * blocks,
+            "tokens_per_s_all_256_seqs": Bt / (per_launch_ms * 1e-3 * blocks),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "algorithmic_bytes_per_elem": bytes_per}}
+
+
+def row_conv(device, stream, pk, inp_dev, cfg, iters=20):
+    import selective_state_space_19_b200 as S
+    import torch
+    x, w, b = inp_dev["x"], inp_dev["conv_w"], inp_dev["conv_b"]
+    out = torch.empty_like(x)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            S.causal_conv1d_silu_fwd(x, w, b, out=out, stream=stream)
+        ms = time_events(lambda: S.causal_conv1d_silu_fwd(x, w, b, out=out, stream=stream), iters, stream)
+    elems = cfg["Bt"] * cfg["L"] * cfg["d"]
+    s = 2 if cfg["io"] == "bf16" else 4
+    gbs = elems * 2 * s / (ms * 1e-3) / 1e9
+    return {"workload": f"standalone conv4+SiLU on {WORKLOAD} x (Bt16 L8192 d1536 bf16)",
+            "value": elems / (ms * 1e-3) / 1e9, "unit": "Gelem/s", "ms_per_launch": ms,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "algorithmic_bytes_per_elem": 2 * s}}
+
+
+# ------------------------------------------------------------------ main arms
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(v, world, device):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = SI.CONFIGS[WORKLOAD]
+    inp = SI.scan_inputs(WORKLOAD)
+    # each step: one bounded sample, sized so that the whole run stays within a few minutes
+    leg = OracleLeg(inp, False)
+    budget = min(args.ref_step_seconds, max(0.2, 150.0 / (args.steps + args.warmup)))
+    n = leg.size_for(budget)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        g = leg.run(n) / 1e9
+        if i >= args.warmup:
+            per_step.append(g)
+    value = statistics.median(per_step)
+    cores, desc = leg.cores, leg.describe(n)
+    elems = cfg["Bt"] * cfg["L"] * cfg["d"]
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": elems / (value * 1e9) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded numpy, long_seq recipe)",
+            "config": {"workload": f"{WORKLOAD}: Bt16 L8192 d1536 N16 K4, bf16 inputs, simplified write, "
+                                   "fused conv4+SiLU and SiLU(z) gate, h_final",
+                       "global_batch": cfg["Bt"], "seq_len": cfg["L"], "parallelism": "oracle on host cores",
+                       "l2": "n/a (host)"},
+            "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import selective_state_space_19_b200 as S
+
+    world, rank, local = dist_setup(args.gpus)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    S.lib()
+    pk = peaks()
+    cfg = dict(SI.CONFIGS[WORKLOAD])
+    if args.case == "small":
+        # profiling case: same kernel and distributions, 2 of the 16 sequences
+        # (25M elements, ~150 MB of inputs: still larger than L2)
+        cfg.update(Bt=2)
+        args.no_rows = args.no_e2e = args.no_cpu_baseline = True
+    zoh = bool(cfg["zoh"])
+    over = {k: cfg[k] for k in ("Bt",)}
+    inp = SI.scan_inputs(WORKLOAD, seed=cfg["seed"] + rank, **over)  # each rank its own batch (weak scaling)
+    Bt, L, d, N = cfg["Bt"], cfg["L"], cfg["d"], cfg["N"]
+    elems = Bt * L * d
+    stream = torch.cuda.Stream(device)
+    keys = ("x", "z", "B", "C", "dt", "A_log", "D", "dt_bias", "conv_w", "conv_b")
+    t = {k: to_dev(inp[k], device) for k in keys}
+    y = torch.empty_like(t["x"])
+    h = torch.empty(Bt, d, N, device=device)
+
+    def step():
+        S.s6_conv_scan_fwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"], z=t["z"],
+                           dt_bias=t["dt_bias"], zoh_mode=int(zoh), y=y, h_final=h, stream=stream)
+
+    clocks = ClockSampler(local).start()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize(device)
+        barrier(world)
+        torch.cuda.synchronize(device)
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        t_all0 = torch.cuda.Event(enable_timing=True)
+        t_all1 = torch.cuda.Event(enable_timing=True)
+        t_all0.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t_all1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(world)
+        torch.cuda.synchronize(device)
+    clocks.stop()
+    assert S.s6_device_status(stream=stream, device=device) == 0
+    total_ms = t_all0.elapsed_time(t_all1)
+    launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = max_over_ranks(total_ms, world, device)
+    ms_per_step = total_ms / args.steps
+    value = world * elems / (ms_per_step * 1e-3) / 1e9
+
+    # roofline of the scan kernel: N exponentials per element on the MUFU pipe
+    ex2_per_s = elems * N / (launch_ms * 1e-3)
+    ck = clocks.summary()
+    peak_ex2 = SMS * MUFU_PER_SM_CLK * pk["sm_max_mhz"] * 1e6
+    bpe = algorithmic_bytes_per_elem(cfg)
+    gbs = elems * bpe / (launch_ms * 1e-3) / 1e9
+    traffic, _ = recorded_traffic()
+    roof = {"bound": "alu", "unit": "Tex2/s", "achieved": ex2_per_s / 1e12, "peak": peak_ex2 / 1e12,
+            "frac": ex2_per_s / peak_ex2, "traffic": traffic,
+            "pipe": "MUFU ex2 (148 SMs x 16/clk x max SM clock)",
+            "peak_at_measured_clock": (SMS * MUFU_PER_SM_CLK * ck["sm_mhz"] * 1e6 / 1e12) if ck.get("sm_mhz") else None,
+            "algorithmic_ex2_per_elem": N, "kernel": "s6_scan_kernel<bf16,16,32,3,conv,simplified>",
+            "kernel_source_sha": kernel_source_sha(),
+            "hbm": {"achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                    "algorithmic_bytes_per_elem": bpe, "peak_source": pk["source"]}}
+
+    # ---- end to end: pinned host buffers -> device -> kernel -> host, every step
+    e2e = None
+    if not args.no_e2e:
+        hin = {k: to_pinned(inp[k]) for k in ("x", "z", "B", "C", "dt")}
+        hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        hh = torch.empty(h.shape, dtype=h.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in hin.values())
+        d2h = hy.numel() * hy.element_size() + hh.numel() * hh.element_size()
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            for k, v in hin.items():
+                t[k].copy_(v, non_blocking=True)
+            step()
+            hy.copy_(y, non_blocking=True)
+            hh.copy_(h, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+            torch.cuda.synchronize(device)
+            barrier(world)
+            e_ms = time_events(e2e_step, e2e_steps, stream)
+            barrier(world)
+        e_ms = max_over_ranks(e_ms, world, device)
+        e2e = {"value": world * elems / (e_ms * 1e-3) / 1e9, "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms, "steps": e2e_steps}
+
+    rows = {}
+    if not args.no_rows and rank == 0:
+        rows["s6_step"] = row_decode(device, stream, pk)
+        rows["causal_conv1d_silu_fwd"] = row_conv(device, stream, pk, t, cfg)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        g, cores, desc = oracle_rate(inp, zoh, budget_s=args.cpu_seconds)
+        cpu = {"value": g, "unit": "Gelem/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
+                "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16 I/O, f32 math and state",
+                "data": "synthetic (seeded numpy, long_seq recipe: x,z,B,C ~ N(0,1), dt_raw ~ 0.5 N(0,1), "
+                        "dt_bias = softplus^-1(U[0.001,0.1]), A_log = log(n+1), D ~ U[0.5,1.5])",
+                "config": {"workload": f"{WORKLOAD}: Bt16 L8192 d1536 N16 K4, bf16 I/O, fp32 state, simplified "
+                                       "dt*B write, fused conv4+SiLU + SiLU(z) gate, h_final",
+                           "global_batch": Bt * world, "seq_len": L, "d_inner": d, "d_state": N,
+                           "parallelism": f"dp{world} (independent batches per GPU)",
+                           "l2": "inputs larger than L2 (1.2 GB read per step), no flush"},
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+                "clocks": {"sm_mhz": ck.get("sm_mhz"), "sm_max_mhz": ck.get("sm_max_mhz"), "reasons": ck.get("reasons"),
+                           "samples": ck.get("samples")},
+                "rows": rows}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--case", choices=["full", "small"], default="full",
+                    help="small: 2 sequences of the workload only (for ncu captures)")
+    ap.add_argument("--no-rows", action="store_true", help="skip the decode-step and standalone-conv rows")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

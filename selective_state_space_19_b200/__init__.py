@@ -1,0 +1,216 @@
+"""B200 (sm_100a) selective scan (Mamba S6) -- Python binding of libs6_b200.so.
+
+This module only marshals arguments: it checks dtype / device / contiguity of
+torch tensors, allocates outputs with torch when the caller passes none, and
+hands raw device pointers plus the current CUDA stream to the C ABI declared in
+``include/s6.h``.  Every arithmetic step runs in the library's CUDA kernels.
+There is no CPU fallback: if the library is missing, the first call raises.
+
+Functions (same names as the C ABI):
+    s6_scan_fwd, s6_conv_scan_fwd, causal_conv1d_silu_fwd, s6_step,
+    s6_device_status, s6_status_string, s6_version
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "S6Error", "lib", "s6_scan_fwd", "s6_conv_scan_fwd", "causal_conv1d_silu_fwd", "s6_step",
+    "s6_device_status", "s6_status_string", "s6_version", "S6_F32", "S6_BF16", "Dims",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libs6_b200.so")
+
+S6_F32, S6_BF16 = 0, 1
+S6_OK, S6_ERR_INVALID_ARG, S6_ERR_UNSUPPORTED, S6_ERR_ALIGNMENT, S6_ERR_CUDA, S6_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+
+
+class Dims(ctypes.Structure):
+    """Mirror of ``s6_dims``."""
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("d_inner", ctypes.c_int64),
+                ("d_state", ctypes.c_int64), ("conv_width", ctypes.c_int64), ("io_dtype", ctypes.c_int32)]
+
+
+class S6Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {s6_status_string(status)} ({status})")
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library {LIB_PATH} is missing: build it with `python -m selective_state_space_19_b200._build`"
+                " (or __graft_entry__.build()); there is no CPU fallback")
+        L = ctypes.CDLL(LIB_PATH)
+        DP = ctypes.POINTER(Dims)
+        L.s6_scan_fwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P]
+        L.s6_conv_scan_fwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P]
+        L.causal_conv1d_silu_fwd.argtypes = [DP, _P, _P, _P, _P, _P]
+        L.s6_step.argtypes = [DP, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.s6_device_status.argtypes = [_P]
+        L.s6_status_string.argtypes = [_I]
+        L.s6_status_string.restype = ctypes.c_char_p
+        L.s6_version.argtypes = []
+        for f in (L.s6_scan_fwd, L.s6_conv_scan_fwd, L.causal_conv1d_silu_fwd, L.s6_step, L.s6_device_status,
+                  L.s6_version):
+            f.restype = _I
+        _lib = L
+    return _lib
+
+
+def s6_status_string(status: int) -> str:
+    return lib().s6_status_string(int(status)).decode()
+
+
+def s6_version() -> int:
+    return lib().s6_version()
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _io_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return S6_F32
+    if t.dtype == torch.bfloat16:
+        return S6_BF16
+    raise TypeError(f"I/O tensors must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t, name, dtype=None, shape=None, device=None):
+    if t is None:
+        return None
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t.data_ptr()
+
+
+def _stream(stream, device):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status, where):
+    if status != S6_OK:
+        raise S6Error(status, where)
+
+
+def _scan(fn, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w, conv_b, want_h, stream):
+    torch = _torch()
+    if x.dim() != 3:
+        raise ValueError("x/u must be [batch, seqlen, d_inner]")
+    Bt, L, d = x.shape
+    io = _io_code(x)
+    N = A_log.shape[-1]
+    dev = x.device
+    f32 = torch.float32
+    K = conv_w.shape[-1] if conv_w is not None else 0
+    if y is None:
+        y = torch.empty_like(x)
+    if h_final is None and want_h:
+        h_final = torch.empty((Bt, d, N), dtype=f32, device=dev)
+    dims = Dims(Bt, L, d, N, K, io)
+    args = [ctypes.byref(dims)]
+    seq = (Bt, L, d)
+    xp = _ptr(x, "x", x.dtype, seq, dev)
+    if conv_w is not None:
+        args += [xp, _ptr(conv_w, "conv_w", f32, (d, K), dev), _ptr(conv_b, "conv_b", f32, (d,), dev)]
+    else:
+        args += [xp]
+    args += [_ptr(dt, "dt", x.dtype, seq, dev), _ptr(A_log, "A_log", f32, (d, N), dev),
+             _ptr(B, "B", x.dtype, (Bt, L, N), dev), _ptr(C, "C", x.dtype, (Bt, L, N), dev),
+             _ptr(D, "D", f32, (d,), dev), _ptr(z, "z", x.dtype, seq, dev),
+             _ptr(dt_bias, "dt_bias", f32, (d,), dev), int(zoh_mode), _ptr(y, "y", x.dtype, seq, dev),
+             _ptr(h_final, "h_final", f32, (Bt, d, N), dev), _stream(stream, dev)]
+    _check(fn(*args), fn.__name__)
+    return y, h_final
+
+
+def s6_scan_fwd(u, dt, A_log, B, C, D, z=None, dt_bias=None, zoh_mode=0, y=None, h_final=None,
+                want_h_final=True, stream=None):
+    """Selective scan of an already-convolved input u.  Returns (y, h_final)."""
+    return _scan(lib().s6_scan_fwd, u, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, None, None,
+                 want_h_final, stream)
+
+
+def s6_conv_scan_fwd(x, conv_w, conv_b, dt, A_log, B, C, D, z=None, dt_bias=None, zoh_mode=0, y=None,
+                     h_final=None, want_h_final=True, stream=None):
+    """Fused causal conv + SiLU + selective scan + gate.  Returns (y, h_final)."""
+    return _scan(lib().s6_conv_scan_fwd, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w,
+                 conv_b, want_h_final, stream)
+
+
+def causal_conv1d_silu_fwd(x, conv_w, conv_b=None, out=None, stream=None):
+    """SiLU(causal depthwise conv(x)) over [batch, seqlen, d_inner]."""
+    torch = _torch()
+    Bt, L, d = x.shape
+    K = conv_w.shape[-1]
+    if out is None:
+        out = torch.empty_like(x)
+    dims = Dims(Bt, L, d, 1, K, _io_code(x))
+    dev = x.device
+    st = lib().causal_conv1d_silu_fwd(ctypes.byref(dims), _ptr(x, "x", x.dtype, (Bt, L, d), dev),
+                                      _ptr(conv_w, "conv_w", torch.float32, (d, K), dev),
+                                      _ptr(conv_b, "conv_b", torch.float32, (d,), dev),
+                                      _ptr(out, "out", x.dtype, (Bt, L, d), dev), _stream(stream, dev))
+    _check(st, "causal_conv1d_silu_fwd")
+    return out
+
+
+def s6_step(u_t, dt_t, B_t, C_t, A_log, D, conv_w, h_ssm, conv_state, z_t=None, dt_bias=None, conv_b=None,
+            zoh_mode=0, y_t=None, stream=None):
+    """One streaming token for a batch of sequences; h_ssm and conv_state are updated in place."""
+    torch = _torch()
+    Bt, d = u_t.shape
+    N = A_log.shape[-1]
+    K = conv_w.shape[-1]
+    io = _io_code(u_t)
+    dev = u_t.device
+    if y_t is None:
+        y_t = torch.empty_like(u_t)
+    f32 = torch.float32
+    dims = Dims(Bt, 1, d, N, K, io)
+    st = lib().s6_step(ctypes.byref(dims), _ptr(A_log, "A_log", f32, (d, N), dev), _ptr(D, "D", f32, (d,), dev),
+                       _ptr(dt_bias, "dt_bias", f32, (d,), dev), _ptr(conv_w, "conv_w", f32, (d, K), dev),
+                       _ptr(conv_b, "conv_b", f32, (d,), dev), int(zoh_mode),
+                       _ptr(u_t, "u_t", u_t.dtype, (Bt, d), dev), _ptr(dt_t, "dt_t", u_t.dtype, (Bt, d), dev),
+                       _ptr(B_t, "B_t", u_t.dtype, (Bt, N), dev), _ptr(C_t, "C_t", u_t.dtype, (Bt, N), dev),
+                       _ptr(z_t, "z_t", u_t.dtype, (Bt, d), dev), _ptr(h_ssm, "h_ssm", f32, (Bt, d, N), dev),
+                       _ptr(conv_state, "conv_state", u_t.dtype, (Bt, d, K - 1), dev),
+                       _ptr(y_t, "y_t", u_t.dtype, (Bt, d), dev), _stream(stream, dev))
+    _check(st, "s6_step")
+    return y_t
+
+
+def s6_device_status(stream=None, device=None) -> int:
+    """Synchronise and return (and clear) the library's device-side error status."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return lib().s6_device_status(_stream(stream, dev))

@@ -1,0 +1,359 @@
+// s6_abi.cu -- the C ABI declared in include/s6.h: argument checks, tensor-map
+// set-up, kernel selection and launch.  Every arithmetic step of the path runs
+// in the kernels of s6_scan.cuh, s6_conv.cuh and s6_step.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "s6.h"
+#include "s6_common.cuh"
+#include "s6_conv.cuh"
+#include "s6_scan.cuh"
+#include "s6_step.cuh"
+
+namespace {
+
+using s6::ScanArgs;
+
+constexpr int kMaxState = 16;
+
+// ------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D map over a [Bt, L, d] row-major tensor (dims innermost first: d, L, Bt)
+// with a box of [1, rows, cols] elements.
+bool make_map_3d(CUtensorMap *map, const void *base, int io, int64_t Bt, int64_t L, int64_t d, int box_cols,
+                 int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const size_t es = io == S6_BF16 ? 2 : 4;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(Bt)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d * es), static_cast<cuuint64_t>(L * d * es)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, io == S6_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                    const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t io_size(int io) { return io == S6_BF16 ? 2 : 4; }
+
+// ------------------------------------------------------------ validation
+int check_dims(const s6_dims *dims, bool need_L, bool need_K) {
+    if (!dims)
+        return S6_ERR_INVALID_ARG;
+    if (dims->batch < 0 || dims->seqlen < 0 || dims->d_inner < 1 || dims->d_state < 1)
+        return S6_ERR_INVALID_ARG;
+    if (dims->io_dtype != S6_F32 && dims->io_dtype != S6_BF16)
+        return S6_ERR_UNSUPPORTED;
+    if (dims->d_state > kMaxState)
+        return S6_ERR_UNSUPPORTED;
+    if (need_K && (dims->conv_width < 2 || dims->conv_width > 4))
+        return S6_ERR_UNSUPPORTED;
+    // 32-bit index arithmetic inside the kernels (per-sequence offsets stay 64-bit)
+    if (dims->d_inner > (1 << 30) || dims->batch > (1 << 30) || (need_L && dims->seqlen > (1 << 30)))
+        return S6_ERR_UNSUPPORTED;
+    return S6_OK;
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? S6_OK : S6_ERR_CUDA; }
+
+// Make the device that owns `stream` current for this library's runtime before
+// any launch (the caller's framework may have selected it through another
+// runtime instance in the same process).  The legacy and per-thread default
+// streams keep the current device.
+int use_stream_device(cudaStream_t stream) {
+    if (stream == nullptr || stream == cudaStreamLegacy || stream == cudaStreamPerThread)
+        return S6_OK;
+    int dev = -1, cur = -1;
+    if (cudaStreamGetDevice(stream, &dev) != cudaSuccess || cudaGetDevice(&cur) != cudaSuccess)
+        return S6_ERR_CUDA;
+    if (dev != cur && cudaSetDevice(dev) != cudaSuccess)
+        return S6_ERR_CUDA;
+    return S6_OK;
+}
+
+// ------------------------------------------------------------ scan dispatch
+template <typename IO, int NS, bool CONV, bool ZOH>
+int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, const ScanArgs &a,
+                  cudaStream_t stream) {
+    constexpr int T = sizeof(IO) == 2 ? 32 : 16;
+    constexpr int STAGES = 3;
+    using Smem = s6::ScanSmem<IO, NS, T, STAGES, CONV>;
+    const int io = dims->io_dtype;
+    CUtensorMap tx, tdt, tz, ty;
+    const int xrows = Smem::XR;
+    if (!make_map_3d(&tx, x, io, dims->batch, dims->seqlen, dims->d_inner, s6::kScanThreads, xrows) ||
+        !make_map_3d(&tdt, dt, io, dims->batch, dims->seqlen, dims->d_inner, s6::kScanThreads, T) ||
+        !make_map_3d(&ty, y, io, dims->batch, dims->seqlen, dims->d_inner, s6::kScanThreads, T))
+        return S6_ERR_CUDA;
+    if (z) {
+        if (!make_map_3d(&tz, z, io, dims->batch, dims->seqlen, dims->d_inner, s6::kScanThreads, T))
+            return S6_ERR_CUDA;
+    } else {
+        tz = tdt;  // never read when has_z == 0
+    }
+    auto kern = s6::s6_scan_kernel<IO, NS, T, STAGES, CONV, ZOH>;
+    const size_t smem = sizeof(Smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess)
+        return S6_ERR_CUDA;
+    dim3 grid(static_cast<unsigned>((dims->d_inner + s6::kScanThreads - 1) / s6::kScanThreads),
+              static_cast<unsigned>(dims->batch));
+    kern<<<grid, s6::kScanThreads, smem, stream>>>(tx, tdt, tz, ty, a);
+    return launch_status(cudaGetLastError());
+}
+
+template <typename IO, bool CONV, bool ZOH>
+int launch_scan_n(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, const ScanArgs &a,
+                  cudaStream_t st) {
+    if (dims->d_state <= 4)
+        return launch_scan_t<IO, 4, CONV, ZOH>(dims, x, dt, z, y, a, st);
+    if (dims->d_state <= 8)
+        return launch_scan_t<IO, 8, CONV, ZOH>(dims, x, dt, z, y, a, st);
+    return launch_scan_t<IO, 16, CONV, ZOH>(dims, x, dt, z, y, a, st);
+}
+
+template <typename IO>
+int launch_scan_io(const s6_dims *dims, bool conv, bool zoh, const void *x, const void *dt, const void *z, void *y,
+                   const ScanArgs &a, cudaStream_t st) {
+    if (conv)
+        return zoh ? launch_scan_n<IO, true, true>(dims, x, dt, z, y, a, st)
+                   : launch_scan_n<IO, true, false>(dims, x, dt, z, y, a, st);
+    return zoh ? launch_scan_n<IO, false, true>(dims, x, dt, z, y, a, st)
+               : launch_scan_n<IO, false, false>(dims, x, dt, z, y, a, st);
+}
+
+int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv_w, const float *conv_b,
+                const void *dt, const float *A_log, const void *B, const void *C, const float *D, const void *z,
+                const float *dt_bias, int zoh_mode, void *y, float *h_final, s6_stream_t stream) {
+    int st = check_dims(dims, true, conv);
+    if (st != S6_OK)
+        return st;
+    if (zoh_mode != 0 && zoh_mode != 1)
+        return S6_ERR_INVALID_ARG;
+    if (dims->batch == 0 || dims->seqlen == 0) {
+        // nothing to scan; h_final of an empty sequence is the zero start state
+        if (h_final && dims->batch > 0) {
+            if (use_stream_device(reinterpret_cast<cudaStream_t>(stream)) != S6_OK)
+                return S6_ERR_CUDA;
+            return launch_status(cudaMemsetAsync(h_final, 0,
+                                                 sizeof(float) * dims->batch * dims->d_inner * dims->d_state,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+        }
+        return S6_OK;
+    }
+    if (!x || !dt || !A_log || !B || !C || !D || !y || (conv && !conv_w))
+        return S6_ERR_INVALID_ARG;
+    const size_t es = io_size(dims->io_dtype);
+    if ((dims->d_inner * es) % 16 != 0)
+        return S6_ERR_ALIGNMENT;
+    const void *ptrs[] = {x, dt, B, C, y, z, A_log, D, dt_bias, conv_w, conv_b, h_final};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return S6_ERR_ALIGNMENT;
+
+    ScanArgs a;
+    a.Bt = static_cast<int>(dims->batch);
+    a.L = static_cast<int>(dims->seqlen);
+    a.d = static_cast<int>(dims->d_inner);
+    a.N = static_cast<int>(dims->d_state);
+    a.has_z = z != nullptr;
+    a.B = B;
+    a.C = C;
+    a.A_log = A_log;
+    a.D = D;
+    a.dt_bias = dt_bias;
+    a.conv_w = conv ? conv_w : nullptr;
+    a.conv_b = conv ? conv_b : nullptr;
+    a.K = conv ? static_cast<int>(dims->conv_width) : 0;
+    a.h_final = h_final;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (use_stream_device(s) != S6_OK)
+        return S6_ERR_CUDA;
+    if (dims->io_dtype == S6_BF16)
+        return launch_scan_io<__nv_bfloat16>(dims, conv, zoh_mode == 1, x, dt, z, y, a, s);
+    return launch_scan_io<float>(dims, conv, zoh_mode == 1, x, dt, z, y, a, s);
+}
+
+// ------------------------------------------------------------ step dispatch
+template <typename IO, int NS, bool ZOH>
+int launch_step_t(const s6::StepArgs &a, cudaStream_t st) {
+    const long long threads = static_cast<long long>(a.Bt) * a.d * (NS / 4);
+    const long long blocks = (threads + s6::kStepThreads - 1) / s6::kStepThreads;
+    if (blocks > 0x7fffffffLL)
+        return S6_ERR_UNSUPPORTED;
+    s6::s6_step_kernel<IO, NS, ZOH><<<static_cast<unsigned>(blocks), s6::kStepThreads, 0, st>>>(a);
+    return launch_status(cudaGetLastError());
+}
+
+template <typename IO, bool ZOH>
+int launch_step_n(const s6::StepArgs &a, cudaStream_t st) {
+    if (a.N <= 4)
+        return launch_step_t<IO, 4, ZOH>(a, st);
+    if (a.N <= 8)
+        return launch_step_t<IO, 8, ZOH>(a, st);
+    return launch_step_t<IO, 16, ZOH>(a, st);
+}
+
+}  // namespace
+
+// ======================================================================= ABI
+extern "C" {
+
+int s6_version(void) { return (1 << 16) | 0; }
+
+const char *s6_status_string(int status) {
+    switch (status) {
+        case S6_OK: return "S6_OK";
+        case S6_ERR_INVALID_ARG: return "S6_ERR_INVALID_ARG: null pointer or invalid size";
+        case S6_ERR_UNSUPPORTED: return "S6_ERR_UNSUPPORTED: size, width or dtype outside the supported range";
+        case S6_ERR_ALIGNMENT: return "S6_ERR_ALIGNMENT: pointer or row not 16-byte aligned";
+        case S6_ERR_CUDA: return "S6_ERR_CUDA: a CUDA call or kernel launch failed";
+        case S6_ERR_TIMEOUT: return "S6_ERR_TIMEOUT: a bounded device-side wait gave up";
+        default: return "S6: unknown status";
+    }
+}
+
+int s6_scan_fwd(const s6_dims *dims, const void *u, const void *dt, const float *A_log, const void *B, const void *C,
+                const float *D, const void *z, const float *dt_bias, int zoh_mode, void *y, float *h_final,
+                s6_stream_t stream) {
+    return scan_common(dims, false, u, nullptr, nullptr, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final,
+                       stream);
+}
+
+int s6_conv_scan_fwd(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b, const void *dt,
+                     const float *A_log, const void *B, const void *C, const float *D, const void *z,
+                     const float *dt_bias, int zoh_mode, void *y, float *h_final, s6_stream_t stream) {
+    return scan_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final,
+                       stream);
+}
+
+int causal_conv1d_silu_fwd(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b, void *out,
+                           s6_stream_t stream) {
+    int st = check_dims(dims, true, true);
+    if (st != S6_OK)
+        return st;
+    if (dims->batch == 0 || dims->seqlen == 0)
+        return S6_OK;
+    if (!x || !conv_w || !out)
+        return S6_ERR_INVALID_ARG;
+    if ((dims->d_inner * io_size(dims->io_dtype)) % 16 != 0)
+        return S6_ERR_ALIGNMENT;
+    if (!aligned16(x) || !aligned16(out) || !aligned16(conv_w) || (conv_b && !aligned16(conv_b)))
+        return S6_ERR_ALIGNMENT;
+    s6::ConvArgs a;
+    a.Bt = static_cast<int>(dims->batch);
+    a.L = static_cast<int>(dims->seqlen);
+    a.d = static_cast<int>(dims->d_inner);
+    a.K = static_cast<int>(dims->conv_width);
+    a.x = x;
+    a.conv_w = conv_w;
+    a.conv_b = conv_b;
+    a.out = out;
+    const int vec = static_cast<int>(16 / io_size(dims->io_dtype));
+    const long long cols = (dims->d_inner + 32LL * vec - 1) / (32LL * vec);
+    const long long rows = (dims->seqlen + 1LL * s6::kConvWarps * s6::kConvRun - 1) / (s6::kConvWarps * s6::kConvRun);
+    if (rows > 65535 || dims->batch > 65535)
+        return S6_ERR_UNSUPPORTED;
+    dim3 grid(static_cast<unsigned>(cols), static_cast<unsigned>(rows), static_cast<unsigned>(dims->batch));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (use_stream_device(s) != S6_OK)
+        return S6_ERR_CUDA;
+    if (dims->io_dtype == S6_BF16)
+        s6::s6_conv_silu_kernel<__nv_bfloat16><<<grid, 32 * s6::kConvWarps, 0, s>>>(a);
+    else
+        s6::s6_conv_silu_kernel<float><<<grid, 32 * s6::kConvWarps, 0, s>>>(a);
+    return launch_status(cudaGetLastError());
+}
+
+int s6_step(const s6_dims *dims, const float *A_log, const float *D, const float *dt_bias, const float *conv_w,
+            const float *conv_b, int zoh_mode, const void *u_t, const void *dt_t, const void *B_t, const void *C_t,
+            const void *z_t, float *h_ssm, void *conv_state, void *y_t, s6_stream_t stream) {
+    int st = check_dims(dims, false, true);
+    if (st != S6_OK)
+        return st;
+    if (zoh_mode != 0 && zoh_mode != 1)
+        return S6_ERR_INVALID_ARG;
+    if (dims->batch == 0)
+        return S6_OK;
+    if (!A_log || !D || !conv_w || !u_t || !dt_t || !B_t || !C_t || !h_ssm || !conv_state || !y_t)
+        return S6_ERR_INVALID_ARG;
+    const void *ptrs[] = {A_log, D, dt_bias, conv_w, conv_b, u_t, dt_t, B_t, C_t, z_t, h_ssm, conv_state, y_t};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p))
+            return S6_ERR_ALIGNMENT;
+    s6::StepArgs a;
+    a.Bt = static_cast<int>(dims->batch);
+    a.d = static_cast<int>(dims->d_inner);
+    a.N = static_cast<int>(dims->d_state);
+    a.K = static_cast<int>(dims->conv_width);
+    a.zoh = zoh_mode;
+    a.has_z = z_t != nullptr;
+    a.A_log = A_log;
+    a.D = D;
+    a.dt_bias = dt_bias;
+    a.conv_w = conv_w;
+    a.conv_b = conv_b;
+    a.u = u_t;
+    a.dt = dt_t;
+    a.B = B_t;
+    a.C = C_t;
+    a.z = z_t;
+    a.h = h_ssm;
+    a.conv_state = conv_state;
+    a.y = y_t;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (use_stream_device(s) != S6_OK)
+        return S6_ERR_CUDA;
+    if (dims->io_dtype == S6_BF16)
+        return zoh_mode ? launch_step_n<__nv_bfloat16, true>(a, s) : launch_step_n<__nv_bfloat16, false>(a, s);
+    return zoh_mode ? launch_step_n<float, true>(a, s) : launch_step_n<float, false>(a, s);
+}
+
+// Read and clear the device-side error word after the stream's work so far
+// (synchronises `stream`).  S6_ERR_TIMEOUT if a bounded wait gave up.
+int s6_device_status(s6_stream_t stream) {
+    unsigned int v = 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (use_stream_device(s) != S6_OK)
+        return S6_ERR_CUDA;
+    if (cudaMemcpyFromSymbolAsync(&v, s6::g_s6_device_error, sizeof(v), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return S6_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return S6_ERR_CUDA;
+    if (v) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbolAsync(s6::g_s6_device_error, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess)
+            return S6_ERR_CUDA;
+        cudaStreamSynchronize(s);
+        return S6_ERR_TIMEOUT;
+    }
+    return S6_OK;
+}
+
+}  // extern "C"

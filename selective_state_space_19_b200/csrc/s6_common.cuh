@@ -1,0 +1,163 @@
+// s6_common.cuh -- device helpers shared by the S6 kernels (sm_100a only).
+//
+// Transcendentals are issued as the MUFU instructions themselves through PTX
+// (ex2.approx / lg2.approx / rcp.approx); every use states the identity it
+// relies on.  Bulk tensor copies (TMA) and their mbarriers are plain PTX as
+// documented for sm_90+/sm_100.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace s6 {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---------------------------------------------------------------- I/O types
+template <typename IO>
+struct io_traits;
+
+template <>
+struct io_traits<float> {
+    static __device__ __forceinline__ float to_f(float v) { return v; }
+    static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+
+template <>
+struct io_traits<__nv_bfloat16> {
+    // bf16 -> f32 is exact: the bf16 bits are the top half of the f32 bits.
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 v) {
+        return __uint_as_float(static_cast<uint32_t>(__bfloat16_as_ushort(v)) << 16);
+    }
+    // f32 -> bf16, round to nearest even (cvt.rn.bf16.f32).
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+
+// ------------------------------------------------------------- MUFU wrappers
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// SiLU(v) = v * sigmoid(v) = v / (1 + 2^(-v log2 e)).  For v -> -inf the
+// power overflows to +inf and the reciprocal to 0, giving -0.
+__device__ __forceinline__ float silu_f(float v) {
+    return v * rcp_approx(1.0f + ex2_approx(-v * kLog2e));
+}
+
+// softplus(v) = log(1 + e^v) = max(v, 0) + log1p(e^-|v|).
+// log1p(e) is formed as log2(1 + e) * ln2, corrected for the rounding of
+// 1 + e by the factor e / ((1 + e) - 1) (the subtraction is exact); when
+// 1 + e rounds to 1, log1p(e) = e to within e^2/2.
+__device__ __forceinline__ float softplus_f(float v) {
+    const float e = ex2_approx(-fabsf(v) * kLog2e);
+    const float u = 1.0f + e;
+    const float um1 = u - 1.0f;
+    float l = lg2_approx(u) * kLn2;
+    l = (um1 == 0.0f) ? e : l * (e * rcp_approx(um1));
+    return fmaxf(v, 0.0f) + l;
+}
+
+// --------------------------------------------------------- mbarrier + TMA
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbarrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false after `limit` polls (each
+// try_wait may itself suspend the thread for a short, hardware-chosen time).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait(bar, parity))
+            return true;
+    return false;
+}
+
+// 3-D tiled bulk tensor load global -> shared, completing on `bar`.
+// Coordinates are element indices, innermost first; out-of-range elements
+// (including negative coordinates of the outer dimensions) are filled with 0.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
+                                            int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// 3-D tiled bulk tensor store shared -> global (out-of-range elements are
+// not written).  Completion is tracked with bulk groups.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (needed before a bulk store reads them).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Device-side error word (one per device image of the library; the library is
+// built as a single translation unit, s6_abi.cu).  Bit 0: a bounded wait gave
+// up.  Read and cleared by the host through s6_device_status.
+__device__ unsigned int g_s6_device_error = 0;
+
+__device__ __forceinline__ void raise_device_error(unsigned int bits) { atomicOr(&g_s6_device_error, bits); }
+
+}  // namespace s6

@@ -1,0 +1,125 @@
+"""CPU-only checks of the boundary: the library builds for sm_100a, loads without
+a GPU, exports every function include/s6.h declares, and rejects bad arguments
+on the host before touching the device.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "s6.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = "\n".join(l for l in src.splitlines() if not l.lstrip().startswith("#"))
+    return re.findall(r"S6_API\s+(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", src)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from selective_state_space_19_b200 import _build
+    import selective_state_space_19_b200 as S
+    _build.build()
+    return S.lib()
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"s6_scan_fwd", "s6_conv_scan_fwd", "causal_conv1d_silu_fwd", "s6_step", "s6_status_string",
+            "s6_device_status", "s6_version"} <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_library_is_built_for_sm100a_only():
+    from selective_state_space_19_b200 import _build
+    flags = " ".join(_build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert "sm_90" not in flags and "sm_80" not in flags
+
+
+def test_status_strings(lib):
+    import selective_state_space_19_b200 as S
+    for st in (S.S6_OK, S.S6_ERR_INVALID_ARG, S.S6_ERR_UNSUPPORTED, S.S6_ERR_ALIGNMENT, S.S6_ERR_CUDA,
+               S.S6_ERR_TIMEOUT):
+        assert S.s6_status_string(st).startswith("S6_")
+    assert "unknown" in S.s6_status_string(12345)
+    assert S.s6_version() >> 16 == 1
+
+
+def _dims(**kw):
+    import selective_state_space_19_b200 as S
+    d = dict(batch=2, seqlen=8, d_inner=64, d_state=16, conv_width=4, io_dtype=0)
+    d.update(kw)
+    return S.Dims(**d)
+
+
+def _call_scan(lib, dims, **ptrs):
+    P = ctypes.c_void_p
+    args = dict(u=16, dt=16, A_log=16, B=16, C=16, D=16, z=None, dt_bias=None, zoh=0, y=16, h=None)
+    args.update(ptrs)
+    return lib.s6_scan_fwd(ctypes.byref(dims) if dims is not None else None, P(args["u"]), P(args["dt"]),
+                           P(args["A_log"]), P(args["B"]), P(args["C"]), P(args["D"]), P(args["z"]),
+                           P(args["dt_bias"]), args["zoh"], P(args["y"]), P(args["h"]), None)
+
+
+def test_host_checks_reject_before_any_launch(lib):
+    import selective_state_space_19_b200 as S
+    assert _call_scan(lib, None) == S.S6_ERR_INVALID_ARG
+    assert _call_scan(lib, _dims(d_state=17)) == S.S6_ERR_UNSUPPORTED
+    assert _call_scan(lib, _dims(d_state=0)) == S.S6_ERR_INVALID_ARG
+    assert _call_scan(lib, _dims(io_dtype=7)) == S.S6_ERR_UNSUPPORTED
+    assert _call_scan(lib, _dims(batch=-1)) == S.S6_ERR_INVALID_ARG
+    assert _call_scan(lib, _dims(), u=None) == S.S6_ERR_INVALID_ARG
+    assert _call_scan(lib, _dims(), zoh=3) == S.S6_ERR_INVALID_ARG
+    assert _call_scan(lib, _dims(d_inner=62)) == S.S6_ERR_ALIGNMENT          # 62*4 B rows
+    assert _call_scan(lib, _dims(d_inner=60, io_dtype=1)) == S.S6_ERR_ALIGNMENT  # 60*2 B rows
+    assert _call_scan(lib, _dims(), dt=24) == S.S6_ERR_ALIGNMENT
+    # empty work is accepted and does nothing (no pointer is touched)
+    assert _call_scan(lib, _dims(batch=0), u=None, dt=None, y=None) == S.S6_OK
+    assert _call_scan(lib, _dims(seqlen=0), u=None, dt=None, y=None) == S.S6_OK
+
+
+def test_conv_and_step_host_checks(lib):
+    import selective_state_space_19_b200 as S
+    P = ctypes.c_void_p
+    d = _dims(conv_width=5)
+    assert lib.causal_conv1d_silu_fwd(ctypes.byref(d), P(16), P(16), None, P(16), None) == S.S6_ERR_UNSUPPORTED
+    d = _dims(conv_width=1)
+    assert lib.causal_conv1d_silu_fwd(ctypes.byref(d), P(16), P(16), None, P(16), None) == S.S6_ERR_UNSUPPORTED
+    d = _dims()
+    assert lib.causal_conv1d_silu_fwd(ctypes.byref(d), None, P(16), None, P(16), None) == S.S6_ERR_INVALID_ARG
+    ok = [P(16)] * 5
+    assert lib.s6_step(ctypes.byref(_dims()), *ok, 0, None, *[P(16)] * 3, None, P(16), P(16), P(16),
+                       None) == S.S6_ERR_INVALID_ARG
+    assert lib.s6_step(ctypes.byref(_dims()), *ok, 2, *[P(16)] * 4, None, P(16), P(16), P(16),
+                       None) == S.S6_ERR_INVALID_ARG
+    assert lib.s6_step(ctypes.byref(_dims(d_state=20)), *ok, 0, *[P(16)] * 4, None, P(16), P(16), P(16),
+                       None) == S.S6_ERR_UNSUPPORTED
+    assert lib.s6_step(ctypes.byref(_dims()), *ok, 0, *[P(16)] * 4, None, P(20), P(16), P(16),
+                       None) == S.S6_ERR_ALIGNMENT
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    import selective_state_space_19_b200 as S
+    x = torch.zeros(1, 4, 8)
+    with pytest.raises(ValueError):
+        S.s6_scan_fwd(x, x, torch.zeros(8, 3), torch.zeros(1, 4, 3), torch.zeros(1, 4, 3), torch.zeros(8))
+
+
+def test_product_path_does_not_use_the_oracle():
+    """The package, its C sources and the header never refer to the oracle."""
+    pkg = os.path.join(ROOT, "selective_state_space_19_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in txt.lower(), f
+    assert "oracle" not in open(HEADER).read().lower()
