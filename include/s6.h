@@ -34,10 +34,13 @@
  *     float32 on the device.
  *  Pointers: DEVICE pointers owned by the caller; the library keeps none of
  *     them after the call returns.  Outputs must not alias inputs.
- *  Alignment: every tensor pointer must be 16-byte aligned, and for the
- *     full-sequence calls d * sizeof(io) must be a multiple of 16 bytes
- *     (d % 4 == 0 for float32, d % 8 == 0 for bfloat16): rows are moved by the
- *     tensor-memory accelerator.  Violations return S6_ERR_ALIGNMENT.
+ *  Alignment: for the full-sequence calls, x/u, dt, z, y (and out) must be
+ *     16-byte aligned and d * sizeof(io) a multiple of 16 bytes (d % 4 == 0
+ *     for float32, d % 8 == 0 for bfloat16): their rows are moved by the
+ *     tensor-memory accelerator or in 16-byte vectors.  For s6_step, h_ssm and
+ *     A_log must be 16-byte aligned when N is 4, 8 or 16.  Every other
+ *     pointer must be aligned to its element size.  Violations return
+ *     S6_ERR_ALIGNMENT.
  *  Streams: every call is asynchronous on `stream` (NULL = legacy default
  *     stream) and returns once the work is enqueued.
  *  Errors: arguments are checked on the host before anything is enqueued;

@@ -58,6 +58,7 @@ bool make_map_3d(CUtensorMap *map, const void *base, int io, int64_t Bt, int64_t
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void *p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
 
 size_t io_size(int io) { return io == S6_BF16 ? 2 : 4; }
 
@@ -171,9 +172,19 @@ int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv
     const size_t es = io_size(dims->io_dtype);
     if ((dims->d_inner * es) % 16 != 0)
         return S6_ERR_ALIGNMENT;
-    const void *ptrs[] = {x, dt, B, C, y, z, A_log, D, dt_bias, conv_w, conv_b, h_final};
-    for (const void *p : ptrs)
+    // rows moved by TMA need 16-byte aligned bases; the rest is read or
+    // written element by element
+    const void *tma_ptrs[] = {x, dt, y, z};
+    for (const void *p : tma_ptrs)
         if (p && !aligned16(p))
+            return S6_ERR_ALIGNMENT;
+    const void *io_ptrs[] = {B, C};
+    for (const void *p : io_ptrs)
+        if (!aligned_to(p, es))
+            return S6_ERR_ALIGNMENT;
+    const void *f32_ptrs[] = {A_log, D, dt_bias, conv_w, conv_b, h_final};
+    for (const void *p : f32_ptrs)
+        if (p && !aligned_to(p, 4))
             return S6_ERR_ALIGNMENT;
 
     ScanArgs a;
@@ -263,7 +274,7 @@ int causal_conv1d_silu_fwd(const s6_dims *dims, const void *x, const float *conv
         return S6_ERR_INVALID_ARG;
     if ((dims->d_inner * io_size(dims->io_dtype)) % 16 != 0)
         return S6_ERR_ALIGNMENT;
-    if (!aligned16(x) || !aligned16(out) || !aligned16(conv_w) || (conv_b && !aligned16(conv_b)))
+    if (!aligned16(x) || !aligned16(out) || !aligned_to(conv_w, 4) || (conv_b && !aligned_to(conv_b, 4)))
         return S6_ERR_ALIGNMENT;
     s6::ConvArgs a;
     a.Bt = static_cast<int>(dims->batch);
@@ -302,9 +313,19 @@ int s6_step(const s6_dims *dims, const float *A_log, const float *D, const float
         return S6_OK;
     if (!A_log || !D || !conv_w || !u_t || !dt_t || !B_t || !C_t || !h_ssm || !conv_state || !y_t)
         return S6_ERR_INVALID_ARG;
-    const void *ptrs[] = {A_log, D, dt_bias, conv_w, conv_b, u_t, dt_t, B_t, C_t, z_t, h_ssm, conv_state, y_t};
-    for (const void *p : ptrs)
-        if (p && !aligned16(p))
+    // h_ssm and A_log rows are moved 16 bytes at a time when N is 4, 8 or 16;
+    // everything else element by element
+    const size_t es = io_size(dims->io_dtype);
+    const bool vec = dims->d_state == 4 || dims->d_state == 8 || dims->d_state == 16;
+    if (!aligned_to(h_ssm, vec ? 16 : 4) || !aligned_to(A_log, vec ? 16 : 4))
+        return S6_ERR_ALIGNMENT;
+    const void *f32_ptrs[] = {D, dt_bias, conv_w, conv_b};
+    for (const void *p : f32_ptrs)
+        if (p && !aligned_to(p, 4))
+            return S6_ERR_ALIGNMENT;
+    const void *io_ptrs[] = {u_t, dt_t, B_t, C_t, z_t, conv_state, y_t};
+    for (const void *p : io_ptrs)
+        if (p && !aligned_to(p, es))
             return S6_ERR_ALIGNMENT;
     s6::StepArgs a;
     a.Bt = static_cast<int>(dims->batch);
