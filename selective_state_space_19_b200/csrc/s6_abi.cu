@@ -89,6 +89,13 @@ int launch_status(cudaError_t e) { return e == cudaSuccess ? S6_OK : S6_ERR_CUDA
 int use_stream_device(cudaStream_t stream) {
     if (stream == nullptr || stream == cudaStreamLegacy || stream == cudaStreamPerThread)
         return S6_OK;
+    // a stream being captured into a graph: the capture already runs on the
+    // current device, and device queries on it would invalidate the capture
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess)
+        return S6_ERR_CUDA;
+    if (cap != cudaStreamCaptureStatusNone)
+        return S6_OK;
     int dev = -1, cur = -1;
     if (cudaStreamGetDevice(stream, &dev) != cudaSuccess || cudaGetDevice(&cur) != cudaSuccess)
         return S6_ERR_CUDA;

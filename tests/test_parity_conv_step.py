@@ -149,3 +149,43 @@ def test_step_rejects_bad_arguments():
     with pytest.raises(S.S6Error) as e:
         S.s6_step(tok["x"], tok["dt"], tok["B"], tok["C"], p["A_log"], p["D"], w5, h, cs4)
     assert e.value.status == S.S6_ERR_UNSUPPORTED
+
+
+def test_calls_capture_into_a_cuda_graph():
+    """The step and the fused scan can be captured in a CUDA graph and replayed;
+    replays equal eager calls."""
+    import selective_state_space_19_b200 as S
+    import torch
+    p = {k: to_dev(v) for k, v in SI.decode_params(1, d=256).items()}
+    toks = [{k: to_dev(v) for k, v in SI.decode_tokens(s, 1, Bt=8, d=256).items()} for s in range(3)]
+    inp = SI.scan_inputs("long_seq", Bt=1, L=300, d=256)
+    t = dev_inputs(inp)
+    stream = torch.cuda.Stream()
+
+    def run(h, cs, ys, y):
+        for i, tok in enumerate(toks):
+            S.s6_step(tok["x"], tok["dt"], tok["B"], tok["C"], p["A_log"], p["D"], p["conv_w"], h, cs, z_t=tok["z"],
+                      dt_bias=p["dt_bias"], conv_b=p["conv_b"], y_t=ys[i], stream=stream)
+        S.s6_conv_scan_fwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"], z=t["z"],
+                           dt_bias=t["dt_bias"], y=y, h_final=hf, stream=stream)
+
+    def fresh():
+        return (torch.zeros(8, 256, 16, device="cuda"), torch.zeros(8, 256, 3, device="cuda"),
+                [torch.empty(8, 256, device="cuda") for _ in toks], torch.empty_like(t["x"]))
+
+    hf = torch.empty(1, 256, 16, device="cuda")
+    with torch.cuda.stream(stream):
+        h0, c0, ys0, y0 = fresh()
+        run(h0, c0, ys0, y0)
+        torch.cuda.synchronize()
+        ref = [v.clone() for v in ys0] + [h0.clone(), y0.clone(), hf.clone()]
+        h1, c1, ys1, y1 = fresh()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run(h1, c1, ys1, y1)
+        g.replay()
+        torch.cuda.synchronize()
+    got = ys1 + [h1, y1, hf]
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+    assert S.s6_device_status() == 0
