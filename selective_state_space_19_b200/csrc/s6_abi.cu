@@ -105,33 +105,142 @@ int use_stream_device(cudaStream_t stream) {
 }
 
 // ------------------------------------------------------------ scan dispatch
-template <typename IO, int NS, bool CONV, bool ZOH>
-int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, const ScanArgs &a,
+// Library-owned scratch for the dynamic scan: a unit counter, one flag per
+// chain and one published end state per chain.  One buffer per device,
+// allocated on first need and grown on demand (never while a stream is being
+// captured); kept until process exit.
+struct DeviceScratch {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+};
+std::mutex g_scratch_mu;
+DeviceScratch g_scratch[64];
+
+int get_scratch(size_t bytes, cudaStream_t stream, void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return S6_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    DeviceScratch &sc = g_scratch[dev];
+    if (sc.bytes < bytes) {
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        if (stream && cudaStreamIsCapturing(stream, &cap) != cudaSuccess)
+            return S6_ERR_CUDA;
+        if (cap != cudaStreamCaptureStatusNone)
+            return S6_ERR_UNSUPPORTED;  // first (growing) call must come before capture
+        if (sc.ptr && cudaFree(sc.ptr) != cudaSuccess)
+            return S6_ERR_CUDA;
+        sc.ptr = nullptr;
+        sc.bytes = 0;
+        const size_t want = bytes < (size_t(1) << 20) ? (size_t(1) << 20) : bytes;
+        if (cudaMalloc(&sc.ptr, want) != cudaSuccess) {
+            sc.ptr = nullptr;
+            return S6_ERR_CUDA;
+        }
+        sc.bytes = want;
+    }
+    *out = sc.ptr;
+    return S6_OK;
+}
+
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
+
+template <typename IO, int NS, int TPC, bool CONV, bool ZOH>
+int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, ScanArgs a,
                   cudaStream_t stream) {
     constexpr int T = sizeof(IO) == 2 ? 32 : 16;
     constexpr int STAGES = 3;
-    using Smem = s6::ScanSmem<IO, NS, T, STAGES, CONV>;
+    using Sh = s6::ScanShape<NS, TPC, T, CONV>;
+    using Smem = s6::ScanSmem<IO, NS, TPC, T, STAGES, CONV>;
+    constexpr int CPB = Sh::CPB;
     const int io = dims->io_dtype;
-    CUtensorMap tx, tdt, tz, ty;
-    const int xrows = Smem::XR;
-    if (!make_map_3d(&tx, x, io, dims->batch, dims->seqlen, dims->d_inner, s6::kScanThreads, xrows) ||
-        !make_map_3d(&tdt, dt, io, dims->batch, dims->seqlen, dims->d_inner, s6::kScanThreads, T) ||
-        !make_map_3d(&ty, y, io, dims->batch, dims->seqlen, dims->d_inner, s6::kScanThreads, T))
+    const size_t es = io_size(io);
+    CUtensorMap tx, tdt, tz, ty, tB, tC;
+    if (!make_map_3d(&tx, x, io, dims->batch, dims->seqlen, dims->d_inner, CPB, Sh::XR) ||
+        !make_map_3d(&tdt, dt, io, dims->batch, dims->seqlen, dims->d_inner, CPB, T) ||
+        !make_map_3d(&ty, y, io, dims->batch, dims->seqlen, dims->d_inner, CPB, T))
         return S6_ERR_CUDA;
     if (z) {
-        if (!make_map_3d(&tz, z, io, dims->batch, dims->seqlen, dims->d_inner, s6::kScanThreads, T))
+        if (!make_map_3d(&tz, z, io, dims->batch, dims->seqlen, dims->d_inner, CPB, T))
             return S6_ERR_CUDA;
     } else {
         tz = tdt;  // never read when has_z == 0
     }
-    auto kern = s6::s6_scan_kernel<IO, NS, T, STAGES, CONV, ZOH>;
+    // B/C rows by TMA when a row is a whole number of 16-byte units
+    a.bc_tma = (dims->d_state * es) % 16 == 0 && aligned16(a.B) && aligned16(a.C);
+    if (a.bc_tma) {
+        if (!make_map_3d(&tB, a.B, io, dims->batch, dims->seqlen, dims->d_state, static_cast<int>(dims->d_state), T) ||
+            !make_map_3d(&tC, a.C, io, dims->batch, dims->seqlen, dims->d_state, static_cast<int>(dims->d_state), T))
+            return S6_ERR_CUDA;
+    } else {
+        tB = tC = tdt;  // never read
+    }
+    auto kern = s6::s6_scan_kernel<IO, NS, TPC, T, STAGES, CONV, ZOH>;
     const size_t smem = sizeof(Smem);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess)
-        return S6_ERR_CUDA;
-    dim3 grid(static_cast<unsigned>((dims->d_inner + s6::kScanThreads - 1) / s6::kScanThreads),
-              static_cast<unsigned>(dims->batch));
-    kern<<<grid, s6::kScanThreads, smem, stream>>>(tx, tdt, tz, ty, a);
+    static int occ = 0;  // resident CTAs per SM for this instantiation
+    if (!occ) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+            return S6_ERR_CUDA;
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, s6::kScanThreads, smem) != cudaSuccess || nb < 1)
+            return S6_ERR_CUDA;
+        occ = nb;
+    }
+
+    // ---- work split: chains of segments, pulled dynamically when there are
+    // too few chains to balance the SMs statically
+    const int64_t L = dims->seqlen;
+    a.tiles = static_cast<int>((dims->d_inner + CPB - 1) / CPB);
+    const int64_t chains = dims->batch * a.tiles;
+    const int64_t workers = static_cast<int64_t>(device_sm_count()) * occ;
+    int64_t nseg = 1, seg_len = round_up(static_cast<size_t>(L), T);
+    if (chains < 4 * workers && L > 4 * T) {
+        const int64_t grid = chains < workers ? chains : workers;
+        int64_t want = (8 * grid + chains - 1) / chains;
+        const int64_t max_seg = L / (4 * T);
+        if (want > max_seg)
+            want = max_seg;
+        if (want > 1) {
+            seg_len = round_up(static_cast<size_t>((L + want - 1) / want), T);
+            nseg = (L + seg_len - 1) / seg_len;
+        }
+    }
+    if (chains * nseg > 0x7fffffffLL)
+        return S6_ERR_UNSUPPORTED;
+    a.nseg = static_cast<int>(nseg);
+    a.seg_len = static_cast<int>(seg_len);
+    a.units = static_cast<int>(chains * nseg);
+    a.dynamic = nseg > 1;
+    unsigned grid = static_cast<unsigned>(chains);
+    if (a.dynamic) {
+        const size_t hdr = round_up(4 + 4 * static_cast<size_t>(chains), 256);
+        const size_t carry = static_cast<size_t>(chains) * CPB * NS * sizeof(float);
+        void *scr = nullptr;
+        const int st = get_scratch(hdr + carry, stream, &scr);
+        if (st != S6_OK)
+            return st;
+        a.counter = static_cast<unsigned int *>(scr);
+        a.flags = a.counter + 1;
+        a.carry = reinterpret_cast<float *>(static_cast<char *>(scr) + hdr);
+        if (cudaMemsetAsync(scr, 0, 4 + 4 * static_cast<size_t>(chains), stream) != cudaSuccess)
+            return S6_ERR_CUDA;
+        grid = static_cast<unsigned>(chains < workers ? chains : workers);
+    }
+    kern<<<grid, s6::kScanThreads, smem, stream>>>(tx, tdt, tz, ty, tB, tC, a);
     return launch_status(cudaGetLastError());
 }
 
@@ -139,10 +248,10 @@ template <typename IO, bool CONV, bool ZOH>
 int launch_scan_n(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, const ScanArgs &a,
                   cudaStream_t st) {
     if (dims->d_state <= 4)
-        return launch_scan_t<IO, 4, CONV, ZOH>(dims, x, dt, z, y, a, st);
+        return launch_scan_t<IO, 4, 1, CONV, ZOH>(dims, x, dt, z, y, a, st);
     if (dims->d_state <= 8)
-        return launch_scan_t<IO, 8, CONV, ZOH>(dims, x, dt, z, y, a, st);
-    return launch_scan_t<IO, 16, CONV, ZOH>(dims, x, dt, z, y, a, st);
+        return launch_scan_t<IO, 8, 1, CONV, ZOH>(dims, x, dt, z, y, a, st);
+    return launch_scan_t<IO, 16, 2, CONV, ZOH>(dims, x, dt, z, y, a, st);
 }
 
 template <typename IO>
@@ -195,6 +304,7 @@ int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv
             return S6_ERR_ALIGNMENT;
 
     ScanArgs a;
+    std::memset(&a, 0, sizeof(a));
     a.Bt = static_cast<int>(dims->batch);
     a.L = static_cast<int>(dims->seqlen);
     a.d = static_cast<int>(dims->d_inner);

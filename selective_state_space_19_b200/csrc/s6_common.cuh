@@ -58,6 +58,116 @@ __device__ __forceinline__ float silu_f(float v) {
     return v * rcp_approx(1.0f + ex2_approx(-v * kLog2e));
 }
 
+// ------------------------------------------- FMA-pipe function evaluation
+// These move work off the special-function (MUFU) pipe, which the decays
+// keep busy, onto the FMA pipe.  Coefficients and constants were fitted for
+// this library (relative-error least squares on Chebyshev points, float64)
+// and checked in float32 Horner evaluation; the bounds are stated per function.
+
+// 1/x for x in [1, 2^120]: exponent-negation seed y0 = bits(K - bits(x))
+// (max relative error 5.1e-2 over a binade for K = 0x7EF311C0), then three
+// Newton steps y <- y (2 - x y) (error squares each step: < 1e-9 before
+// float32 rounding).
+__device__ __forceinline__ float rcp_newton(float x) {
+    float y = __int_as_float(0x7EF311C0 - __float_as_int(x));
+    float e = fmaf(-x, y, 1.0f);
+    y = fmaf(y, e, y);
+    e = fmaf(-x, y, 1.0f);
+    y = fmaf(y, e, y);
+    e = fmaf(-x, y, 1.0f);
+    return fmaf(y, e, y);
+}
+
+// SiLU with one MUFU op: the exponent argument is clamped at 120 so the
+// reciprocal stays in the normal range (SiLU(v) < 1e-34 there anyway).
+__device__ __forceinline__ float silu_fast(float v) {
+    const float e = ex2_approx(fminf(-v * kLog2e, 120.0f));
+    return v * rcp_newton(1.0f + e);
+}
+
+// log1p(e) / e on [0, 1], degree 9 (float32 evaluation: max relative error
+// 1.4e-7 for log1p(e) = e * q(e)).
+__device__ __forceinline__ float log1p_over_x_01(float e) {
+    float q = -0.0032439918722957373f;
+    q = fmaf(q, e, 0.019851312041282654f);
+    q = fmaf(q, e, -0.056959252804517746f);
+    q = fmaf(q, e, 0.10603626072406769f);
+    q = fmaf(q, e, -0.15305575728416443f);
+    q = fmaf(q, e, 0.19675932824611664f);
+    q = fmaf(q, e, -0.24954132735729218f);
+    q = fmaf(q, e, 0.3332996368408203f);
+    q = fmaf(q, e, -0.4999990165233612f);
+    return fmaf(q, e, 1.0f);
+}
+
+// softplus(v) = max(v, 0) + log1p(e^-|v|) with one MUFU op (the power) and
+// the log1p on the FMA pipe; relative accuracy ~1.5e-7 down to tiny results.
+__device__ __forceinline__ float softplus_fast(float v) {
+    const float e = ex2_approx(-fabsf(v) * kLog2e);
+    return fmaf(e, log1p_over_x_01(e), fmaxf(v, 0.0f));
+}
+
+// ----------------------------------------------------- packed float32 pairs
+// sm_100 executes two float32 lanes per instruction (add/mul/fma .f32x2);
+// a pair lives in one 64-bit register (low half = first element).
+typedef unsigned long long f2_t;
+
+__device__ __forceinline__ f2_t f2_pack(float lo, float hi) {
+    f2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(f2_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
+    f2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f2_t f2_mul(f2_t a, f2_t b) {
+    f2_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2_t f2_add(f2_t a, f2_t b) {
+    f2_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2_t f2_sub(f2_t a, f2_t b) {
+    f2_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for a pair x <= 0 on the FMA pipe: x = n + f with n = round(x) taken
+// from the low mantissa bits of x + 1.5*2^23, f in [-1/2, 1/2], 2^f by a
+// degree-6 polynomial (float32 relative error 7.9e-8), scaled by adding n to
+// the exponent field.  x is clamped at -125 (results stay normal; the decay
+// is below 1e-37 there).
+__device__ __forceinline__ f2_t f2_exp2_poly(f2_t x) {
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const f2_t magic = f2_pack(12582912.0f, 12582912.0f);
+    const f2_t t = f2_add(x, magic);
+    const f2_t f = f2_sub(x, f2_sub(t, magic));
+    f2_t p = f2_pack(0.0001534580806037411f, 0.0001534580806037411f);
+    p = f2_fma(p, f, f2_pack(0.0013399930903688073f, 0.0013399930903688073f));
+    p = f2_fma(p, f, f2_pack(0.009618489071726799f, 0.009618489071726799f));
+    p = f2_fma(p, f, f2_pack(0.05550328642129898f, 0.05550328642129898f));
+    p = f2_fma(p, f, f2_pack(0.24022646248340607f, 0.24022646248340607f));
+    p = f2_fma(p, f, f2_pack(0.6931471824645996f, 0.6931471824645996f));
+    p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
+    float t0, t1, p0, p1;
+    f2_unpack(t, t0, t1);
+    f2_unpack(p, p0, p1);
+    p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+    return f2_pack(p0, p1);
+}
+
 // softplus(v) = log(1 + e^v) = max(v, 0) + log1p(e^-|v|).
 // log1p(e) is formed as log2(1 + e) * ln2, corrected for the rounding of
 // 1 + e by the factor e / ((1 + e) - 1) (the subtraction is exact); when
@@ -87,6 +197,10 @@ __device__ __forceinline__ void fence_mbarrier_init() {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
@@ -151,6 +265,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------- flags between thread blocks
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned int *p, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 // Device-side error word (one per device image of the library; the library is
