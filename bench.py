@@ -344,12 +344,13 @@ def run_ours(args):
     pk = peaks()
     cfg = dict(SI.CONFIGS[WORKLOAD])
     if args.case == "small":
-        # profiling case: same kernel and distributions, 2 of the 16 sequences
-        # (25M elements, ~150 MB of inputs: still larger than L2)
-        cfg.update(Bt=2)
+        # profiling case: same kernel, distributions, batch and width, 1/8 of the
+        # sequence (25M elements, ~150 MB of inputs: still larger than L2; the
+        # same 384 (sequence, channel-tile) chains as the full workload)
+        cfg.update(L=1024)
         args.no_rows = args.no_e2e = args.no_cpu_baseline = True
     zoh = bool(cfg["zoh"])
-    over = {k: cfg[k] for k in ("Bt",)}
+    over = {k: cfg[k] for k in ("Bt", "L")}
     inp = SI.scan_inputs(WORKLOAD, seed=cfg["seed"] + rank, **over)  # each rank its own batch (weak scaling)
     Bt, L, d, N = cfg["Bt"], cfg["L"], cfg["d"], cfg["N"]
     elems = Bt * L * d
@@ -473,7 +474,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--case", choices=["full", "small"], default="full",
-                    help="small: 2 sequences of the workload only (for ncu captures)")
+                    help="small: the workload at L=1024 (for ncu captures)")
     ap.add_argument("--no-rows", action="store_true", help="skip the decode-step and standalone-conv rows")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
