@@ -171,7 +171,7 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     CUtensorMap tx, tdt, tz, ty, tB, tC;
     if (!make_map_3d(&tx, x, io, dims->batch, dims->seqlen, dims->d_inner, CPB, Sh::XR) ||
         !make_map_3d(&tdt, dt, io, dims->batch, dims->seqlen, dims->d_inner, CPB, T) ||
-        !make_map_3d(&ty, y, io, dims->batch, dims->seqlen, dims->d_inner, CPB, T))
+        !make_map_3d(&ty, y, io, dims->batch, dims->seqlen, dims->d_inner, Sh::CPW, T))  // per-warp stores
         return S6_ERR_CUDA;
     if (z) {
         if (!make_map_3d(&tz, z, io, dims->batch, dims->seqlen, dims->d_inner, CPB, T))
@@ -196,7 +196,7 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
             cudaSuccess)
             return S6_ERR_CUDA;
         int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, s6::kScanThreads, smem) != cudaSuccess || nb < 1)
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, s6::kScanBlock, smem) != cudaSuccess || nb < 1)
             return S6_ERR_CUDA;
         occ = nb;
     }
@@ -227,7 +227,8 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     a.dynamic = nseg > 1;
     unsigned grid = static_cast<unsigned>(chains);
     if (a.dynamic) {
-        const size_t hdr = round_up(4 + 4 * static_cast<size_t>(chains), 256);
+        const size_t nflags = static_cast<size_t>(chains) * s6::kConsumerWarps;
+        const size_t hdr = round_up(4 + 4 * nflags, 256);
         const size_t carry = static_cast<size_t>(chains) * CPB * NS * sizeof(float);
         void *scr = nullptr;
         const int st = get_scratch(hdr + carry, stream, &scr);
@@ -236,11 +237,11 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
         a.counter = static_cast<unsigned int *>(scr);
         a.flags = a.counter + 1;
         a.carry = reinterpret_cast<float *>(static_cast<char *>(scr) + hdr);
-        if (cudaMemsetAsync(scr, 0, 4 + 4 * static_cast<size_t>(chains), stream) != cudaSuccess)
+        if (cudaMemsetAsync(scr, 0, 4 + 4 * nflags, stream) != cudaSuccess)
             return S6_ERR_CUDA;
         grid = static_cast<unsigned>(chains < workers ? chains : workers);
     }
-    kern<<<grid, s6::kScanThreads, smem, stream>>>(tx, tdt, tz, ty, tB, tC, a);
+    kern<<<grid, s6::kScanBlock, smem, stream>>>(tx, tdt, tz, ty, tB, tC, a);
     return launch_status(cudaGetLastError());
 }
 

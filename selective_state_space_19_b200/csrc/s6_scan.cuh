@@ -12,36 +12,40 @@
 //     h[n]   = A_bar * h[n] + write
 //     y      = (sum_n h[n] C_t[n] + D u) * SiLU(z_t)   (C reads the updated state)
 //
-// Work decomposition.  TPC threads share one channel (TPC = 2 at N = 16:
-// each keeps NH = N/TPC float32 states in registers), so a CTA of 128
-// threads owns CPB = 128/TPC consecutive channels of one sequence.  A
+// Work decomposition.  TPC threads share one channel (TPC = 2 at N = 16,
+// each keeping NH = N/TPC float32 states in registers); the 4 consumer warps
+// of a CTA own CPB = 128/TPC consecutive channels of one sequence.  A
 // sequence's channel tile is a chain of segments of seg_len tokens; a
 // (segment, tile) pair is a unit of work.  In the dynamic mode persistent
-// CTAs pull units, segment-major, from a global counter; a unit whose segment
-// is not the first waits (bounded) for the state its predecessor publishes in
-// a carry buffer -- the predecessor was pulled earlier by a running CTA, so
-// the wait always ends.  This spreads B*d/CPB chains evenly over every SM
-// whatever their count, without recomputing a single decay.  In the static
-// mode (plenty of chains) each CTA runs one whole chain.
+// CTAs pull units, segment-major, from a global counter, and a unit whose
+// segment is not the first starts from the state its predecessor published in
+// a carry buffer.  The predecessor was pulled earlier by a running CTA, so the
+// (bounded) wait for it always ends.  This spreads B*d/CPB chains evenly over
+// every SM whatever their count, without recomputing a single decay.  In the
+// static mode (plenty of chains) each CTA runs one whole chain.
 //
-// Data movement.  Per chunk of T tokens one elected thread issues TMA tile
-// loads of the [T(+3 halo) x CPB] slices of x, dt and z and the [T x N] rows
-// of B and C into a STAGES-deep shared-memory ring (mbarrier completion; the
-// chunk's unit, first token and flags travel with it in shared memory).  The
-// 3 halo rows give the conv its K-1 earlier inputs; rows before token 0 are
-// zero-filled by the TMA unit (the conv's zero left padding).  B/C rows are
-// converted once per chunk to float32 (shared by all channels); each thread
-// reads its channel column and the broadcast B/C rows and writes y into a
-// triple-buffered tile that the elected thread stores with a TMA bulk store.
+// Warp roles.  Warp 4 is the producer: it pulls units, issues per chunk of T
+// tokens the TMA tile loads of the [T(+3 halo) x CPB] slices of x, dt, z and
+// the [T x N] rows of B and C into a STAGES-deep shared-memory ring, fetches a
+// unit's start state from the carry buffer once its flags are published, and
+// converts each chunk's B/C rows to float32 before marking the stage ready.
+// The 3 halo rows give the conv its K-1 earlier inputs; rows before token 0
+// are zero-filled by the TMA unit (the conv's zero left padding).  Warps 0-3
+// are consumers: each waits for a ready stage, runs its 32/TPC channels over
+// the chunk, releases the stage, and stores its own y tile with a TMA bulk
+// store -- no CTA-wide barrier in the steady state.
 //
 // Arithmetic.  The 16 decays per element are the binding work (one live
-// exponential per state per token, "the s6 cell").  They go to the MUFU ex2
-// pipe; SiLU and softplus use one MUFU op each, with their reciprocal and
-// log1p on the FMA pipe; with TPC = 2 the two threads of a channel split the
-// two SiLUs (conv output, gate) and exchange them with one shuffle.  State
-// arithmetic runs on packed float32 pairs (f32x2).  Scalars of token j+1 are
-// computed before the state update of token j to give the scheduler
-// independent work.
+// exponential per state per token, "the s6 cell") and go to the MUFU ex2
+// pipe.  SiLU and softplus take one MUFU op each, their reciprocal and log1p
+// run on the FMA pipe.  With TPC = 2 the two threads of a channel walk the
+// tokens in pairs: each computes every per-token scalar (conv, both SiLUs,
+// softplus) of one token of the pair and the two swap u and Delta with
+// shuffles, so no scalar is computed twice; each then updates its NH states
+// for both tokens, and the partial readouts are swapped so that each thread
+// finishes and writes the output of its own token.  State arithmetic runs on
+// packed float32 pairs (f32x2); the scalars of the next pair are computed
+// before the state update of the current one.
 //
 // No tensor cores: the recurrence is diagonal (an elementwise product with a
 // data-dependent decay), not a contraction.
@@ -51,12 +55,15 @@
 
 namespace s6 {
 
-constexpr int kScanThreads = 128;
-constexpr int kHalo = 3;  // conv history rows (taps padded to 4)
+constexpr int kConsumerWarps = 4;
+constexpr int kScanThreads = 32 * kConsumerWarps;  // consumer threads
+constexpr int kScanBlock = kScanThreads + 32;      // + one producer warp
+constexpr int kHalo = 3;                           // conv history rows (taps padded to 4)
 
 constexpr int kMetaFirst = 1;  // first chunk of its unit
 constexpr int kMetaLast = 2;   // last chunk of its unit
 constexpr int kMetaEnd = 4;    // no more work
+constexpr int kMetaCarry = 8;  // the unit starts from a published carry
 
 struct ScanArgs {
     int Bt, L, d, N, K;
@@ -76,7 +83,7 @@ struct ScanArgs {
     const float *conv_b;   // [d] or null
     float *h_final;        // [Bt, d, N] or null
     unsigned int *counter;  // dynamic: next unit to hand out (zeroed before launch)
-    unsigned int *flags;    // dynamic: [Bt*tiles] segments whose end state is published
+    unsigned int *flags;    // dynamic: [Bt*tiles][consumer warps] last published segment + 1
     float *carry;           // dynamic: [Bt*tiles][CPB][NS] published end states
 };
 
@@ -84,8 +91,10 @@ template <int NS, int TPC, int T, bool CONV>
 struct ScanShape {
     static constexpr int NH = NS / TPC;             // states per thread
     static constexpr int CPB = kScanThreads / TPC;  // channels per CTA
+    static constexpr int CPW = 32 / TPC;            // channels per consumer warp
     static constexpr int XR = T + (CONV ? kHalo : 0);
     static_assert(NH % 4 == 0, "states per thread must be a multiple of 4");
+    static_assert(T % 2 == 0, "chunks hold whole token pairs");
 };
 
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV>
@@ -94,12 +103,15 @@ struct ScanSmem {
     IO x[STAGES][Sh::XR][Sh::CPB];
     IO dt[STAGES][T][Sh::CPB];
     IO z[STAGES][T][Sh::CPB];
-    IO y[3][T][Sh::CPB];
+    IO y[kConsumerWarps][3][T][Sh::CPW];  // per consumer warp, triple-buffered
     IO braw[STAGES][T * NS];
     IO craw[STAGES][T * NS];
-    float bc[2][T][2][NS];  // [buffer][token][B|C][n], float32, zero-padded to NS
-    int4 meta[STAGES];      // {unit, t0, tcount, flags}
-    uint64_t full[STAGES];
+    float bc[STAGES][T][2][NS];        // [stage][token][B|C][n], float32, zero-padded
+    float hinit[STAGES][Sh::CPB][NS];  // start state of a unit that begins in the stage
+    int4 meta[STAGES];                 // {unit, t0, tcount, flags}
+    uint64_t full[STAGES];             // TMA bytes landed (producer waits)
+    uint64_t ready[STAGES];            // stage complete and converted (consumers wait)
+    uint64_t empty[STAGES];            // all consumer warps done with the stage
 };
 
 struct UnitPos {
@@ -116,13 +128,10 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
     return p;
 }
 
-// Per-token scalars of one channel.
-struct TokScalars {
-    float u, delta, g;
-};
+constexpr uint32_t kWaitPolls = 1u << 24;
 
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, bool ZOH>
-__global__ void __launch_bounds__(kScanThreads, 2)
+__global__ void __launch_bounds__(kScanBlock, 1)
     s6_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
                    const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -133,117 +142,205 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     constexpr int NH = Sh::NH;
     constexpr int NP = NH / 2;  // state pairs per thread
     constexpr int CPB = Sh::CPB;
+    constexpr int CPW = Sh::CPW;
+    constexpr int XR = Sh::XR;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
 
     const int tid = threadIdx.x;
-    const int cl = tid / TPC;                    // channel within the tile
-    const int half = (TPC == 2) ? (tid & 1) : 0;  // which NH states of the channel
-    const int n0 = half * NH;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
 
-    // ------------------------------------------------ producer (thread 0 only)
-    int p_unit = -1, p_k = 0, p_nk = 0, p_tlo = 0, p_thi = 0, p_count = 0;
-    bool p_done = false, p_first_pull = true;
-    auto pull_unit = [&]() {
-        int u;
-        if (a.dynamic) {
-            u = static_cast<int>(atomicAdd(a.counter, 1u));
-        } else {
-            u = p_first_pull ? static_cast<int>(blockIdx.x) : a.units;
-        }
-        p_first_pull = false;
-        if (u >= a.units) {
-            p_done = true;
-            return;
-        }
-        const UnitPos up = unit_pos(u, a);
-        p_unit = u;
-        p_k = 0;
-        p_tlo = up.seg * a.seg_len;
-        p_thi = min(a.L, p_tlo + a.seg_len);
-        p_nk = (p_thi - p_tlo + T - 1) / T;
-    };
-    auto produce = [&](int s) {
-        ++p_count;
-        if (!p_done && p_k == p_nk)
-            pull_unit();
-        if (p_done) {
-            sm.meta[s] = make_int4(-1, 0, 0, kMetaEnd);
-            mbar_arrive(&sm.full[s]);
-            return;
-        }
-        const UnitPos up = unit_pos(p_unit, a);
-        const int t0 = p_tlo + p_k * T;
-        const int fl = (p_k == 0 ? kMetaFirst : 0) | (p_k == p_nk - 1 ? kMetaLast : 0);
-        sm.meta[s] = make_int4(p_unit, t0, min(T, p_thi - t0), fl);
-        const int c0 = up.tile * CPB;
-        constexpr uint32_t kX = Sh::XR * CPB * sizeof(IO);
-        constexpr uint32_t kR = T * CPB * sizeof(IO);
-        const uint32_t kBC = a.bc_tma ? 2u * T * a.N * static_cast<uint32_t>(sizeof(IO)) : 0u;
-        mbar_arrive_expect_tx(&sm.full[s], kX + kR + (a.has_z ? kR : 0u) + kBC);
-        tma_load_3d(&sm.x[s][0][0], &tm_x, &sm.full[s], c0, t0 - (CONV ? kHalo : 0), up.b);
-        tma_load_3d(&sm.dt[s][0][0], &tm_dt, &sm.full[s], c0, t0, up.b);
-        if (a.has_z)
-            tma_load_3d(&sm.z[s][0][0], &tm_z, &sm.full[s], c0, t0, up.b);
-        if (a.bc_tma) {
-            tma_load_3d(&sm.braw[s][0], &tm_B, &sm.full[s], 0, t0, up.b);
-            tma_load_3d(&sm.craw[s][0], &tm_C, &sm.full[s], 0, t0, up.b);
-        }
-        ++p_k;
-    };
-
-    // B/C rows of a chunk -> float32 buffer (all threads; zero beyond N and L)
-    auto stage_bc = [&](int s, int buf) {
-        constexpr int kSlots = 2 * T * NS;
-        const int4 m = sm.meta[s];
-        if (m.w & kMetaEnd)
-            return;
-        const UnitPos up = unit_pos(m.x, a);
+    if (tid == 0) {
 #pragma unroll
-        for (int k = 0; k < (kSlots + kScanThreads - 1) / kScanThreads; ++k) {
-            const int j = tid + k * kScanThreads;
-            if (j < kSlots) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.ready[s], 1);
+            mbar_init(&sm.empty[s], kConsumerWarps);
+        }
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+
+    if (warp == kConsumerWarps) {
+        // =========================================================== producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_x);
+            prefetch_tensormap(&tm_dt);
+            if (a.has_z)
+                prefetch_tensormap(&tm_z);
+            if (a.bc_tma) {
+                prefetch_tensormap(&tm_B);
+                prefetch_tensormap(&tm_C);
+            }
+        }
+        int unit = -1, k = 0, nk = 0, tlo = 0, thi = 0;
+        bool done = false, first_pull = true, ok = true;
+
+        // B/C rows of chunk cc -> float32 (all 32 lanes), then the stage is ready
+        auto finish = [&](int cc) {
+            const int sp = cc % STAGES;
+            __syncwarp();  // lane 0's metadata write is visible to the warp
+            bool got = true;
+            if (lane == 0)
+                got = mbar_wait_bounded(&sm.full[sp], (cc / STAGES) & 1, kWaitPolls);
+            got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+            if (!got) {
+                if (lane == 0)
+                    raise_device_error(1u);
+                ok = false;
+            }
+            const int4 m = sm.meta[sp];
+            const UnitPos up = unit_pos(m.x, a);
+            constexpr int kSlots = 2 * T * NS;
+            if (got && a.bc_tma && a.N == NS) {
+                // whole rows: four values per lane step
+                for (int j = lane; j < kSlots / 4; j += 32) {
+                    const int which = j / (T * NS / 4);
+                    const int rem = j - which * (T * NS / 4);
+                    const int tt = rem / (NS / 4);
+                    const int n = (rem - tt * (NS / 4)) * 4;
+                    const IO *src = which ? &sm.craw[sp][tt * NS + n] : &sm.braw[sp][tt * NS + n];
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (tt < m.z) {
+                        if constexpr (sizeof(IO) == 2) {
+                            const uint2 r = *reinterpret_cast<const uint2 *>(src);
+                            v = make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u),
+                                            __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
+                        } else {
+                            v = *reinterpret_cast<const float4 *>(src);
+                        }
+                    }
+                    *reinterpret_cast<float4 *>(&sm.bc[sp][tt][which][n]) = v;
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sm.ready[sp]);
+                return;
+            }
+            for (int j = lane; j < kSlots; j += 32) {
                 const int which = j / (T * NS);
                 const int rem = j - which * (T * NS);
                 const int tt = rem / NS;
                 const int n = rem - tt * NS;
                 float v = 0.0f;
-                if (n < a.N && tt < m.z) {
+                if (got && n < a.N && tt < m.z) {
                     if (a.bc_tma) {
-                        v = tr::to_f(which ? sm.craw[s][tt * a.N + n] : sm.braw[s][tt * a.N + n]);
+                        v = tr::to_f(which ? sm.craw[sp][tt * a.N + n] : sm.braw[sp][tt * a.N + n]);
                     } else {
                         const size_t off = (static_cast<size_t>(up.b) * a.L + m.y + tt) * a.N + n;
                         v = tr::to_f(which ? static_cast<const IO *>(a.C)[off] : static_cast<const IO *>(a.B)[off]);
                     }
                 }
-                sm.bc[buf][tt][which][n] = v;
+                sm.bc[sp][tt][which][n] = v;
             }
-        }
-    };
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.ready[sp]);
+        };
 
-    if (tid == 0) {
-        prefetch_tensormap(&tm_x);
-        prefetch_tensormap(&tm_dt);
-        prefetch_tensormap(&tm_y);
-        if (a.has_z)
-            prefetch_tensormap(&tm_z);
-        if (a.bc_tma) {
-            prefetch_tensormap(&tm_B);
-            prefetch_tensormap(&tm_C);
+        int c = 0;
+        for (;; ++c) {
+            const int s = c % STAGES;
+            if (c >= STAGES) {
+                bool got = true;
+                if (lane == 0)
+                    got = mbar_wait_bounded(&sm.empty[s], ((c / STAGES) - 1) & 1, kWaitPolls);
+                got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                if (!got) {
+                    if (lane == 0)
+                        raise_device_error(1u);
+                    ok = false;
+                }
+            }
+            if (ok && !done && k == nk) {
+                int u = 0;
+                if (lane == 0) {
+                    if (a.dynamic)
+                        u = static_cast<int>(atomicAdd(a.counter, 1u));
+                    else
+                        u = first_pull ? static_cast<int>(blockIdx.x) : a.units;
+                }
+                u = __shfl_sync(0xffffffffu, u, 0);
+                first_pull = false;
+                if (u >= a.units) {
+                    done = true;
+                } else {
+                    const UnitPos up = unit_pos(u, a);
+                    unit = u;
+                    k = 0;
+                    tlo = up.seg * a.seg_len;
+                    thi = min(a.L, tlo + a.seg_len);
+                    nk = (thi - tlo + T - 1) / T;
+                }
+            }
+            if (done || !ok) {
+                if (lane == 0)
+                    sm.meta[s] = make_int4(-1, 0, 0, kMetaEnd);
+                if (c >= 1)
+                    finish(c - 1);
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sm.ready[s]);
+                break;
+            }
+            const UnitPos up = unit_pos(unit, a);
+            const int t0 = tlo + k * T;
+            const bool carry_in = a.dynamic && k == 0 && up.seg > 0;
+            const int fl = (k == 0 ? kMetaFirst : 0) | (k == nk - 1 ? kMetaLast : 0) | (carry_in ? kMetaCarry : 0);
+            if (lane == 0) {
+                sm.meta[s] = make_int4(unit, t0, min(T, thi - t0), fl);
+                const int c0 = up.tile * CPB;
+                constexpr uint32_t kX = XR * CPB * sizeof(IO);
+                constexpr uint32_t kR = T * CPB * sizeof(IO);
+                const uint32_t kBC = a.bc_tma ? 2u * T * a.N * static_cast<uint32_t>(sizeof(IO)) : 0u;
+                mbar_arrive_expect_tx(&sm.full[s], kX + kR + (a.has_z ? kR : 0u) + kBC);
+                tma_load_3d(&sm.x[s][0][0], &tm_x, &sm.full[s], c0, t0 - (CONV ? kHalo : 0), up.b);
+                tma_load_3d(&sm.dt[s][0][0], &tm_dt, &sm.full[s], c0, t0, up.b);
+                if (a.has_z)
+                    tma_load_3d(&sm.z[s][0][0], &tm_z, &sm.full[s], c0, t0, up.b);
+                if (a.bc_tma) {
+                    tma_load_3d(&sm.braw[s][0], &tm_B, &sm.full[s], 0, t0, up.b);
+                    tma_load_3d(&sm.craw[s][0], &tm_C, &sm.full[s], 0, t0, up.b);
+                }
+            }
+            if (carry_in) {
+                // the predecessor segment publishes one flag per consumer warp
+                bool got = true;
+                if (lane < kConsumerWarps) {
+                    got = false;
+                    const unsigned int *f = &a.flags[static_cast<size_t>(up.chain) * kConsumerWarps + lane];
+                    for (uint32_t i = 0; i < (1u << 22); ++i) {
+                        if (ld_acquire_gpu(f) >= static_cast<unsigned int>(up.seg)) {
+                            got = true;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                }
+                if (!__all_sync(0xffffffffu, got)) {
+                    if (lane == 0)
+                        raise_device_error(2u);
+                }
+                const float4 *src =
+                    reinterpret_cast<const float4 *>(a.carry + static_cast<size_t>(up.chain) * CPB * NS);
+                float4 *dst = reinterpret_cast<float4 *>(&sm.hinit[s][0][0]);
+                for (int i = lane; i < CPB * NS / 4; i += 32)
+                    dst[i] = __ldcg(src + i);
+            }
+            if (c >= 1)
+                finish(c - 1);
+            ++k;
         }
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s)
-            mbar_init(&sm.full[s], 1);
-        fence_mbarrier_init();
-    }
-    __syncthreads();
-    if (tid == 0) {
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s)
-            produce(s);
+        return;
     }
 
-    // ------------------------------------------------ per-channel state
+    // ============================================================== consumers
+    const int cw = lane / TPC;       // channel within the warp
+    const int cl = warp * CPW + cw;  // channel within the CTA tile
+    const int half = (TPC == 2) ? (lane & 1) : 0;
+    const int n0 = half * NH;
+
     f2_t hp[NP], A2p[NP], nrAp[NP];
     float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, cb = 0.f, Dd = 0.f, bias = 0.f;
     bool live = false;
@@ -252,23 +349,58 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     for (int q = 0; q < NP; ++q)
         hp[q] = A2p[q] = nrAp[q] = f2_pack(0.f, 0.f);
 
-    bool ok = mbar_wait_bounded(&sm.full[0], 0, 1u << 24);
-    if (ok)
-        stage_bc(0, 0);
-    ok = !__syncthreads_or(!ok);
-    if (!ok && tid == 0)
-        raise_device_error(1u);
+    // one token's contribution to this thread's states; returns the partial readout
+    auto update = [&](const float(*bcrow)[NS], float u, float delta) -> float {
+        const f2_t dd = f2_pack(delta, delta);
+        const f2_t uu = f2_pack(u, u);
+        const f2_t du = f2_mul(dd, uu);
+        f2_t acc = f2_pack(0.f, 0.f);
+        const ulonglong2 *Bq = reinterpret_cast<const ulonglong2 *>(&bcrow[0][n0]);
+        const ulonglong2 *Cq = reinterpret_cast<const ulonglong2 *>(&bcrow[1][n0]);
+#pragma unroll
+        for (int q2 = 0; q2 < NP / 2; ++q2) {
+            const ulonglong2 Bv = Bq[q2];
+            const ulonglong2 Cv = Cq[q2];
+            const f2_t Bp[2] = {Bv.x, Bv.y};
+            const f2_t Cp[2] = {Cv.x, Cv.y};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int q = 2 * q2 + e;
+                const f2_t dA = f2_mul(dd, A2p[q]);
+                float d0, d1;
+                f2_unpack(dA, d0, d1);
+                const f2_t ab = f2_pack(ex2_approx(d0), ex2_approx(d1));
+                if (ZOH) {
+                    // h' = abar*h + (abar-1)*k, k = B u / A; with nk = -k:
+                    // h' = abar*(h - nk) + nk
+                    const f2_t nk = f2_mul(nrAp[q], f2_mul(uu, Bp[e]));
+                    hp[q] = f2_fma(ab, f2_sub(hp[q], nk), nk);
+                } else {
+                    hp[q] = f2_fma(ab, hp[q], f2_mul(du, Bp[e]));
+                }
+                acc = f2_fma(hp[q], Cp[e], acc);
+            }
+        }
+        float a0, a1;
+        f2_unpack(acc, a0, a1);
+        return a0 + a1;
+    };
 
-    int ci = 0;
-    while (ok) {
-        const int s = ci % STAGES;
+    for (int c = 0;; ++c) {
+        const int s = c % STAGES;
+        const bool got = mbar_wait_bounded(&sm.ready[s], (c / STAGES) & 1, kWaitPolls);
+        if (!__all_sync(0xffffffffu, got)) {
+            if (lane == 0)
+                raise_device_error(1u);
+            break;
+        }
         const int4 m = sm.meta[s];
         if (m.w & kMetaEnd)
             break;
-        const UnitPos up = unit_pos(m.x, a);
 
         if (m.w & kMetaFirst) {
             // ---- a new unit: this thread's channel parameters and start state
+            const UnitPos up = unit_pos(m.x, a);
             chain = up.chain;
             seg = up.seg;
             bseq = up.b;
@@ -280,9 +412,9 @@ __global__ void __launch_bounds__(kScanThreads, 2)
                 // taps right-aligned into 4 slots: width K is the width-4 conv
                 // with its 4-K oldest taps zero, so the halo is always 3 rows
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int src = k - (4 - a.K);
-                    wv[k] = (src >= 0) ? a.conv_w[static_cast<size_t>(ch) * a.K + src] : 0.0f;
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int src = kk - (4 - a.K);
+                    wv[kk] = (src >= 0) ? a.conv_w[static_cast<size_t>(ch) * a.K + src] : 0.0f;
                 }
             }
             w0 = wv[0];
@@ -292,6 +424,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
             cb = (CONV && live && a.conv_b) ? a.conv_b[ch] : 0.0f;
             Dd = live ? a.D[ch] : 0.0f;
             bias = (live && a.dt_bias) ? a.dt_bias[ch] : 0.0f;
+            const bool carry_in = (m.w & kMetaCarry) != 0;
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
                 float al[2] = {0.f, 0.f}, nr[2] = {0.f, 0.f};
@@ -306,31 +439,8 @@ __global__ void __launch_bounds__(kScanThreads, 2)
                 }
                 A2p[q] = f2_pack(al[0], al[1]);
                 nrAp[q] = f2_pack(nr[0], nr[1]);
-                hp[q] = f2_pack(0.f, 0.f);
-            }
-            if (a.dynamic && seg > 0) {
-                // wait for the end state of the previous segment of this chain
-                bool got = true;
-                if (tid == 0) {
-                    got = false;
-                    for (uint32_t i = 0; i < (1u << 22); ++i) {
-                        if (ld_acquire_gpu(&a.flags[chain]) >= static_cast<unsigned int>(seg)) {
-                            got = true;
-                            break;
-                        }
-                        __nanosleep(64);
-                    }
-                    if (!got)
-                        raise_device_error(2u);
-                }
-                __syncthreads();
-                const float *cp = a.carry + (static_cast<size_t>(chain) * CPB + cl) * NS + n0;
-#pragma unroll
-                for (int q = 0; q < NP; q += 2) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4 *>(cp + 2 * q));
-                    hp[q] = f2_pack(v.x, v.y);
-                    hp[q + 1] = f2_pack(v.z, v.w);
-                }
+                hp[q] = carry_in ? f2_pack(sm.hinit[s][cl][n0 + 2 * q], sm.hinit[s][cl][n0 + 2 * q + 1])
+                                 : f2_pack(0.f, 0.f);
             }
         }
 
@@ -339,90 +449,99 @@ __global__ void __launch_bounds__(kScanThreads, 2)
         const IO(*xs)[CPB] = sm.x[s];
         const IO(*dts)[CPB] = sm.dt[s];
         const IO(*zs)[CPB] = sm.z[s];
-        IO(*ys)[CPB] = sm.y[ci % 3];
-        const float(*bc)[2][NS] = sm.bc[ci & 1];
+        IO(*yw)[CPW] = sm.y[warp][c % 3];
+        const float(*bc)[2][NS] = sm.bc[s];
 
-        float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
-        if (CONV) {
-            xm3 = tr::to_f(xs[0][cl]);
-            xm2 = tr::to_f(xs[1][cl]);
-            xm1 = tr::to_f(xs[2][cl]);
-        }
-        // scalars of token j (advances the conv history by one token)
-        auto scalars = [&](int j) {
-            TokScalars r;
-            const float zv = a.has_z ? tr::to_f(zs[j][cl]) : 0.0f;
-            float pre;
+        if constexpr (TPC == 2) {
+            // token pairs (p, p+1): this thread computes the scalars of token
+            // p + half -- its own token -- and writes that token's output
+            float xw0 = 0.f, xw1 = 0.f, xw2 = 0.f, xw3 = 0.f;  // rows own..own+3 (tokens own-3..own)
+            auto xrow = [&](int r) { return tr::to_f(xs[r < XR ? r : XR - 1][cl]); };
             if (CONV) {
-                const float x0 = tr::to_f(xs[j + kHalo][cl]);
-                pre = fmaf(w0, xm3, cb);
-                pre = fmaf(w1, xm2, pre);
-                pre = fmaf(w2, xm1, pre);
-                pre = fmaf(w3, x0, pre);
-                xm3 = xm2;
-                xm2 = xm1;
-                xm1 = x0;
-            } else {
-                pre = tr::to_f(xs[j][cl]);
+                xw0 = xrow(half);
+                xw1 = xrow(half + 1);
+                xw2 = xrow(half + 2);
+                xw3 = xrow(half + 3);
             }
-            if (TPC == 2) {
-                // the two threads of a channel take one SiLU each and swap
-                const float v = (CONV && half == 0) ? pre : zv;
-                const float sv = silu_fast(v);
-                const float other = __shfl_xor_sync(0xffffffffu, sv, 1);
-                r.u = CONV ? (half == 0 ? sv : other) : pre;
-                r.g = a.has_z ? (CONV ? (half == 0 ? other : sv) : sv) : 1.0f;
-            } else {
-                r.u = CONV ? silu_fast(pre) : pre;
-                r.g = a.has_z ? silu_fast(zv) : 1.0f;
-            }
-            r.delta = softplus_fast(tr::to_f(dts[j][cl]) + bias);
-            return r;
-        };
-
-        TokScalars cur = scalars(0);
-#pragma unroll 2
-        for (int j = 0; j < tcount; ++j) {
-            const TokScalars nxt = scalars(j + 1 < tcount ? j + 1 : j);
-            const f2_t dd = f2_pack(cur.delta, cur.delta);
-            const f2_t uu = f2_pack(cur.u, cur.u);
-            const f2_t du = f2_mul(dd, uu);
-            f2_t acc = f2_pack(0.f, 0.f);
-            const ulonglong2 *Bq = reinterpret_cast<const ulonglong2 *>(&bc[j][0][n0]);
-            const ulonglong2 *Cq = reinterpret_cast<const ulonglong2 *>(&bc[j][1][n0]);
-#pragma unroll
-            for (int q2 = 0; q2 < NP / 2; ++q2) {
-                const ulonglong2 Bv = Bq[q2];
-                const ulonglong2 Cv = Cq[q2];
-                const f2_t Bp[2] = {Bv.x, Bv.y};
-                const f2_t Cp[2] = {Cv.x, Cv.y};
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int q = 2 * q2 + e;
-                    const f2_t dA = f2_mul(dd, A2p[q]);
-                    float d0, d1;
-                    f2_unpack(dA, d0, d1);
-                    const f2_t ab = f2_pack(ex2_approx(d0), ex2_approx(d1));
-                    if (ZOH) {
-                        // h' = abar*h + (abar-1)*k, k = B u / A; with nk = -k:
-                        // h' = abar*(h - nk) + nk
-                        const f2_t nk = f2_mul(nrAp[q], f2_mul(uu, Bp[e]));
-                        hp[q] = f2_fma(ab, f2_sub(hp[q], nk), nk);
-                    } else {
-                        hp[q] = f2_fma(ab, hp[q], f2_mul(du, Bp[e]));
-                    }
-                    acc = f2_fma(hp[q], Cp[e], acc);
+            // scalars of this thread's token of pair p; advances the window
+            auto own_scalars = [&](int p, float &u, float &delta, float &g) {
+                const int j = p + half;
+                const int jr = j < tcount ? j : tcount - 1;
+                if (CONV) {
+                    float pre = fmaf(w0, xw0, cb);
+                    pre = fmaf(w1, xw1, pre);
+                    pre = fmaf(w2, xw2, pre);
+                    pre = fmaf(w3, xw3, pre);
+                    xw0 = xw2;
+                    xw1 = xw3;
+                    xw2 = xrow(j + 4);
+                    xw3 = xrow(j + 5);
+                    u = silu_fast(pre);
+                } else {
+                    u = tr::to_f(xs[jr][cl]);
                 }
+                g = a.has_z ? silu_fast(tr::to_f(zs[jr][cl])) : 1.0f;
+                delta = softplus_fast(tr::to_f(dts[jr][cl]) + bias);
+            };
+            float u_c, d_c, g_c;
+            own_scalars(0, u_c, d_c, g_c);
+#pragma unroll 1
+            for (int p = 0; p < tcount; p += 2) {
+                float u_n, d_n, g_n;
+                own_scalars(p + 2 < tcount ? p + 2 : p, u_n, d_n, g_n);
+                // swap u and Delta within the channel's thread pair
+                const float u_o = __shfl_xor_sync(0xffffffffu, u_c, 1);
+                const float d_o = __shfl_xor_sync(0xffffffffu, d_c, 1);
+                const float u_e = half ? u_o : u_c, d_e = half ? d_o : d_c;  // token p
+                const float u_d = half ? u_c : u_o, d_d = half ? d_c : d_o;  // token p+1
+                const float acc_e = update(bc[p], u_e, d_e);
+                const float acc_d = (p + 1 < tcount) ? update(bc[p + 1], u_d, d_d) : 0.0f;
+                // each thread finishes its own token: own partial + the partner's
+                const float send = half ? acc_e : acc_d;
+                const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                const float yv = fmaf(Dd, u_c, (half ? acc_d : acc_e) + recv) * g_c;
+                if (p + half < tcount)
+                    yw[p + half][cw] = tr::from_f(yv);
+                u_c = u_n;
+                d_c = d_n;
+                g_c = g_n;
             }
-            float a0, a1;
-            f2_unpack(acc, a0, a1);
-            float yv = a0 + a1;
-            if (TPC == 2)
-                yv += __shfl_xor_sync(0xffffffffu, yv, 1);
-            yv = fmaf(Dd, cur.u, yv) * cur.g;
-            if (half == 0)
-                ys[j][cl] = tr::from_f(yv);
-            cur = nxt;
+        } else {
+            float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
+            if (CONV) {
+                xm3 = tr::to_f(xs[0][cl]);
+                xm2 = tr::to_f(xs[1][cl]);
+                xm1 = tr::to_f(xs[2][cl]);
+            }
+            auto scalars = [&](int j, float &u, float &delta, float &g) {
+                if (CONV) {
+                    const float x0 = tr::to_f(xs[j + kHalo][cl]);
+                    float pre = fmaf(w0, xm3, cb);
+                    pre = fmaf(w1, xm2, pre);
+                    pre = fmaf(w2, xm1, pre);
+                    pre = fmaf(w3, x0, pre);
+                    xm3 = xm2;
+                    xm2 = xm1;
+                    xm1 = x0;
+                    u = silu_fast(pre);
+                } else {
+                    u = tr::to_f(xs[j][cl]);
+                }
+                g = a.has_z ? silu_fast(tr::to_f(zs[j][cl])) : 1.0f;
+                delta = softplus_fast(tr::to_f(dts[j][cl]) + bias);
+            };
+            float u_c, d_c, g_c;
+            scalars(0, u_c, d_c, g_c);
+#pragma unroll 2
+            for (int j = 0; j < tcount; ++j) {
+                float u_n, d_n, g_n;
+                scalars(j + 1 < tcount ? j + 1 : j, u_n, d_n, g_n);
+                const float acc = update(bc[j], u_c, d_c);
+                yw[j][cw] = tr::from_f(fmaf(Dd, u_c, acc) * g_c);
+                u_c = u_n;
+                d_c = d_n;
+                g_c = g_n;
+            }
         }
 
         if (m.w & kMetaLast) {
@@ -435,6 +554,12 @@ __global__ void __launch_bounds__(kScanThreads, 2)
                     f2_unpack(hp[q], v0, v1);
                     f2_unpack(hp[q + 1], v2, v3);
                     __stcg(reinterpret_cast<float4 *>(cp + 2 * q), make_float4(v0, v1, v2, v3));
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();
+                    st_release_gpu(&a.flags[static_cast<size_t>(chain) * kConsumerWarps + warp],
+                                   static_cast<unsigned int>(seg + 1));
                 }
             } else if (live && a.h_final) {
                 float *hf = a.h_final + (static_cast<size_t>(bseq) * a.d + ch) * a.N;
@@ -450,40 +575,22 @@ __global__ void __launch_bounds__(kScanThreads, 2)
             }
         }
 
-        // ---- the next chunk: wait for its stage and stage its B/C rows
-        const int s1 = (ci + 1) % STAGES;
-        const bool got = mbar_wait_bounded(&sm.full[s1], ((ci + 1) / STAGES) & 1, 1u << 24);
-        if (got)
-            stage_bc(s1, (ci + 1) & 1);
+        // release the stage, then store this warp's y tile
         fence_proxy_async_smem();
-        if (__syncthreads_or(!got)) {
-            if (tid == 0)
-                raise_device_error(1u);
-            ok = false;
-        }
-        if (tid == 0) {
-            if ((m.w & kMetaLast) && a.dynamic && seg + 1 < a.nseg) {
-                __threadfence();
-                st_release_gpu(&a.flags[chain], static_cast<unsigned int>(seg + 1));
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&sm.empty[s]);
+            if (c0 + warp * CPW < a.d) {  // a tile's last warps may lie past d
+                tma_store_3d(&tm_y, &sm.y[warp][c % 3][0][0], c0 + warp * CPW, m.y, bseq);
+                bulk_commit_group();
             }
-            tma_store_3d(&tm_y, &sm.y[ci % 3][0][0], c0, m.y, bseq);
-            bulk_commit_group();
-            if (ok)
-                produce(s);
-            // the y buffer written next-but-one chunk must be free again
+            // the buffer written next-but-one chunk must be free again
             bulk_wait_group_read<1>();
         }
-        ++ci;
+        __syncwarp();
     }
-    if (tid == 0) {
-        if (!ok) {
-            // after a failed wait, give the loads still in flight a bounded
-            // chance to land before the shared memory they target is released
-            for (int c = ci + 1; c < p_count; ++c)
-                (void)mbar_wait_bounded(&sm.full[c % STAGES], (c / STAGES) & 1, 1u << 20);
-        }
+    if (lane == 0)
         bulk_wait_group<0>();
-    }
 }
 
 }  // namespace s6
