@@ -304,6 +304,11 @@ __global__ void __launch_bounds__(kScanBlock, 1)
                     tma_load_3d(&sm.craw[s][0], &tm_C, &sm.full[s], 0, t0, up.b);
                 }
             }
+            // Make the previous chunk ready before waiting for a carry: the
+            // unit that publishes it may be this CTA's own previous unit, whose
+            // last chunk the consumers must still be able to run.
+            if (c >= 1)
+                finish(c - 1);
             if (carry_in) {
                 // the predecessor segment publishes one flag per consumer warp
                 bool got = true;
@@ -328,8 +333,6 @@ __global__ void __launch_bounds__(kScanBlock, 1)
                 for (int i = lane; i < CPB * NS / 4; i += 32)
                     dst[i] = __ldcg(src + i);
             }
-            if (c >= 1)
-                finish(c - 1);
             ++k;
         }
         return;
