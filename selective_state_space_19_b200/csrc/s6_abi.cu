@@ -162,7 +162,7 @@ template <typename IO, int NS, int TPC, bool CONV, bool ZOH>
 int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, ScanArgs a,
                   cudaStream_t stream) {
     constexpr int T = sizeof(IO) == 2 ? 32 : 16;
-    constexpr int STAGES = 3;
+    constexpr int STAGES = 2;
     using Sh = s6::ScanShape<NS, TPC, T, CONV>;
     using Smem = s6::ScanSmem<IO, NS, TPC, T, STAGES, CONV>;
     constexpr int CPB = Sh::CPB;

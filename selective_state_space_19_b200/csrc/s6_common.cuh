@@ -141,6 +141,49 @@ __device__ __forceinline__ f2_t f2_sub(f2_t a, f2_t b) {
     return d;
 }
 
+// SiLU of a pair: one MUFU ex2 per element, reciprocal by the same seed and
+// Newton steps as rcp_newton, in packed arithmetic.
+__device__ __forceinline__ f2_t f2_silu_fast(f2_t v) {
+    float v0, v1;
+    f2_unpack(v, v0, v1);
+    const float e0 = ex2_approx(fminf(-v0 * kLog2e, 120.0f));
+    const float e1 = ex2_approx(fminf(-v1 * kLog2e, 120.0f));
+    const f2_t one = f2_pack(1.0f, 1.0f);
+    const f2_t x = f2_add(f2_pack(e0, e1), one);
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    f2_t y = f2_pack(__int_as_float(0x7EF311C0 - __float_as_int(x0)), __int_as_float(0x7EF311C0 - __float_as_int(x1)));
+    const f2_t nx = f2_mul(x, f2_pack(-1.0f, -1.0f));
+    f2_t e = f2_fma(nx, y, one);
+    y = f2_fma(y, e, y);
+    e = f2_fma(nx, y, one);
+    y = f2_fma(y, e, y);
+    e = f2_fma(nx, y, one);
+    y = f2_fma(y, e, y);
+    return f2_mul(v, y);
+}
+
+// softplus of a pair: one MUFU ex2 per element, log1p(e) = e q(e) with the
+// degree-9 polynomial of log1p_over_x_01 in packed arithmetic.
+__device__ __forceinline__ f2_t f2_softplus_fast(f2_t v) {
+    float v0, v1;
+    f2_unpack(v, v0, v1);
+    const f2_t e = f2_pack(ex2_approx(-fabsf(v0) * kLog2e), ex2_approx(-fabsf(v1) * kLog2e));
+#define S6_C2(c) f2_pack(c, c)
+    f2_t q = S6_C2(-0.0032439918722957373f);
+    q = f2_fma(q, e, S6_C2(0.019851312041282654f));
+    q = f2_fma(q, e, S6_C2(-0.056959252804517746f));
+    q = f2_fma(q, e, S6_C2(0.10603626072406769f));
+    q = f2_fma(q, e, S6_C2(-0.15305575728416443f));
+    q = f2_fma(q, e, S6_C2(0.19675932824611664f));
+    q = f2_fma(q, e, S6_C2(-0.24954132735729218f));
+    q = f2_fma(q, e, S6_C2(0.3332996368408203f));
+    q = f2_fma(q, e, S6_C2(-0.4999990165233612f));
+    q = f2_fma(q, e, S6_C2(1.0f));
+#undef S6_C2
+    return f2_fma(e, q, f2_pack(fmaxf(v0, 0.0f), fmaxf(v1, 0.0f)));
+}
+
 // 2^x for a pair x <= 0 on the FMA pipe: x = n + f with n = round(x) taken
 // from the low mantissa bits of x + 1.5*2^23, f in [-1/2, 1/2], 2^f by a
 // degree-6 polynomial (float32 relative error 7.9e-8), scaled by adding n to

@@ -94,7 +94,7 @@ struct ScanShape {
     static constexpr int CPW = 32 / TPC;            // channels per consumer warp
     static constexpr int XR = T + (CONV ? kHalo : 0);
     static_assert(NH % 4 == 0, "states per thread must be a multiple of 4");
-    static_assert(T % 2 == 0, "chunks hold whole token pairs");
+    static_assert(T % 4 == 0, "chunks hold whole token quads");
 };
 
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV>
@@ -131,7 +131,7 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
 constexpr uint32_t kWaitPolls = 1u << 24;
 
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, bool ZOH>
-__global__ void __launch_bounds__(kScanBlock, 1)
+__global__ void __launch_bounds__(kScanBlock, 3)
     s6_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
                    const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -242,6 +242,11 @@ __global__ void __launch_bounds__(kScanBlock, 1)
         int c = 0;
         for (;; ++c) {
             const int s = c % STAGES;
+            // Make the previous chunk ready first: the consumers can start on it
+            // while this warp waits for a free stage or for a carry -- which may
+            // be published by this CTA's own previous unit.
+            if (c >= 1)
+                finish(c - 1);
             if (c >= STAGES) {
                 bool got = true;
                 if (lane == 0)
@@ -277,8 +282,6 @@ __global__ void __launch_bounds__(kScanBlock, 1)
             if (done || !ok) {
                 if (lane == 0)
                     sm.meta[s] = make_int4(-1, 0, 0, kMetaEnd);
-                if (c >= 1)
-                    finish(c - 1);
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&sm.ready[s]);
@@ -304,11 +307,6 @@ __global__ void __launch_bounds__(kScanBlock, 1)
                     tma_load_3d(&sm.craw[s][0], &tm_C, &sm.full[s], 0, t0, up.b);
                 }
             }
-            // Make the previous chunk ready before waiting for a carry: the
-            // unit that publishes it may be this CTA's own previous unit, whose
-            // last chunk the consumers must still be able to run.
-            if (c >= 1)
-                finish(c - 1);
             if (carry_in) {
                 // the predecessor segment publishes one flag per consumer warp
                 bool got = true;
@@ -357,7 +355,7 @@ __global__ void __launch_bounds__(kScanBlock, 1)
         const f2_t dd = f2_pack(delta, delta);
         const f2_t uu = f2_pack(u, u);
         const f2_t du = f2_mul(dd, uu);
-        f2_t acc = f2_pack(0.f, 0.f);
+        f2_t acc = f2_pack(0.f, 0.f), acc_b = f2_pack(0.f, 0.f);
         const ulonglong2 *Bq = reinterpret_cast<const ulonglong2 *>(&bcrow[0][n0]);
         const ulonglong2 *Cq = reinterpret_cast<const ulonglong2 *>(&bcrow[1][n0]);
 #pragma unroll
@@ -381,11 +379,14 @@ __global__ void __launch_bounds__(kScanBlock, 1)
                 } else {
                     hp[q] = f2_fma(ab, hp[q], f2_mul(du, Bp[e]));
                 }
-                acc = f2_fma(hp[q], Cp[e], acc);
+                if (e == 0)
+                    acc = f2_fma(hp[q], Cp[e], acc);
+                else
+                    acc_b = f2_fma(hp[q], Cp[e], acc_b);
             }
         }
         float a0, a1;
-        f2_unpack(acc, a0, a1);
+        f2_unpack(f2_add(acc, acc_b), a0, a1);
         return a0 + a1;
     };
 
@@ -456,58 +457,80 @@ __global__ void __launch_bounds__(kScanBlock, 1)
         const float(*bc)[2][NS] = sm.bc[s];
 
         if constexpr (TPC == 2) {
-            // token pairs (p, p+1): this thread computes the scalars of token
-            // p + half -- its own token -- and writes that token's output
-            float xw0 = 0.f, xw1 = 0.f, xw2 = 0.f, xw3 = 0.f;  // rows own..own+3 (tokens own-3..own)
+            // Tokens in quads (p .. p+3) = pairs (p, p+1), (p+2, p+3).  This
+            // thread owns tokens ja = p + half and jb = ja + 2: it computes their
+            // scalars (packed, one pair of values per instruction) and writes
+            // their outputs.
             auto xrow = [&](int r) { return tr::to_f(xs[r < XR ? r : XR - 1][cl]); };
+            auto srow = [&](const IO(*t)[CPB], int j) { return tr::to_f(t[j < tcount ? j : tcount - 1][cl]); };
+            // conv window: rows ja .. ja+5 hold tokens ja-3 .. jb
+            float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f, r4 = 0.f, r5 = 0.f;
             if (CONV) {
-                xw0 = xrow(half);
-                xw1 = xrow(half + 1);
-                xw2 = xrow(half + 2);
-                xw3 = xrow(half + 3);
+                r0 = xrow(half);
+                r1 = xrow(half + 1);
+                r2 = xrow(half + 2);
+                r3 = xrow(half + 3);
+                r4 = xrow(half + 4);
+                r5 = xrow(half + 5);
             }
-            // scalars of this thread's token of pair p; advances the window
-            auto own_scalars = [&](int p, float &u, float &delta, float &g) {
-                const int j = p + half;
-                const int jr = j < tcount ? j : tcount - 1;
+            const f2_t W0 = f2_pack(w0, w0), W1 = f2_pack(w1, w1), W2 = f2_pack(w2, w2), W3 = f2_pack(w3, w3);
+            const f2_t CB = f2_pack(cb, cb), BIAS = f2_pack(bias, bias);
+            // scalars of this thread's two tokens of quad p; advances the window
+            auto quad_scalars = [&](int p, f2_t &u2, f2_t &d2, f2_t &g2) {
+                const int ja = p + half;
                 if (CONV) {
-                    float pre = fmaf(w0, xw0, cb);
-                    pre = fmaf(w1, xw1, pre);
-                    pre = fmaf(w2, xw2, pre);
-                    pre = fmaf(w3, xw3, pre);
-                    xw0 = xw2;
-                    xw1 = xw3;
-                    xw2 = xrow(j + 4);
-                    xw3 = xrow(j + 5);
-                    u = silu_fast(pre);
+                    f2_t pre = f2_fma(W0, f2_pack(r0, r2), CB);
+                    pre = f2_fma(W1, f2_pack(r1, r3), pre);
+                    pre = f2_fma(W2, f2_pack(r2, r4), pre);
+                    pre = f2_fma(W3, f2_pack(r3, r5), pre);
+                    r0 = r4;
+                    r1 = r5;
+                    r2 = xrow(ja + 6);
+                    r3 = xrow(ja + 7);
+                    r4 = xrow(ja + 8);
+                    r5 = xrow(ja + 9);
+                    u2 = f2_silu_fast(pre);
                 } else {
-                    u = tr::to_f(xs[jr][cl]);
+                    u2 = f2_pack(srow(xs, ja), srow(xs, ja + 2));
                 }
-                g = a.has_z ? silu_fast(tr::to_f(zs[jr][cl])) : 1.0f;
-                delta = softplus_fast(tr::to_f(dts[jr][cl]) + bias);
+                g2 = a.has_z ? f2_silu_fast(f2_pack(srow(zs, ja), srow(zs, ja + 2))) : f2_pack(1.0f, 1.0f);
+                d2 = f2_softplus_fast(f2_add(f2_pack(srow(dts, ja), srow(dts, ja + 2)), BIAS));
             };
-            float u_c, d_c, g_c;
-            own_scalars(0, u_c, d_c, g_c);
+            f2_t u2c, d2c, g2c;
+            quad_scalars(0, u2c, d2c, g2c);
 #pragma unroll 1
-            for (int p = 0; p < tcount; p += 2) {
-                float u_n, d_n, g_n;
-                own_scalars(p + 2 < tcount ? p + 2 : p, u_n, d_n, g_n);
+            for (int p = 0; p < tcount; p += 4) {
+                f2_t u2n, d2n, g2n;
+                quad_scalars(p + 4 < tcount ? p + 4 : p, u2n, d2n, g2n);
+                float ua, ub, da, db, ga, gb;
+                f2_unpack(u2c, ua, ub);
+                f2_unpack(d2c, da, db);
+                f2_unpack(g2c, ga, gb);
                 // swap u and Delta within the channel's thread pair
-                const float u_o = __shfl_xor_sync(0xffffffffu, u_c, 1);
-                const float d_o = __shfl_xor_sync(0xffffffffu, d_c, 1);
-                const float u_e = half ? u_o : u_c, d_e = half ? d_o : d_c;  // token p
-                const float u_d = half ? u_c : u_o, d_d = half ? d_c : d_o;  // token p+1
-                const float acc_e = update(bc[p], u_e, d_e);
-                const float acc_d = (p + 1 < tcount) ? update(bc[p + 1], u_d, d_d) : 0.0f;
-                // each thread finishes its own token: own partial + the partner's
-                const float send = half ? acc_e : acc_d;
-                const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-                const float yv = fmaf(Dd, u_c, (half ? acc_d : acc_e) + recv) * g_c;
+                const float oua = __shfl_xor_sync(0xffffffffu, ua, 1);
+                const float oda = __shfl_xor_sync(0xffffffffu, da, 1);
+                const float oub = __shfl_xor_sync(0xffffffffu, ub, 1);
+                const float odb = __shfl_xor_sync(0xffffffffu, db, 1);
+                const float acc0 = update(bc[p], half ? oua : ua, half ? oda : da);
+                float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+                if (p + 1 < tcount)
+                    acc1 = update(bc[p + 1], half ? ua : oua, half ? da : oda);
+                if (p + 2 < tcount)
+                    acc2 = update(bc[p + 2], half ? oub : ub, half ? odb : db);
+                if (p + 3 < tcount)
+                    acc3 = update(bc[p + 3], half ? ub : oub, half ? db : odb);
+                // each thread finishes its own tokens: own partial + the partner's
+                const float ra = __shfl_xor_sync(0xffffffffu, half ? acc0 : acc1, 1);
+                const float rb = __shfl_xor_sync(0xffffffffu, half ? acc2 : acc3, 1);
+                const float ya = fmaf(Dd, ua, (half ? acc1 : acc0) + ra) * ga;
+                const float yb = fmaf(Dd, ub, (half ? acc3 : acc2) + rb) * gb;
                 if (p + half < tcount)
-                    yw[p + half][cw] = tr::from_f(yv);
-                u_c = u_n;
-                d_c = d_n;
-                g_c = g_n;
+                    yw[p + half][cw] = tr::from_f(ya);
+                if (p + 2 + half < tcount)
+                    yw[p + 2 + half][cw] = tr::from_f(yb);
+                u2c = u2n;
+                d2c = d2n;
+                g2c = g2n;
             }
         } else {
             float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
