@@ -344,10 +344,10 @@ def run_ours(args):
     pk = peaks()
     cfg = dict(SI.CONFIGS[WORKLOAD])
     if args.case == "small":
-        # profiling case: same kernel, distributions, batch and width, 1/8 of the
-        # sequence (25M elements, ~150 MB of inputs: still larger than L2; the
+        # profiling case: same kernel, distributions, batch and width, 1/4 of the
+        # sequence (50M elements, ~300 MB of inputs: larger than L2; the
         # same 384 (sequence, channel-tile) chains as the full workload)
-        cfg.update(L=1024)
+        cfg.update(L=2048)
         args.no_rows = args.no_e2e = args.no_cpu_baseline = True
     zoh = bool(cfg["zoh"])
     over = {k: cfg[k] for k in ("Bt", "L")}
@@ -474,7 +474,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--case", choices=["full", "small"], default="full",
-                    help="small: the workload at L=1024 (for ncu captures)")
+                    help="small: the workload at L=2048 (for ncu captures)")
     ap.add_argument("--no-rows", action="store_true", help="skip the decode-step and standalone-conv rows")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
