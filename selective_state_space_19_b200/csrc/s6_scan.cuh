@@ -51,6 +51,8 @@
 // data-dependent decay), not a contraction.
 #pragma once
 
+#include <type_traits>
+
 #include "s6_common.cuh"
 
 namespace s6 {
@@ -493,45 +495,58 @@ __global__ void __launch_bounds__(kScanBlock, 3)
                 } else {
                     u2 = f2_pack(srow(xs, ja), srow(xs, ja + 2));
                 }
-                g2 = a.has_z ? f2_silu_fast(f2_pack(srow(zs, ja), srow(zs, ja + 2))) : f2_pack(1.0f, 1.0f);
+                // the gate is computed unconditionally and replaced by 1 without z
+                // (a select, not a branch: the z tile is then not loaded)
+                const f2_t gz = f2_silu_fast(f2_pack(srow(zs, ja), srow(zs, ja + 2)));
+                g2 = a.has_z ? gz : f2_pack(1.0f, 1.0f);
                 d2 = f2_softplus_fast(f2_add(f2_pack(srow(dts, ja), srow(dts, ja + 2)), BIAS));
             };
-            f2_t u2c, d2c, g2c;
-            quad_scalars(0, u2c, d2c, g2c);
+            // Full chunks (all but a sequence's last) run without bounds tests,
+            // so that each quad is one basic block the scheduler can interleave.
+            auto run = [&](auto full_tag) {
+                constexpr bool FULL = decltype(full_tag)::value;
+                const int tc = FULL ? T : tcount;
+                f2_t u2c, d2c, g2c;
+                quad_scalars(0, u2c, d2c, g2c);
 #pragma unroll 1
-            for (int p = 0; p < tcount; p += 4) {
-                f2_t u2n, d2n, g2n;
-                quad_scalars(p + 4 < tcount ? p + 4 : p, u2n, d2n, g2n);
-                float ua, ub, da, db, ga, gb;
-                f2_unpack(u2c, ua, ub);
-                f2_unpack(d2c, da, db);
-                f2_unpack(g2c, ga, gb);
-                // swap u and Delta within the channel's thread pair
-                const float oua = __shfl_xor_sync(0xffffffffu, ua, 1);
-                const float oda = __shfl_xor_sync(0xffffffffu, da, 1);
-                const float oub = __shfl_xor_sync(0xffffffffu, ub, 1);
-                const float odb = __shfl_xor_sync(0xffffffffu, db, 1);
-                const float acc0 = update(bc[p], half ? oua : ua, half ? oda : da);
-                float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-                if (p + 1 < tcount)
-                    acc1 = update(bc[p + 1], half ? ua : oua, half ? da : oda);
-                if (p + 2 < tcount)
-                    acc2 = update(bc[p + 2], half ? oub : ub, half ? odb : db);
-                if (p + 3 < tcount)
-                    acc3 = update(bc[p + 3], half ? ub : oub, half ? db : odb);
-                // each thread finishes its own tokens: own partial + the partner's
-                const float ra = __shfl_xor_sync(0xffffffffu, half ? acc0 : acc1, 1);
-                const float rb = __shfl_xor_sync(0xffffffffu, half ? acc2 : acc3, 1);
-                const float ya = fmaf(Dd, ua, (half ? acc1 : acc0) + ra) * ga;
-                const float yb = fmaf(Dd, ub, (half ? acc3 : acc2) + rb) * gb;
-                if (p + half < tcount)
-                    yw[p + half][cw] = tr::from_f(ya);
-                if (p + 2 + half < tcount)
-                    yw[p + 2 + half][cw] = tr::from_f(yb);
-                u2c = u2n;
-                d2c = d2n;
-                g2c = g2n;
-            }
+                for (int p = 0; p < tc; p += 4) {
+                    f2_t u2n, d2n, g2n;
+                    quad_scalars(p + 4 < tc ? p + 4 : p, u2n, d2n, g2n);
+                    float ua, ub, da, db, ga, gb;
+                    f2_unpack(u2c, ua, ub);
+                    f2_unpack(d2c, da, db);
+                    f2_unpack(g2c, ga, gb);
+                    // swap u and Delta within the channel's thread pair
+                    const float oua = __shfl_xor_sync(0xffffffffu, ua, 1);
+                    const float oda = __shfl_xor_sync(0xffffffffu, da, 1);
+                    const float oub = __shfl_xor_sync(0xffffffffu, ub, 1);
+                    const float odb = __shfl_xor_sync(0xffffffffu, db, 1);
+                    const float acc0 = update(bc[p], half ? oua : ua, half ? oda : da);
+                    float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+                    if (FULL || p + 1 < tc)
+                        acc1 = update(bc[p + 1], half ? ua : oua, half ? da : oda);
+                    if (FULL || p + 2 < tc)
+                        acc2 = update(bc[p + 2], half ? oub : ub, half ? odb : db);
+                    if (FULL || p + 3 < tc)
+                        acc3 = update(bc[p + 3], half ? ub : oub, half ? db : odb);
+                    // each thread finishes its own tokens: own partial + the partner's
+                    const float ra = __shfl_xor_sync(0xffffffffu, half ? acc0 : acc1, 1);
+                    const float rb = __shfl_xor_sync(0xffffffffu, half ? acc2 : acc3, 1);
+                    const float ya = fmaf(Dd, ua, (half ? acc1 : acc0) + ra) * ga;
+                    const float yb = fmaf(Dd, ub, (half ? acc3 : acc2) + rb) * gb;
+                    if (FULL || p + half < tc)
+                        yw[p + half][cw] = tr::from_f(ya);
+                    if (FULL || p + 2 + half < tc)
+                        yw[p + 2 + half][cw] = tr::from_f(yb);
+                    u2c = u2n;
+                    d2c = d2n;
+                    g2c = g2n;
+                }
+            };
+            if (tcount == T)
+                run(std::true_type{});
+            else
+                run(std::false_type{});
         } else {
             float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
             if (CONV) {
