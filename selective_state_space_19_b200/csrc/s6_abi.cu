@@ -252,7 +252,7 @@ int launch_scan_n(const s6_dims *dims, const void *x, const void *dt, const void
         return launch_scan_t<IO, 4, 1, CONV, ZOH>(dims, x, dt, z, y, a, st);
     if (dims->d_state <= 8)
         return launch_scan_t<IO, 8, 1, CONV, ZOH>(dims, x, dt, z, y, a, st);
-    return launch_scan_t<IO, 16, 2, CONV, ZOH>(dims, x, dt, z, y, a, st);
+    return launch_scan_t<IO, 16, 4, CONV, ZOH>(dims, x, dt, z, y, a, st);
 }
 
 template <typename IO>

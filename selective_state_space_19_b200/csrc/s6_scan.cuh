@@ -96,7 +96,7 @@ struct ScanShape {
     static constexpr int CPW = 32 / TPC;            // channels per consumer warp
     static constexpr int XR = T + (CONV ? kHalo : 0);
     static_assert(NH % 4 == 0, "states per thread must be a multiple of 4");
-    static_assert(T % 4 == 0, "chunks hold whole token quads");
+    static_assert(T % (2 * TPC) == 0, "chunks hold whole token groups");
 };
 
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV>
@@ -110,6 +110,7 @@ struct ScanSmem {
     IO craw[STAGES][T * NS];
     float bc[STAGES][T][2][NS];        // [stage][token][B|C][n], float32, zero-padded
     float hinit[STAGES][Sh::CPB][NS];  // start state of a unit that begins in the stage
+    float4 xch[kConsumerWarps][32];    // per-lane (u, Delta) of its own tokens (TPC = 4)
     int4 meta[STAGES];                 // {unit, t0, tcount, flags}
     uint64_t full[STAGES];             // TMA bytes landed (producer waits)
     uint64_t ready[STAGES];            // stage complete and converted (consumers wait)
@@ -133,7 +134,7 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
 constexpr uint32_t kWaitPolls = 1u << 24;
 
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, bool ZOH>
-__global__ void __launch_bounds__(kScanBlock, 3)
+__global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
     s6_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
                    const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -341,8 +342,9 @@ __global__ void __launch_bounds__(kScanBlock, 3)
     // ============================================================== consumers
     const int cw = lane / TPC;       // channel within the warp
     const int cl = warp * CPW + cw;  // channel within the CTA tile
-    const int half = (TPC == 2) ? (lane & 1) : 0;
-    const int n0 = half * NH;
+    const int sub = lane % TPC;  // which NH states of the channel this thread holds
+    const int half = (TPC == 2) ? sub : 0;
+    const int n0 = sub * NH;
 
     f2_t hp[NP], A2p[NP], nrAp[NP];
     float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, cb = 0.f, Dd = 0.f, bias = 0.f;
@@ -458,7 +460,94 @@ __global__ void __launch_bounds__(kScanBlock, 3)
         IO(*yw)[CPW] = sm.y[warp][c % 3];
         const float(*bc)[2][NS] = sm.bc[s];
 
-        if constexpr (TPC == 2) {
+        if constexpr (TPC == 4) {
+            // Tokens in octets (p .. p+7).  Lane r of a channel's four threads
+            // owns tokens ja = p + r and jb = ja + 4: it computes their scalars
+            // (packed, one pair of values per instruction), publishes (u, Delta)
+            // of both through shared memory to the channel's other threads,
+            // updates its 4 states for all eight tokens, and after a
+            // reduce-scatter of the eight partial readouts writes its two outputs.
+            const int r = lane & 3;
+            auto xrow = [&](int rr) { return tr::to_f(xs[rr < XR ? rr : XR - 1][cl]); };
+            auto srow = [&](const IO(*t)[CPB], int j) { return tr::to_f(t[j < tcount ? j : tcount - 1][cl]); };
+            const f2_t W0 = f2_pack(w0, w0), W1 = f2_pack(w1, w1), W2 = f2_pack(w2, w2), W3 = f2_pack(w3, w3);
+            const f2_t CB = f2_pack(cb, cb), BIAS = f2_pack(bias, bias);
+            auto oct_scalars = [&](int p, f2_t &u2, f2_t &d2, f2_t &g2) {
+                const int ja = p + r;
+                if (CONV) {
+                    // token j reads x rows j .. j+3 (tokens j-3 .. j)
+                    f2_t pre = f2_fma(W0, f2_pack(xrow(ja), xrow(ja + 4)), CB);
+                    pre = f2_fma(W1, f2_pack(xrow(ja + 1), xrow(ja + 5)), pre);
+                    pre = f2_fma(W2, f2_pack(xrow(ja + 2), xrow(ja + 6)), pre);
+                    pre = f2_fma(W3, f2_pack(xrow(ja + 3), xrow(ja + 7)), pre);
+                    u2 = f2_silu_fast(pre);
+                } else {
+                    u2 = f2_pack(srow(xs, ja), srow(xs, ja + 4));
+                }
+                const f2_t gz = f2_silu_fast(f2_pack(srow(zs, ja), srow(zs, ja + 4)));
+                g2 = a.has_z ? gz : f2_pack(1.0f, 1.0f);
+                d2 = f2_softplus_fast(f2_add(f2_pack(srow(dts, ja), srow(dts, ja + 4)), BIAS));
+            };
+            float4 *xw = sm.xch[warp];
+            const int base = lane & ~3;
+            auto run = [&](auto full_tag) {
+                constexpr bool FULL = decltype(full_tag)::value;
+                const int tc = FULL ? T : tcount;
+                f2_t u2c, d2c, g2c;
+                oct_scalars(0, u2c, d2c, g2c);
+#pragma unroll 1
+                for (int p = 0; p < tc; p += 8) {
+                    f2_t u2n, d2n, g2n;
+                    oct_scalars(p + 8 < tc ? p + 8 : p, u2n, d2n, g2n);
+                    float ua, ub, da, db, ga, gb;
+                    f2_unpack(u2c, ua, ub);
+                    f2_unpack(d2c, da, db);
+                    f2_unpack(g2c, ga, gb);
+                    __syncwarp();  // the previous octet's slots have been read
+                    xw[lane] = make_float4(ua, da, ub, db);
+                    __syncwarp();
+                    float acc[8];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float4 v = xw[base + k];  // tokens p+k and p+4+k
+                        acc[k] = (FULL || p + k < tc) ? update(bc[p + k], v.x, v.y) : 0.0f;
+                        acc[4 + k] = (FULL || p + 4 + k < tc) ? update(bc[p + 4 + k], v.z, v.w) : 0.0f;
+                    }
+                    // reduce-scatter over the channel's four threads: lane r keeps
+                    // the totals of tokens r and 4 + r
+                    float t1[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        // pairs of tokens (2i, 2i+1); keep the one with parity r & 1
+                        const float keep = (r & 1) ? acc[2 * i + 1] : acc[2 * i];
+                        const float send = (r & 1) ? acc[2 * i] : acc[2 * i + 1];
+                        t1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                    }
+                    // t1[i] = token 2i + (r & 1); keep those with bit 1 equal to r's
+                    float t2[2];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const float keep = (r & 2) ? t1[2 * i + 1] : t1[2 * i];
+                        const float send = (r & 2) ? t1[2 * i] : t1[2 * i + 1];
+                        t2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                    }
+                    // t2[0] = token r, t2[1] = token 4 + r
+                    const float ya = fmaf(Dd, ua, t2[0]) * ga;
+                    const float yb = fmaf(Dd, ub, t2[1]) * gb;
+                    if (FULL || p + r < tc)
+                        yw[p + r][cw] = tr::from_f(ya);
+                    if (FULL || p + 4 + r < tc)
+                        yw[p + 4 + r][cw] = tr::from_f(yb);
+                    u2c = u2n;
+                    d2c = d2n;
+                    g2c = g2n;
+                }
+            };
+            if (tcount == T)
+                run(std::true_type{});
+            else
+                run(std::false_type{});
+        } else if constexpr (TPC == 2) {
             // Tokens in quads (p .. p+3) = pairs (p, p+1), (p+2, p+3).  This
             // thread owns tokens ja = p + half and jb = ja + 2: it computes their
             // scalars (packed, one pair of values per instruction) and writes
