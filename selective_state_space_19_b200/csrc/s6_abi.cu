@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -166,6 +167,14 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     using Sh = s6::ScanShape<NS, TPC, T, CONV>;
     using Smem = s6::ScanSmem<IO, NS, TPC, T, STAGES, CONV>;
     constexpr int CPB = Sh::CPB;
+    // TMA destinations and sources must start on 128-byte boundaries
+    static_assert(offsetof(Smem, x) % 128 == 0 && offsetof(Smem, dt) % 128 == 0 && offsetof(Smem, z) % 128 == 0 &&
+                      offsetof(Smem, y) % 128 == 0 && offsetof(Smem, braw) % 128 == 0 &&
+                      offsetof(Smem, craw) % 128 == 0 && sizeof(s6::Tile<IO, Sh::XR, CPB>) % 128 == 0,
+                  "TMA buffers must be 128-byte aligned");
+    static_assert(offsetof(Smem, bc) % 16 == 0 && offsetof(Smem, hinit) % 16 == 0 && offsetof(Smem, xch) % 16 == 0 &&
+                      offsetof(Smem, meta) % 16 == 0 && offsetof(Smem, full) % 8 == 0,
+                  "vector and barrier fields must be aligned");
     const int io = dims->io_dtype;
     const size_t es = io_size(io);
     CUtensorMap tx, tdt, tz, ty, tB, tC;

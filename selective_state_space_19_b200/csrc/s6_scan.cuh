@@ -99,15 +99,21 @@ struct ScanShape {
     static_assert(T % (2 * TPC) == 0, "chunks hold whole token groups");
 };
 
+// A tile moved by TMA: every buffer starts on a 128-byte boundary.
+template <typename E, int R, int C>
+struct alignas(128) Tile {
+    E v[R][C];
+};
+
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV>
 struct ScanSmem {
     using Sh = ScanShape<NS, TPC, T, CONV>;
-    IO x[STAGES][Sh::XR][Sh::CPB];
-    IO dt[STAGES][T][Sh::CPB];
-    IO z[STAGES][T][Sh::CPB];
-    IO y[kConsumerWarps][3][T][Sh::CPW];  // per consumer warp, triple-buffered
-    IO braw[STAGES][T * NS];
-    IO craw[STAGES][T * NS];
+    Tile<IO, Sh::XR, Sh::CPB> x[STAGES];
+    Tile<IO, T, Sh::CPB> dt[STAGES];
+    Tile<IO, T, Sh::CPB> z[STAGES];
+    Tile<IO, T, Sh::CPW> y[kConsumerWarps][3];  // per consumer warp, triple-buffered
+    Tile<IO, 1, T * NS> braw[STAGES];
+    Tile<IO, 1, T * NS> craw[STAGES];
     float bc[STAGES][T][2][NS];        // [stage][token][B|C][n], float32, zero-padded
     float hinit[STAGES][Sh::CPB][NS];  // start state of a unit that begins in the stage
     float4 xch[kConsumerWarps][32];    // per-lane (u, Delta) of its own tokens (TPC = 4)
@@ -203,7 +209,7 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
                     const int rem = j - which * (T * NS / 4);
                     const int tt = rem / (NS / 4);
                     const int n = (rem - tt * (NS / 4)) * 4;
-                    const IO *src = which ? &sm.craw[sp][tt * NS + n] : &sm.braw[sp][tt * NS + n];
+                    const IO *src = which ? &sm.craw[sp].v[0][tt * NS + n] : &sm.braw[sp].v[0][tt * NS + n];
                     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
                     if (tt < m.z) {
                         if constexpr (sizeof(IO) == 2) {
@@ -229,7 +235,7 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
                 float v = 0.0f;
                 if (got && n < a.N && tt < m.z) {
                     if (a.bc_tma) {
-                        v = tr::to_f(which ? sm.craw[sp][tt * a.N + n] : sm.braw[sp][tt * a.N + n]);
+                        v = tr::to_f(which ? sm.craw[sp].v[0][tt * a.N + n] : sm.braw[sp].v[0][tt * a.N + n]);
                     } else {
                         const size_t off = (static_cast<size_t>(up.b) * a.L + m.y + tt) * a.N + n;
                         v = tr::to_f(which ? static_cast<const IO *>(a.C)[off] : static_cast<const IO *>(a.B)[off]);
@@ -301,13 +307,13 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
                 constexpr uint32_t kR = T * CPB * sizeof(IO);
                 const uint32_t kBC = a.bc_tma ? 2u * T * a.N * static_cast<uint32_t>(sizeof(IO)) : 0u;
                 mbar_arrive_expect_tx(&sm.full[s], kX + kR + (a.has_z ? kR : 0u) + kBC);
-                tma_load_3d(&sm.x[s][0][0], &tm_x, &sm.full[s], c0, t0 - (CONV ? kHalo : 0), up.b);
-                tma_load_3d(&sm.dt[s][0][0], &tm_dt, &sm.full[s], c0, t0, up.b);
+                tma_load_3d(&sm.x[s].v[0][0], &tm_x, &sm.full[s], c0, t0 - (CONV ? kHalo : 0), up.b);
+                tma_load_3d(&sm.dt[s].v[0][0], &tm_dt, &sm.full[s], c0, t0, up.b);
                 if (a.has_z)
-                    tma_load_3d(&sm.z[s][0][0], &tm_z, &sm.full[s], c0, t0, up.b);
+                    tma_load_3d(&sm.z[s].v[0][0], &tm_z, &sm.full[s], c0, t0, up.b);
                 if (a.bc_tma) {
-                    tma_load_3d(&sm.braw[s][0], &tm_B, &sm.full[s], 0, t0, up.b);
-                    tma_load_3d(&sm.craw[s][0], &tm_C, &sm.full[s], 0, t0, up.b);
+                    tma_load_3d(&sm.braw[s].v[0][0], &tm_B, &sm.full[s], 0, t0, up.b);
+                    tma_load_3d(&sm.craw[s].v[0][0], &tm_C, &sm.full[s], 0, t0, up.b);
                 }
             }
             if (carry_in) {
@@ -454,10 +460,10 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
 
         // ---------------------------------------------- the chunk's tokens
         const int tcount = m.z;
-        const IO(*xs)[CPB] = sm.x[s];
-        const IO(*dts)[CPB] = sm.dt[s];
-        const IO(*zs)[CPB] = sm.z[s];
-        IO(*yw)[CPW] = sm.y[warp][c % 3];
+        const IO(*xs)[CPB] = sm.x[s].v;
+        const IO(*dts)[CPB] = sm.dt[s].v;
+        const IO(*zs)[CPB] = sm.z[s].v;
+        IO(*yw)[CPW] = sm.y[warp][c % 3].v;
         const float(*bc)[2][NS] = sm.bc[s];
 
         if constexpr (TPC == 4) {
@@ -506,13 +512,18 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
                     __syncwarp();  // the previous octet's slots have been read
                     xw[lane] = make_float4(ua, da, ub, db);
                     __syncwarp();
+                    // the state advances token by token: p .. p+3, then p+4 .. p+7
+                    float4 v[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        v[k] = xw[base + k];  // (u, Delta) of tokens p+k and p+4+k
                     float acc[8];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float4 v = xw[base + k];  // tokens p+k and p+4+k
-                        acc[k] = (FULL || p + k < tc) ? update(bc[p + k], v.x, v.y) : 0.0f;
-                        acc[4 + k] = (FULL || p + 4 + k < tc) ? update(bc[p + 4 + k], v.z, v.w) : 0.0f;
-                    }
+                    for (int k = 0; k < 4; ++k)
+                        acc[k] = (FULL || p + k < tc) ? update(bc[p + k], v[k].x, v[k].y) : 0.0f;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        acc[4 + k] = (FULL || p + 4 + k < tc) ? update(bc[p + 4 + k], v[k].z, v[k].w) : 0.0f;
                     // reduce-scatter over the channel's four threads: lane r keeps
                     // the totals of tokens r and 4 + r
                     float t1[4];
@@ -711,7 +722,7 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
         if (lane == 0) {
             mbar_arrive(&sm.empty[s]);
             if (c0 + warp * CPW < a.d) {  // a tile's last warps may lie past d
-                tma_store_3d(&tm_y, &sm.y[warp][c % 3][0][0], c0 + warp * CPW, m.y, bseq);
+                tma_store_3d(&tm_y, &sm.y[warp][c % 3].v[0][0], c0 + warp * CPW, m.y, bseq);
                 bulk_commit_group();
             }
             // the buffer written next-but-one chunk must be free again
