@@ -215,7 +215,13 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     const int64_t L = dims->seqlen;
     a.tiles = static_cast<int>((dims->d_inner + CPB - 1) / CPB);
     const int64_t chains = dims->batch * a.tiles;
-    const int64_t workers = static_cast<int64_t>(device_sm_count()) * occ;
+    // Every SM gets the same number of persistent CTAs, and no more CTAs run
+    // than there are chains (a CTA beyond that would only wait).
+    const int64_t sms = device_sm_count();
+    int64_t per_sm = occ;
+    while (per_sm > 1 && per_sm * sms > chains)
+        --per_sm;
+    const int64_t workers = sms * per_sm;
     int64_t nseg = 1, seg_len = round_up(static_cast<size_t>(L), T);
     if (chains < 4 * workers && L > 4 * T) {
         const int64_t grid = chains < workers ? chains : workers;

@@ -95,6 +95,7 @@ struct ScanShape {
     static constexpr int CPB = kScanThreads / TPC;  // channels per CTA
     static constexpr int CPW = 32 / TPC;            // channels per consumer warp
     static constexpr int XR = T + (CONV ? kHalo : 0);
+    static constexpr int XPAD = 4;  // rows after the x tile read only for tokens past the chunk
     static_assert(NH % 4 == 0, "states per thread must be a multiple of 4");
     static_assert(T % (2 * TPC) == 0, "chunks hold whole token groups");
 };
@@ -108,7 +109,7 @@ struct alignas(128) Tile {
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV>
 struct ScanSmem {
     using Sh = ScanShape<NS, TPC, T, CONV>;
-    Tile<IO, Sh::XR, Sh::CPB> x[STAGES];
+    Tile<IO, Sh::XR + Sh::XPAD, Sh::CPB> x[STAGES];
     Tile<IO, T, Sh::CPB> dt[STAGES];
     Tile<IO, T, Sh::CPB> z[STAGES];
     Tile<IO, T, Sh::CPW> y[kConsumerWarps][3];  // per consumer warp, triple-buffered
@@ -474,7 +475,7 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
             // updates its 4 states for all eight tokens, and after a
             // reduce-scatter of the eight partial readouts writes its two outputs.
             const int r = lane & 3;
-            auto xrow = [&](int rr) { return tr::to_f(xs[rr < XR ? rr : XR - 1][cl]); };
+            auto xrow = [&](int rr) { return tr::to_f(xs[rr][cl]); };
             auto srow = [&](const IO(*t)[CPB], int j) { return tr::to_f(t[j < tcount ? j : tcount - 1][cl]); };
             const f2_t W0 = f2_pack(w0, w0), W1 = f2_pack(w1, w1), W2 = f2_pack(w2, w2), W3 = f2_pack(w3, w3);
             const f2_t CB = f2_pack(cb, cb), BIAS = f2_pack(bias, bias);
@@ -563,7 +564,7 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
             // thread owns tokens ja = p + half and jb = ja + 2: it computes their
             // scalars (packed, one pair of values per instruction) and writes
             // their outputs.
-            auto xrow = [&](int r) { return tr::to_f(xs[r < XR ? r : XR - 1][cl]); };
+            auto xrow = [&](int r) { return tr::to_f(xs[r][cl]); };
             auto srow = [&](const IO(*t)[CPB], int j) { return tr::to_f(t[j < tcount ? j : tcount - 1][cl]); };
             // conv window: rows ja .. ja+5 hold tokens ja-3 .. jb
             float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f, r4 = 0.f, r5 = 0.f;
@@ -648,41 +649,77 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
             else
                 run(std::false_type{});
         } else {
-            float xm3 = 0.f, xm2 = 0.f, xm1 = 0.f;
+            // One thread per channel.  Tokens in pairs (p, p+1): the scalars of
+            // the next pair are computed in packed form (one pair of values per
+            // instruction) while the state advances through the current pair.
+            // Rows past the chunk (read only for the pair after the last) lie in
+            // the tile's padding, so no index needs clamping.
+            const IO *xp = &xs[0][cl];
+            const IO *dp = &dts[0][cl];
+            const IO *zp = &zs[0][cl];
+            auto ld = [&](const IO *q, int row) { return tr::to_f(q[row * CPB]); };
+            const f2_t W0 = f2_pack(w0, w0), W1 = f2_pack(w1, w1), W2 = f2_pack(w2, w2), W3 = f2_pack(w3, w3);
+            const f2_t CB = f2_pack(cb, cb), BIAS = f2_pack(bias, bias);
+            // conv window: rows p .. p+4 hold tokens p-3 .. p+1
+            float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f, r4 = 0.f;
             if (CONV) {
-                xm3 = tr::to_f(xs[0][cl]);
-                xm2 = tr::to_f(xs[1][cl]);
-                xm1 = tr::to_f(xs[2][cl]);
+                r0 = ld(xp, 0);
+                r1 = ld(xp, 1);
+                r2 = ld(xp, 2);
+                r3 = ld(xp, 3);
+                r4 = ld(xp, 4);
             }
-            auto scalars = [&](int j, float &u, float &delta, float &g) {
+            auto pair_scalars = [&](int p, int pr, f2_t &u2, f2_t &d2, f2_t &g2) {
+                // p: first token of the pair; pr: row index used for dt / z
                 if (CONV) {
-                    const float x0 = tr::to_f(xs[j + kHalo][cl]);
-                    float pre = fmaf(w0, xm3, cb);
-                    pre = fmaf(w1, xm2, pre);
-                    pre = fmaf(w2, xm1, pre);
-                    pre = fmaf(w3, x0, pre);
-                    xm3 = xm2;
-                    xm2 = xm1;
-                    xm1 = x0;
-                    u = silu_fast(pre);
+                    f2_t pre = f2_fma(W0, f2_pack(r0, r1), CB);
+                    pre = f2_fma(W1, f2_pack(r1, r2), pre);
+                    pre = f2_fma(W2, f2_pack(r2, r3), pre);
+                    pre = f2_fma(W3, f2_pack(r3, r4), pre);
+                    r0 = r2;
+                    r1 = r3;
+                    r2 = r4;
+                    r3 = ld(xp, p + 5);
+                    r4 = ld(xp, p + 6);
+                    u2 = f2_silu_fast(pre);
                 } else {
-                    u = tr::to_f(xs[j][cl]);
+                    u2 = f2_pack(ld(xp, pr), ld(xp, pr + 1));
                 }
-                g = a.has_z ? silu_fast(tr::to_f(zs[j][cl])) : 1.0f;
-                delta = softplus_fast(tr::to_f(dts[j][cl]) + bias);
+                const f2_t gz = f2_silu_fast(f2_pack(ld(zp, pr), ld(zp, pr + 1)));
+                g2 = a.has_z ? gz : f2_pack(1.0f, 1.0f);
+                d2 = f2_softplus_fast(f2_add(f2_pack(ld(dp, pr), ld(dp, pr + 1)), BIAS));
             };
-            float u_c, d_c, g_c;
-            scalars(0, u_c, d_c, g_c);
-#pragma unroll 2
-            for (int j = 0; j < tcount; ++j) {
-                float u_n, d_n, g_n;
-                scalars(j + 1 < tcount ? j + 1 : j, u_n, d_n, g_n);
-                const float acc = update(bc[j], u_c, d_c);
-                yw[j][cw] = tr::from_f(fmaf(Dd, u_c, acc) * g_c);
-                u_c = u_n;
-                d_c = d_n;
-                g_c = g_n;
-            }
+            auto run = [&](auto full_tag) {
+                constexpr bool FULL = decltype(full_tag)::value;
+                const int tc = FULL ? T : tcount;
+                // pairs start at even p < tc <= T (T even), so rows p and p+1 of the
+                // dt / z tiles always exist; past tcount they only feed tokens
+                // that are not written
+                f2_t u2c, d2c, g2c;
+                pair_scalars(0, 0, u2c, d2c, g2c);
+#pragma unroll 1
+                for (int p = 0; p < tc; p += 2) {
+                    f2_t u2n, d2n, g2n;
+                    pair_scalars(p + 2, p + 2 < tc ? p + 2 : p, u2n, d2n, g2n);
+                    float u0, u1, d0, d1, g0, g1;
+                    f2_unpack(u2c, u0, u1);
+                    f2_unpack(d2c, d0, d1);
+                    f2_unpack(g2c, g0, g1);
+                    const float acc0 = update(bc[p], u0, d0);
+                    yw[p][cw] = tr::from_f(fmaf(Dd, u0, acc0) * g0);
+                    if (FULL || p + 1 < tc) {
+                        const float acc1 = update(bc[p + 1], u1, d1);
+                        yw[p + 1][cw] = tr::from_f(fmaf(Dd, u1, acc1) * g1);
+                    }
+                    u2c = u2n;
+                    d2c = d2n;
+                    g2c = g2n;
+                }
+            };
+            if (tcount == T)
+                run(std::true_type{});
+            else
+                run(std::false_type{});
         }
 
         if (m.w & kMetaLast) {
