@@ -401,6 +401,59 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
         return a0 + a1;
     };
 
+    // Software-pipelined form: ab[] holds this token's decays; the next
+    // token's decays are issued pair by pair among this token's FMAs, so the
+    // MUFU pipe is fed while the state arithmetic proceeds.
+    f2_t ab[NP];
+    auto decays = [&](float delta) {
+        const f2_t dd = f2_pack(delta, delta);
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            float d0, d1;
+            f2_unpack(f2_mul(dd, A2p[q]), d0, d1);
+            ab[q] = f2_pack(ex2_approx(d0), ex2_approx(d1));
+        }
+    };
+    auto update_pipe = [&](const float(*bcrow)[NS], float u, float delta, float delta_next, auto next_tag) -> float {
+        constexpr bool NEXT = decltype(next_tag)::value;
+        const f2_t uu = f2_pack(u, u);
+        const f2_t du = f2_mul(f2_pack(delta, delta), uu);
+        const f2_t ddn = f2_pack(delta_next, delta_next);
+        f2_t acc = f2_pack(0.f, 0.f), acc_b = f2_pack(0.f, 0.f);
+        const ulonglong2 *Bq = reinterpret_cast<const ulonglong2 *>(&bcrow[0][n0]);
+        const ulonglong2 *Cq = reinterpret_cast<const ulonglong2 *>(&bcrow[1][n0]);
+#pragma unroll
+        for (int q2 = 0; q2 < NP / 2; ++q2) {
+            const ulonglong2 Bv = Bq[q2];
+            const ulonglong2 Cv = Cq[q2];
+            const f2_t Bp[2] = {Bv.x, Bv.y};
+            const f2_t Cp[2] = {Cv.x, Cv.y};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int q = 2 * q2 + e;
+                const f2_t abq = ab[q];
+                if (NEXT) {
+                    float d0, d1;
+                    f2_unpack(f2_mul(ddn, A2p[q]), d0, d1);
+                    ab[q] = f2_pack(ex2_approx(d0), ex2_approx(d1));
+                }
+                if (ZOH) {
+                    const f2_t nk = f2_mul(nrAp[q], f2_mul(uu, Bp[e]));
+                    hp[q] = f2_fma(abq, f2_sub(hp[q], nk), nk);
+                } else {
+                    hp[q] = f2_fma(abq, hp[q], f2_mul(du, Bp[e]));
+                }
+                if (e == 0)
+                    acc = f2_fma(hp[q], Cp[e], acc);
+                else
+                    acc_b = f2_fma(hp[q], Cp[e], acc_b);
+            }
+        }
+        float a0, a1;
+        f2_unpack(f2_add(acc, acc_b), a0, a1);
+        return a0 + a1;
+    };
+
     for (int c = 0;; ++c) {
         const int s = c % STAGES;
         const bool got = mbar_wait_bounded(&sm.ready[s], (c / STAGES) & 1, kWaitPolls);
@@ -697,23 +750,45 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
                 // that are not written
                 f2_t u2c, d2c, g2c;
                 pair_scalars(0, 0, u2c, d2c, g2c);
-#pragma unroll 1
-                for (int p = 0; p < tc; p += 2) {
+                {
+                    float d0, d1;
+                    f2_unpack(d2c, d0, d1);
+                    decays(d0);  // the chunk's first token
+                }
+                // one pair: token p issues token p+1's decays; token p+1 issues
+                // the next pair's first decays when LAST is false
+                auto pair = [&](int p, auto last_tag) {
+                    constexpr bool LAST = decltype(last_tag)::value;
                     f2_t u2n, d2n, g2n;
-                    pair_scalars(p + 2, p + 2 < tc ? p + 2 : p, u2n, d2n, g2n);
-                    float u0, u1, d0, d1, g0, g1;
+                    pair_scalars(p + 2, LAST ? p : p + 2, u2n, d2n, g2n);
+                    float u0, u1, d0, d1, g0, g1, dn0, dn1;
                     f2_unpack(u2c, u0, u1);
                     f2_unpack(d2c, d0, d1);
                     f2_unpack(g2c, g0, g1);
-                    const float acc0 = update(bc[p], u0, d0);
+                    f2_unpack(d2n, dn0, dn1);
+                    const float acc0 = update_pipe(bc[p], u0, d0, d1, std::true_type{});
                     yw[p][cw] = tr::from_f(fmaf(Dd, u0, acc0) * g0);
                     if (FULL || p + 1 < tc) {
-                        const float acc1 = update(bc[p + 1], u1, d1);
+                        const float acc1 = update_pipe(bc[p + 1], u1, d1, dn0, std::integral_constant<bool, !LAST>{});
                         yw[p + 1][cw] = tr::from_f(fmaf(Dd, u1, acc1) * g1);
                     }
                     u2c = u2n;
                     d2c = d2n;
                     g2c = g2n;
+                };
+                if (FULL) {
+#pragma unroll 1
+                    for (int p = 0; p < T - 2; p += 2)
+                        pair(p, std::false_type{});
+                    pair(T - 2, std::true_type{});
+                } else {
+#pragma unroll 1
+                    for (int p = 0; p < tc; p += 2) {
+                        if (p + 2 < tc)
+                            pair(p, std::false_type{});
+                        else
+                            pair(p, std::true_type{});
+                    }
                 }
             };
             if (tcount == T)
