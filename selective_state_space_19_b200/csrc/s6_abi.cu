@@ -172,7 +172,7 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
                       offsetof(Smem, y) % 128 == 0 && offsetof(Smem, braw) % 128 == 0 &&
                       offsetof(Smem, craw) % 128 == 0 && sizeof(s6::Tile<IO, Sh::XR, CPB>) % 128 == 0,
                   "TMA buffers must be 128-byte aligned");
-    static_assert(offsetof(Smem, bc) % 16 == 0 && offsetof(Smem, hinit) % 16 == 0 && offsetof(Smem, xch) % 16 == 0 &&
+    static_assert(offsetof(Smem, bc) % 16 == 0 && offsetof(Smem, hinit) % 16 == 0 && offsetof(Smem, tab) % 16 == 0 &&
                       offsetof(Smem, meta) % 16 == 0 && offsetof(Smem, full) % 8 == 0,
                   "vector and barrier fields must be aligned");
     const int io = dims->io_dtype;
@@ -267,7 +267,7 @@ int launch_scan_n(const s6_dims *dims, const void *x, const void *dt, const void
         return launch_scan_t<IO, 4, 1, CONV, ZOH>(dims, x, dt, z, y, a, st);
     if (dims->d_state <= 8)
         return launch_scan_t<IO, 8, 1, CONV, ZOH>(dims, x, dt, z, y, a, st);
-    return launch_scan_t<IO, 16, 4, CONV, ZOH>(dims, x, dt, z, y, a, st);
+    return launch_scan_t<IO, 16, 2, CONV, ZOH>(dims, x, dt, z, y, a, st);
 }
 
 template <typename IO>
