@@ -172,7 +172,7 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
                       offsetof(Smem, y) % 128 == 0 && offsetof(Smem, braw) % 128 == 0 &&
                       offsetof(Smem, craw) % 128 == 0 && sizeof(s6::Tile<IO, Sh::XR, CPB>) % 128 == 0,
                   "TMA buffers must be 128-byte aligned");
-    static_assert(offsetof(Smem, bc) % 16 == 0 && offsetof(Smem, hinit) % 16 == 0 && offsetof(Smem, tab) % 16 == 0 &&
+    static_assert(offsetof(Smem, bc) % 16 == 0 && offsetof(Smem, hinit) % 16 == 0 && offsetof(Smem, xch) % 16 == 0 &&
                       offsetof(Smem, meta) % 16 == 0 && offsetof(Smem, full) % 8 == 0,
                   "vector and barrier fields must be aligned");
     const int io = dims->io_dtype;
