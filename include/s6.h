@@ -90,7 +90,8 @@ typedef enum {
     S6_ERR_UNSUPPORTED = -2, /* N > 16, K outside [2,4], unknown dtype          */
     S6_ERR_ALIGNMENT = -3,   /* pointer or row not 16-byte aligned              */
     S6_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed            */
-    S6_ERR_TIMEOUT = -5      /* a bounded device-side wait gave up              */
+    S6_ERR_TIMEOUT = -5,     /* a bounded device-side wait gave up              */
+    S6_ERR_SCRATCH_LIMIT = -6 /* fixed scratch too small (s6_conv_scan_fwd_noalloc) */
 } s6_status;
 
 /*
@@ -132,6 +133,40 @@ S6_API int s6_conv_scan_fwd(const s6_dims *dims, const void *x, const float *con
                      const void *dt, const float *A_log, const void *B, const void *C,
                      const float *D, const void *z, const float *dt_bias, int zoh_mode,
                      void *y, float *h_final, s6_stream_t stream);
+
+/*
+ * s6_conv_scan_fwd_noalloc -- s6_conv_scan_fwd for callers that must not
+ * allocate device memory.  The pages have no counterpart: this is a deployment
+ * variant of the same computation, not a step of the method.
+ *
+ * Who needs it: a caller whose device memory is entirely owned by its own
+ * allocator (a framework's caching pool that has reserved the GPU), or a
+ * latency-critical process with a fixed memory plan, cannot let a library call
+ * cudaMalloc on its behalf -- the allocation may fail, block, or synchronise
+ * the device.  s6_conv_scan_fwd may allocate (its carry scratch, on first use
+ * and when a larger problem arrives); this entry point never does.
+ *
+ * Same arguments, layouts and results as s6_conv_scan_fwd.  When the schedule
+ * splits sequences into segments it keeps the segment carries in one fixed
+ * 4 MiB array compiled into the library (every GPU that loads the library holds
+ * it until the process exits), instead of allocated memory.  The carries need
+ * about 4 KiB per (sequence, 64-channel tile) at N = 16; a problem that would
+ * need more than the array holds returns S6_ERR_SCRATCH_LIMIT and enqueues
+ * nothing.  Problems with enough (sequence, tile) pairs to be scheduled without
+ * segments use no scratch at all.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device); make that first call before capturing a stream.  The array is
+ * shared by every call on the device and keeps the last call's contents; the
+ * call clears on its stream what must start at zero.  Calls whose executions
+ * overlap on the GPU (different streams, or different host threads) race on
+ * the array and must be serialised by the caller.
+ */
+S6_API int s6_conv_scan_fwd_noalloc(const s6_dims *dims, const void *x, const float *conv_w,
+                                    const float *conv_b, const void *dt, const float *A_log,
+                                    const void *B, const void *C, const float *D, const void *z,
+                                    const float *dt_bias, int zoh_mode, void *y, float *h_final,
+                                    s6_stream_t stream);
 
 /*
  * causal_conv1d_silu_fwd -- the conv + SiLU alone ("mamba, live":

@@ -7,8 +7,8 @@ hands raw device pointers plus the current CUDA stream to the C ABI declared in
 There is no CPU fallback: if the library is missing, the first call raises.
 
 Functions (same names as the C ABI):
-    s6_scan_fwd, s6_conv_scan_fwd, causal_conv1d_silu_fwd, s6_step,
-    s6_device_status, s6_status_string, s6_version
+    s6_scan_fwd, s6_conv_scan_fwd, s6_conv_scan_fwd_noalloc, causal_conv1d_silu_fwd,
+    s6_step, s6_device_status, s6_status_string, s6_version
 """
 from __future__ import annotations
 
@@ -16,7 +16,7 @@ import ctypes
 import os
 
 __all__ = [
-    "S6Error", "lib", "s6_scan_fwd", "s6_conv_scan_fwd", "causal_conv1d_silu_fwd", "s6_step",
+    "S6Error", "lib", "s6_scan_fwd", "s6_conv_scan_fwd", "s6_conv_scan_fwd_noalloc", "causal_conv1d_silu_fwd", "s6_step",
     "s6_device_status", "s6_status_string", "s6_version", "S6_F32", "S6_BF16", "Dims",
 ]
 
@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libs6_b200.so")
 
 S6_F32, S6_BF16 = 0, 1
 S6_OK, S6_ERR_INVALID_ARG, S6_ERR_UNSUPPORTED, S6_ERR_ALIGNMENT, S6_ERR_CUDA, S6_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+S6_ERR_SCRATCH_LIMIT = -6
 
 
 class Dims(ctypes.Structure):
@@ -56,14 +57,15 @@ def lib() -> ctypes.CDLL:
         DP = ctypes.POINTER(Dims)
         L.s6_scan_fwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P]
         L.s6_conv_scan_fwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P]
+        L.s6_conv_scan_fwd_noalloc.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P]
         L.causal_conv1d_silu_fwd.argtypes = [DP, _P, _P, _P, _P, _P]
         L.s6_step.argtypes = [DP, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.s6_device_status.argtypes = [_P]
         L.s6_status_string.argtypes = [_I]
         L.s6_status_string.restype = ctypes.c_char_p
         L.s6_version.argtypes = []
-        for f in (L.s6_scan_fwd, L.s6_conv_scan_fwd, L.causal_conv1d_silu_fwd, L.s6_step, L.s6_device_status,
-                  L.s6_version):
+        for f in (L.s6_scan_fwd, L.s6_conv_scan_fwd, L.s6_conv_scan_fwd_noalloc, L.causal_conv1d_silu_fwd, L.s6_step,
+                  L.s6_device_status, L.s6_version):
             f.restype = _I
         _lib = L
     return _lib
@@ -164,6 +166,15 @@ def s6_conv_scan_fwd(x, conv_w, conv_b, dt, A_log, B, C, D, z=None, dt_bias=None
                      h_final=None, want_h_final=True, stream=None):
     """Fused causal conv + SiLU + selective scan + gate.  Returns (y, h_final)."""
     return _scan(lib().s6_conv_scan_fwd, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w,
+                 conv_b, want_h_final, stream)
+
+
+def s6_conv_scan_fwd_noalloc(x, conv_w, conv_b, dt, A_log, B, C, D, z=None, dt_bias=None, zoh_mode=0, y=None,
+                             h_final=None, want_h_final=True, stream=None):
+    """s6_conv_scan_fwd for callers that cannot let the library allocate device
+    memory: the segment carries live in a fixed array inside the library.  Pass
+    y and h_final to keep this call free of allocations on the torch side too."""
+    return _scan(lib().s6_conv_scan_fwd_noalloc, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w,
                  conv_b, want_h_final, stream)
 
 

@@ -144,6 +144,12 @@ int get_scratch(size_t bytes, cudaStream_t stream, void **out) {
     return S6_OK;
 }
 
+// A caller-independent scratch region of fixed size (see s6_conv_scan_fwd_noalloc).
+struct FixedScratch {
+    void *ptr;
+    size_t bytes;
+};
+
 int device_sm_count() {
     static int cached[64] = {0};
     int dev = 0;
@@ -161,7 +167,7 @@ size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
 
 template <typename IO, int NS, int TPC, bool CONV, bool ZOH>
 int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, ScanArgs a,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, const FixedScratch *fixed = nullptr) {
     constexpr int T = sizeof(IO) == 2 ? 32 : 16;
     constexpr int STAGES = 2;
     using Sh = s6::ScanShape<NS, TPC, T, CONV>;
@@ -246,9 +252,15 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
         const size_t hdr = round_up(4 + 4 * nflags, 256);
         const size_t carry = static_cast<size_t>(chains) * CPB * NS * sizeof(float);
         void *scr = nullptr;
-        const int st = get_scratch(hdr + carry, stream, &scr);
-        if (st != S6_OK)
-            return st;
+        if (fixed) {
+            if (hdr + carry > fixed->bytes)
+                return S6_ERR_SCRATCH_LIMIT;
+            scr = fixed->ptr;
+        } else {
+            const int st = get_scratch(hdr + carry, stream, &scr);
+            if (st != S6_OK)
+                return st;
+        }
         a.counter = static_cast<unsigned int *>(scr);
         a.flags = a.counter + 1;
         a.carry = reinterpret_cast<float *>(static_cast<char *>(scr) + hdr);
@@ -262,27 +274,28 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
 
 template <typename IO, bool CONV, bool ZOH>
 int launch_scan_n(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, const ScanArgs &a,
-                  cudaStream_t st) {
+                  cudaStream_t st, const FixedScratch *fixed = nullptr) {
     if (dims->d_state <= 4)
-        return launch_scan_t<IO, 4, 1, CONV, ZOH>(dims, x, dt, z, y, a, st);
+        return launch_scan_t<IO, 4, 1, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
     if (dims->d_state <= 8)
-        return launch_scan_t<IO, 8, 1, CONV, ZOH>(dims, x, dt, z, y, a, st);
-    return launch_scan_t<IO, 16, 2, CONV, ZOH>(dims, x, dt, z, y, a, st);
+        return launch_scan_t<IO, 8, 1, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
+    return launch_scan_t<IO, 16, 2, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
 }
 
 template <typename IO>
 int launch_scan_io(const s6_dims *dims, bool conv, bool zoh, const void *x, const void *dt, const void *z, void *y,
-                   const ScanArgs &a, cudaStream_t st) {
+                   const ScanArgs &a, cudaStream_t st, const FixedScratch *fixed = nullptr) {
     if (conv)
-        return zoh ? launch_scan_n<IO, true, true>(dims, x, dt, z, y, a, st)
-                   : launch_scan_n<IO, true, false>(dims, x, dt, z, y, a, st);
-    return zoh ? launch_scan_n<IO, false, true>(dims, x, dt, z, y, a, st)
-               : launch_scan_n<IO, false, false>(dims, x, dt, z, y, a, st);
+        return zoh ? launch_scan_n<IO, true, true>(dims, x, dt, z, y, a, st, fixed)
+                   : launch_scan_n<IO, true, false>(dims, x, dt, z, y, a, st, fixed);
+    return zoh ? launch_scan_n<IO, false, true>(dims, x, dt, z, y, a, st, fixed)
+               : launch_scan_n<IO, false, false>(dims, x, dt, z, y, a, st, fixed);
 }
 
 int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv_w, const float *conv_b,
                 const void *dt, const float *A_log, const void *B, const void *C, const float *D, const void *z,
-                const float *dt_bias, int zoh_mode, void *y, float *h_final, s6_stream_t stream) {
+                const float *dt_bias, int zoh_mode, void *y, float *h_final, s6_stream_t stream,
+                const FixedScratch *fixed = nullptr) {
     int st = check_dims(dims, true, conv);
     if (st != S6_OK)
         return st;
@@ -339,8 +352,8 @@ int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv
     if (use_stream_device(s) != S6_OK)
         return S6_ERR_CUDA;
     if (dims->io_dtype == S6_BF16)
-        return launch_scan_io<__nv_bfloat16>(dims, conv, zoh_mode == 1, x, dt, z, y, a, s);
-    return launch_scan_io<float>(dims, conv, zoh_mode == 1, x, dt, z, y, a, s);
+        return launch_scan_io<__nv_bfloat16>(dims, conv, zoh_mode == 1, x, dt, z, y, a, s, fixed);
+    return launch_scan_io<float>(dims, conv, zoh_mode == 1, x, dt, z, y, a, s, fixed);
 }
 
 // ------------------------------------------------------------ step dispatch
@@ -363,6 +376,37 @@ int launch_step_n(const s6::StepArgs &a, cudaStream_t st) {
     return launch_step_t<IO, 16, ZOH>(a, st);
 }
 
+// ------------------------------------------------ scratch that is never allocated
+// The carry scratch of s6_conv_scan_fwd_noalloc: one fixed array in the
+// library's device image, present on every GPU that loads the library until
+// the process exits.  Host code must not pass this name to a kernel (on the host
+// it only stands for the symbol); its device address is looked up once per
+// device with cudaGetSymbolAddress while that device is current.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_s6_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[64] = {nullptr};
+
+// Device address of the fixed scratch on the device that owns `stream`.
+int noalloc_scratch(cudaStream_t stream, FixedScratch *out) {
+    if (use_stream_device(stream) != S6_OK)
+        return S6_ERR_CUDA;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return S6_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_s6_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return S6_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    out->ptr = g_noalloc_addr[dev];
+    out->bytes = kNoAllocScratchBytes;
+    return S6_OK;
+}
+
 }  // namespace
 
 // ======================================================================= ABI
@@ -378,6 +422,8 @@ const char *s6_status_string(int status) {
         case S6_ERR_ALIGNMENT: return "S6_ERR_ALIGNMENT: pointer or row not 16-byte aligned";
         case S6_ERR_CUDA: return "S6_ERR_CUDA: a CUDA call or kernel launch failed";
         case S6_ERR_TIMEOUT: return "S6_ERR_TIMEOUT: a bounded device-side wait gave up";
+        case S6_ERR_SCRATCH_LIMIT:
+            return "S6_ERR_SCRATCH_LIMIT: the problem needs more carry scratch than the fixed 4 MiB array holds";
         default: return "S6: unknown status";
     }
 }
@@ -394,6 +440,18 @@ int s6_conv_scan_fwd(const s6_dims *dims, const void *x, const float *conv_w, co
                      const float *dt_bias, int zoh_mode, void *y, float *h_final, s6_stream_t stream) {
     return scan_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final,
                        stream);
+}
+
+int s6_conv_scan_fwd_noalloc(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b,
+                             const void *dt, const float *A_log, const void *B, const void *C, const float *D,
+                             const void *z, const float *dt_bias, int zoh_mode, void *y, float *h_final,
+                             s6_stream_t stream) {
+    FixedScratch fx;
+    const int st = noalloc_scratch(reinterpret_cast<cudaStream_t>(stream), &fx);
+    if (st != S6_OK)
+        return st;
+    return scan_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, stream,
+                       &fx);
 }
 
 int causal_conv1d_silu_fwd(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b, void *out,
