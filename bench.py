@@ -285,6 +285,7 @@ def dist_setup(n_gpus):
 
 
 def max_over_ranks(v, world, device):
+    """The slowest rank's time (the job is done when every rank is)."""
     if world == 1:
         return v
     import torch
@@ -292,6 +293,18 @@ def max_over_ranks(v, world, device):
     t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(elems_per_rank, world, total_ms_max, steps):
+    """Whole-job Gelem/s: every rank scans its own batch (weak scaling), the time
+    is the max over ranks of the timed region, divided into `steps` steps."""
+    ms_per_step = total_ms_max / steps
+    return world * elems_per_rank / (ms_per_step * 1e-3) / 1e9, ms_per_step
+
+
+def rank_seed(base_seed, rank):
+    """Each rank draws its own batch of the workload."""
+    return base_seed + rank
 
 
 def barrier(world):
@@ -351,7 +364,7 @@ def run_ours(args):
         args.no_rows = args.no_e2e = args.no_cpu_baseline = True
     zoh = bool(cfg["zoh"])
     over = {k: cfg[k] for k in ("Bt", "L")}
-    inp = SI.scan_inputs(WORKLOAD, seed=cfg["seed"] + rank, **over)  # each rank its own batch (weak scaling)
+    inp = SI.scan_inputs(WORKLOAD, seed=rank_seed(cfg["seed"], rank), **over)  # each rank its own batch
     Bt, L, d, N = cfg["Bt"], cfg["L"], cfg["d"], cfg["N"]
     elems = Bt * L * d
     stream = torch.cuda.Stream(device)
@@ -389,8 +402,7 @@ def run_ours(args):
     total_ms = t_all0.elapsed_time(t_all1)
     launch_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
     total_ms = max_over_ranks(total_ms, world, device)
-    ms_per_step = total_ms / args.steps
-    value = world * elems / (ms_per_step * 1e-3) / 1e9
+    value, ms_per_step = job_throughput(elems, world, total_ms, args.steps)
 
     # roofline of the scan kernel: N exponentials per element on the MUFU pipe
     ex2_per_s = elems * N / (launch_ms * 1e-3)
