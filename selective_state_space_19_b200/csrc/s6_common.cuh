@@ -163,6 +163,24 @@ __device__ __forceinline__ f2_t f2_silu_fast(f2_t v) {
     return f2_mul(v, y);
 }
 
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// SiLU of a pair through the hyperbolic tangent: SiLU(v) = v sigmoid(v) =
+// (v/2)(1 + tanh(v/2)), one MUFU op per element and two packed FMA-pipe ops.
+// tanh.approx carries a relative error of about 2^-11, below the rounding of a
+// bfloat16 output; float32 I/O uses f2_silu_fast instead.
+__device__ __forceinline__ f2_t f2_silu_tanh(f2_t v) {
+    const f2_t hv = f2_mul(v, f2_pack(0.5f, 0.5f));
+    float h0, h1;
+    f2_unpack(hv, h0, h1);
+    const f2_t t = f2_pack(tanh_approx(h0), tanh_approx(h1));
+    return f2_fma(hv, t, hv);
+}
+
 // softplus of a pair: one MUFU ex2 per element, log1p(e) = e q(e) with the
 // degree-9 polynomial of log1p_over_x_01 in packed arithmetic.
 __device__ __forceinline__ f2_t f2_softplus_fast(f2_t v) {

@@ -97,6 +97,7 @@ struct ScanShape {
     static constexpr int XR = T + (CONV ? kHalo : 0);
     static constexpr int XPAD = 4;  // rows after the x tile read only for tokens past the chunk
     static_assert(NH % 4 == 0, "states per thread must be a multiple of 4");
+    static_assert(TPC == 1 || TPC == 2, "one or two threads per channel");
     static_assert(T % (2 * TPC) == 0, "chunks hold whole token groups");
 };
 
@@ -110,14 +111,14 @@ template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV>
 struct ScanSmem {
     using Sh = ScanShape<NS, TPC, T, CONV>;
     Tile<IO, Sh::XR + Sh::XPAD, Sh::CPB> x[STAGES];
-    Tile<IO, T, Sh::CPB> dt[STAGES];
-    Tile<IO, T, Sh::CPB> z[STAGES];
+    Tile<IO, T + Sh::XPAD, Sh::CPB> dt[STAGES];
+    Tile<IO, T + Sh::XPAD, Sh::CPB> z[STAGES];
     Tile<IO, T, Sh::CPW> y[kConsumerWarps][3];  // per consumer warp, triple-buffered
     Tile<IO, 1, T * NS> braw[STAGES];
     Tile<IO, 1, T * NS> craw[STAGES];
     float bc[STAGES][T][2][NS];        // [stage][token][B|C][n], float32, zero-padded
     float hinit[STAGES][Sh::CPB][NS];  // start state of a unit that begins in the stage
-    float4 xch[kConsumerWarps][32];    // per-lane (u, Delta) of its own tokens (TPC = 4)
+    float4 xch[2][kConsumerWarps][32];  // per-lane (u, Delta) of its own tokens, by quad parity
     int4 meta[STAGES];                 // {unit, t0, tcount, flags}
     uint64_t full[STAGES];             // TMA bytes landed (producer waits)
     uint64_t ready[STAGES];            // stage complete and converted (consumers wait)
@@ -141,7 +142,7 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
 constexpr uint32_t kWaitPolls = 1u << 24;
 
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, bool ZOH>
-__global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
+__global__ void __launch_bounds__(kScanBlock, 3)
     s6_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
                    const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -361,46 +362,6 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
     for (int q = 0; q < NP; ++q)
         hp[q] = A2p[q] = nrAp[q] = f2_pack(0.f, 0.f);
 
-    // one token's contribution to this thread's states; returns the partial readout
-    auto update = [&](const float(*bcrow)[NS], float u, float delta) -> float {
-        const f2_t dd = f2_pack(delta, delta);
-        const f2_t uu = f2_pack(u, u);
-        const f2_t du = f2_mul(dd, uu);
-        f2_t acc = f2_pack(0.f, 0.f), acc_b = f2_pack(0.f, 0.f);
-        const ulonglong2 *Bq = reinterpret_cast<const ulonglong2 *>(&bcrow[0][n0]);
-        const ulonglong2 *Cq = reinterpret_cast<const ulonglong2 *>(&bcrow[1][n0]);
-#pragma unroll
-        for (int q2 = 0; q2 < NP / 2; ++q2) {
-            const ulonglong2 Bv = Bq[q2];
-            const ulonglong2 Cv = Cq[q2];
-            const f2_t Bp[2] = {Bv.x, Bv.y};
-            const f2_t Cp[2] = {Cv.x, Cv.y};
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int q = 2 * q2 + e;
-                const f2_t dA = f2_mul(dd, A2p[q]);
-                float d0, d1;
-                f2_unpack(dA, d0, d1);
-                const f2_t ab = f2_pack(ex2_approx(d0), ex2_approx(d1));
-                if (ZOH) {
-                    // h' = abar*h + (abar-1)*k, k = B u / A; with nk = -k:
-                    // h' = abar*(h - nk) + nk
-                    const f2_t nk = f2_mul(nrAp[q], f2_mul(uu, Bp[e]));
-                    hp[q] = f2_fma(ab, f2_sub(hp[q], nk), nk);
-                } else {
-                    hp[q] = f2_fma(ab, hp[q], f2_mul(du, Bp[e]));
-                }
-                if (e == 0)
-                    acc = f2_fma(hp[q], Cp[e], acc);
-                else
-                    acc_b = f2_fma(hp[q], Cp[e], acc_b);
-            }
-        }
-        float a0, a1;
-        f2_unpack(f2_add(acc, acc_b), a0, a1);
-        return a0 + a1;
-    };
-
     // Software-pipelined form: ab[] holds this token's decays; the next
     // token's decays are issued pair by pair among this token's FMAs, so the
     // MUFU pipe is fed while the state arithmetic proceeds.
@@ -520,120 +481,37 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
         IO(*yw)[CPW] = sm.y[warp][c % 3].v;
         const float(*bc)[2][NS] = sm.bc[s];
 
-        if constexpr (TPC == 4) {
-            // Tokens in octets (p .. p+7).  Lane r of a channel's four threads
-            // owns tokens ja = p + r and jb = ja + 4: it computes their scalars
-            // (packed, one pair of values per instruction), publishes (u, Delta)
-            // of both through shared memory to the channel's other threads,
-            // updates its 4 states for all eight tokens, and after a
-            // reduce-scatter of the eight partial readouts writes its two outputs.
-            const int r = lane & 3;
-            auto xrow = [&](int rr) { return tr::to_f(xs[rr][cl]); };
-            auto srow = [&](const IO(*t)[CPB], int j) { return tr::to_f(t[j < tcount ? j : tcount - 1][cl]); };
-            const f2_t W0 = f2_pack(w0, w0), W1 = f2_pack(w1, w1), W2 = f2_pack(w2, w2), W3 = f2_pack(w3, w3);
-            const f2_t CB = f2_pack(cb, cb), BIAS = f2_pack(bias, bias);
-            auto oct_scalars = [&](int p, f2_t &u2, f2_t &d2, f2_t &g2) {
-                const int ja = p + r;
-                if (CONV) {
-                    // token j reads x rows j .. j+3 (tokens j-3 .. j)
-                    f2_t pre = f2_fma(W0, f2_pack(xrow(ja), xrow(ja + 4)), CB);
-                    pre = f2_fma(W1, f2_pack(xrow(ja + 1), xrow(ja + 5)), pre);
-                    pre = f2_fma(W2, f2_pack(xrow(ja + 2), xrow(ja + 6)), pre);
-                    pre = f2_fma(W3, f2_pack(xrow(ja + 3), xrow(ja + 7)), pre);
-                    u2 = f2_silu_fast(pre);
-                } else {
-                    u2 = f2_pack(srow(xs, ja), srow(xs, ja + 4));
-                }
-                const f2_t gz = f2_silu_fast(f2_pack(srow(zs, ja), srow(zs, ja + 4)));
-                g2 = a.has_z ? gz : f2_pack(1.0f, 1.0f);
-                d2 = f2_softplus_fast(f2_add(f2_pack(srow(dts, ja), srow(dts, ja + 4)), BIAS));
-            };
-            float4 *xw = sm.xch[warp];
-            const int base = lane & ~3;
-            auto run = [&](auto full_tag) {
-                constexpr bool FULL = decltype(full_tag)::value;
-                const int tc = FULL ? T : tcount;
-                f2_t u2c, d2c, g2c;
-                oct_scalars(0, u2c, d2c, g2c);
-#pragma unroll 1
-                for (int p = 0; p < tc; p += 8) {
-                    f2_t u2n, d2n, g2n;
-                    oct_scalars(p + 8 < tc ? p + 8 : p, u2n, d2n, g2n);
-                    float ua, ub, da, db, ga, gb;
-                    f2_unpack(u2c, ua, ub);
-                    f2_unpack(d2c, da, db);
-                    f2_unpack(g2c, ga, gb);
-                    __syncwarp();  // the previous octet's slots have been read
-                    xw[lane] = make_float4(ua, da, ub, db);
-                    __syncwarp();
-                    // the state advances token by token: p .. p+3, then p+4 .. p+7
-                    float4 v[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        v[k] = xw[base + k];  // (u, Delta) of tokens p+k and p+4+k
-                    float acc[8];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        acc[k] = (FULL || p + k < tc) ? update(bc[p + k], v[k].x, v[k].y) : 0.0f;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        acc[4 + k] = (FULL || p + 4 + k < tc) ? update(bc[p + 4 + k], v[k].z, v[k].w) : 0.0f;
-                    // reduce-scatter over the channel's four threads: lane r keeps
-                    // the totals of tokens r and 4 + r
-                    float t1[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        // pairs of tokens (2i, 2i+1); keep the one with parity r & 1
-                        const float keep = (r & 1) ? acc[2 * i + 1] : acc[2 * i];
-                        const float send = (r & 1) ? acc[2 * i] : acc[2 * i + 1];
-                        t1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-                    }
-                    // t1[i] = token 2i + (r & 1); keep those with bit 1 equal to r's
-                    float t2[2];
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const float keep = (r & 2) ? t1[2 * i + 1] : t1[2 * i];
-                        const float send = (r & 2) ? t1[2 * i] : t1[2 * i + 1];
-                        t2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-                    }
-                    // t2[0] = token r, t2[1] = token 4 + r
-                    const float ya = fmaf(Dd, ua, t2[0]) * ga;
-                    const float yb = fmaf(Dd, ub, t2[1]) * gb;
-                    if (FULL || p + r < tc)
-                        yw[p + r][cw] = tr::from_f(ya);
-                    if (FULL || p + 4 + r < tc)
-                        yw[p + 4 + r][cw] = tr::from_f(yb);
-                    u2c = u2n;
-                    d2c = d2n;
-                    g2c = g2n;
-                }
-            };
-            if (tcount == T)
-                run(std::true_type{});
-            else
-                run(std::false_type{});
-        } else if constexpr (TPC == 2) {
-            // Tokens in quads (p .. p+3) = pairs (p, p+1), (p+2, p+3).  This
-            // thread owns tokens ja = p + half and jb = ja + 2: it computes their
-            // scalars (packed, one pair of values per instruction) and writes
-            // their outputs.
-            auto xrow = [&](int r) { return tr::to_f(xs[r][cl]); };
-            auto srow = [&](const IO(*t)[CPB], int j) { return tr::to_f(t[j < tcount ? j : tcount - 1][cl]); };
-            // conv window: rows ja .. ja+5 hold tokens ja-3 .. jb
-            float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f, r4 = 0.f, r5 = 0.f;
+        if constexpr (TPC == 2) {
+            // Tokens in quads (p .. p+3).  This thread owns tokens ja = p + half
+            // and jb = ja + 2: it computes their scalars (packed, one pair of
+            // values per instruction), publishes (u, Delta) of both in a per-lane
+            // shared slot, reads the channel's four tokens back in order from
+            // its own and its partner's slot, updates its NH states token by
+            // token -- each update also issuing the next token's decays -- and
+            // after swapping partial readouts writes its two outputs.  Rows past
+            // the chunk lie in the tiles' padding and feed only unwritten tokens.
+            const IO *xq = &xs[half][cl];  // row r: token half + r - 3
+            const IO *dq = &dts[half][cl];
+            const IO *zq = &zs[half][cl];
+            auto ld = [&](const IO *q, int row) { return tr::to_f(q[row * CPB]); };
+            float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f, r4 = 0.f, r5 = 0.f;  // rows p+half .. p+half+5
             if (CONV) {
-                r0 = xrow(half);
-                r1 = xrow(half + 1);
-                r2 = xrow(half + 2);
-                r3 = xrow(half + 3);
-                r4 = xrow(half + 4);
-                r5 = xrow(half + 5);
+                r0 = ld(xq, 0);
+                r1 = ld(xq, 1);
+                r2 = ld(xq, 2);
+                r3 = ld(xq, 3);
+                r4 = ld(xq, 4);
+                r5 = ld(xq, 5);
             }
             const f2_t W0 = f2_pack(w0, w0), W1 = f2_pack(w1, w1), W2 = f2_pack(w2, w2), W3 = f2_pack(w3, w3);
             const f2_t CB = f2_pack(cb, cb), BIAS = f2_pack(bias, bias);
-            // scalars of this thread's two tokens of quad p; advances the window
+            auto silu2 = [&](f2_t v) {
+                if constexpr (sizeof(IO) == 2)
+                    return f2_silu_tanh(v);
+                else
+                    return f2_silu_fast(v);
+            };
             auto quad_scalars = [&](int p, f2_t &u2, f2_t &d2, f2_t &g2) {
-                const int ja = p + half;
                 if (CONV) {
                     f2_t pre = f2_fma(W0, f2_pack(r0, r2), CB);
                     pre = f2_fma(W1, f2_pack(r1, r3), pre);
@@ -641,51 +519,61 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
                     pre = f2_fma(W3, f2_pack(r3, r5), pre);
                     r0 = r4;
                     r1 = r5;
-                    r2 = xrow(ja + 6);
-                    r3 = xrow(ja + 7);
-                    r4 = xrow(ja + 8);
-                    r5 = xrow(ja + 9);
-                    u2 = f2_silu_fast(pre);
+                    r2 = ld(xq, p + 6);
+                    r3 = ld(xq, p + 7);
+                    r4 = ld(xq, p + 8);
+                    r5 = ld(xq, p + 9);
+                    u2 = silu2(pre);
                 } else {
-                    u2 = f2_pack(srow(xs, ja), srow(xs, ja + 2));
+                    u2 = f2_pack(ld(xq, p), ld(xq, p + 2));
                 }
-                // the gate is computed unconditionally and replaced by 1 without z
-                // (a select, not a branch: the z tile is then not loaded)
-                const f2_t gz = f2_silu_fast(f2_pack(srow(zs, ja), srow(zs, ja + 2)));
+                const f2_t gz = silu2(f2_pack(ld(zq, p), ld(zq, p + 2)));
                 g2 = a.has_z ? gz : f2_pack(1.0f, 1.0f);
-                d2 = f2_softplus_fast(f2_add(f2_pack(srow(dts, ja), srow(dts, ja + 2)), BIAS));
+                d2 = f2_softplus_fast(f2_add(f2_pack(ld(dq, p), ld(dq, p + 2)), BIAS));
             };
-            // Full chunks (all but a sequence's last) run without bounds tests,
-            // so that each quad is one basic block the scheduler can interleave.
+            const int base = lane & ~1;
+            // publish this thread's (u, Delta) of its two tokens; read the quad's
+            // four tokens in order: p = slot[base].xy, p+1 = slot[base+1].xy,
+            // p+2 = slot[base].zw, p+3 = slot[base+1].zw
+            auto exchange = [&](int buf, f2_t u2, f2_t d2, float4 &s0, float4 &s1) {
+                float ua, ub, da, db;
+                f2_unpack(u2, ua, ub);
+                f2_unpack(d2, da, db);
+                sm.xch[buf][warp][lane] = make_float4(ua, da, ub, db);
+                __syncwarp();
+                s0 = sm.xch[buf][warp][base];
+                s1 = sm.xch[buf][warp][base + 1];
+            };
             auto run = [&](auto full_tag) {
                 constexpr bool FULL = decltype(full_tag)::value;
                 const int tc = FULL ? T : tcount;
                 f2_t u2c, d2c, g2c;
+                float4 c0s, c1s;
                 quad_scalars(0, u2c, d2c, g2c);
-#pragma unroll 1
-                for (int p = 0; p < tc; p += 4) {
+                exchange(0, u2c, d2c, c0s, c1s);
+                decays(c0s.y);  // the chunk's first token
+                auto quad = [&](int p, int q, auto last_tag) {
+                    constexpr bool LAST = decltype(last_tag)::value;
                     f2_t u2n, d2n, g2n;
-                    quad_scalars(p + 4 < tc ? p + 4 : p, u2n, d2n, g2n);
-                    float ua, ub, da, db, ga, gb;
-                    f2_unpack(u2c, ua, ub);
-                    f2_unpack(d2c, da, db);
-                    f2_unpack(g2c, ga, gb);
-                    // swap u and Delta within the channel's thread pair
-                    const float oua = __shfl_xor_sync(0xffffffffu, ua, 1);
-                    const float oda = __shfl_xor_sync(0xffffffffu, da, 1);
-                    const float oub = __shfl_xor_sync(0xffffffffu, ub, 1);
-                    const float odb = __shfl_xor_sync(0xffffffffu, db, 1);
-                    const float acc0 = update(bc[p], half ? oua : ua, half ? oda : da);
+                    float4 n0s, n1s;
+                    // the last quad of a chunk recomputes its own scalars instead of
+                    // reading rows past the tile's padding (the values go unused)
+                    quad_scalars(LAST ? p : p + 4, u2n, d2n, g2n);
+                    exchange((q + 1) & 1, u2n, d2n, n0s, n1s);
+                    const float acc0 = update_pipe(bc[p], c0s.x, c0s.y, c1s.y, std::true_type{});
                     float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
                     if (FULL || p + 1 < tc)
-                        acc1 = update(bc[p + 1], half ? ua : oua, half ? da : oda);
+                        acc1 = update_pipe(bc[p + 1], c1s.x, c1s.y, c0s.w, std::true_type{});
                     if (FULL || p + 2 < tc)
-                        acc2 = update(bc[p + 2], half ? oub : ub, half ? odb : db);
+                        acc2 = update_pipe(bc[p + 2], c0s.z, c0s.w, c1s.w, std::true_type{});
                     if (FULL || p + 3 < tc)
-                        acc3 = update(bc[p + 3], half ? ub : oub, half ? db : odb);
+                        acc3 = update_pipe(bc[p + 3], c1s.z, c1s.w, n0s.y, std::integral_constant<bool, !LAST>{});
                     // each thread finishes its own tokens: own partial + the partner's
                     const float ra = __shfl_xor_sync(0xffffffffu, half ? acc0 : acc1, 1);
                     const float rb = __shfl_xor_sync(0xffffffffu, half ? acc2 : acc3, 1);
+                    float ua, ub, ga, gb;
+                    f2_unpack(u2c, ua, ub);
+                    f2_unpack(g2c, ga, gb);
                     const float ya = fmaf(Dd, ua, (half ? acc1 : acc0) + ra) * ga;
                     const float yb = fmaf(Dd, ub, (half ? acc3 : acc2) + rb) * gb;
                     if (FULL || p + half < tc)
@@ -693,8 +581,23 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 3)
                     if (FULL || p + 2 + half < tc)
                         yw[p + 2 + half][cw] = tr::from_f(yb);
                     u2c = u2n;
-                    d2c = d2n;
                     g2c = g2n;
+                    c0s = n0s;
+                    c1s = n1s;
+                };
+                if (FULL) {
+#pragma unroll 1
+                    for (int p = 0; p < T - 4; p += 4)
+                        quad(p, p >> 2, std::false_type{});
+                    quad(T - 4, (T - 4) >> 2, std::true_type{});
+                } else {
+#pragma unroll 1
+                    for (int p = 0; p < tc; p += 4) {
+                        if (p + 4 < tc)
+                            quad(p, p >> 2, std::false_type{});
+                        else
+                            quad(p, p >> 2, std::true_type{});
+                    }
                 }
             };
             if (tcount == T)
