@@ -554,12 +554,14 @@ __global__ void __launch_bounds__(kScanBlock, 3)
                 decays(c0s.y);  // the chunk's first token
                 auto quad = [&](int p, int q, auto last_tag) {
                     constexpr bool LAST = decltype(last_tag)::value;
-                    f2_t u2n, d2n, g2n;
-                    float4 n0s, n1s;
-                    // the last quad of a chunk recomputes its own scalars instead of
-                    // reading rows past the tile's padding (the values go unused)
-                    quad_scalars(LAST ? p : p + 4, u2n, d2n, g2n);
-                    exchange((q + 1) & 1, u2n, d2n, n0s, n1s);
+                    // the next quad's scalars (none after a chunk's last quad: its
+                    // last token issues no further decays)
+                    f2_t u2n = u2c, d2n = d2c, g2n = g2c;
+                    float4 n0s = c0s, n1s = c1s;
+                    if (!LAST) {
+                        quad_scalars(p + 4, u2n, d2n, g2n);
+                        exchange((q + 1) & 1, u2n, d2n, n0s, n1s);
+                    }
                     const float acc0 = update_pipe(bc[p], c0s.x, c0s.y, c1s.y, std::true_type{});
                     float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
                     if (FULL || p + 1 < tc)
@@ -662,8 +664,9 @@ __global__ void __launch_bounds__(kScanBlock, 3)
                 // the next pair's first decays when LAST is false
                 auto pair = [&](int p, auto last_tag) {
                     constexpr bool LAST = decltype(last_tag)::value;
-                    f2_t u2n, d2n, g2n;
-                    pair_scalars(p + 2, LAST ? p : p + 2, u2n, d2n, g2n);
+                    f2_t u2n = u2c, d2n = d2c, g2n = g2c;
+                    if (!LAST)  // no next pair after a chunk's last
+                        pair_scalars(p + 2, p + 2, u2n, d2n, g2n);
                     float u0, u1, d0, d1, g0, g1, dn0, dn1;
                     f2_unpack(u2c, u0, u1);
                     f2_unpack(d2c, d0, d1);
