@@ -142,7 +142,7 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
 constexpr uint32_t kWaitPolls = 1u << 24;
 
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, bool ZOH>
-__global__ void __launch_bounds__(kScanBlock, 3)
+__global__ void __launch_bounds__(kScanBlock, 2)
     s6_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
                    const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -588,7 +588,7 @@ __global__ void __launch_bounds__(kScanBlock, 3)
                     c1s = n1s;
                 };
                 if (FULL) {
-#pragma unroll 1
+#pragma unroll 2
                     for (int p = 0; p < T - 4; p += 4)
                         quad(p, p >> 2, std::false_type{});
                     quad(T - 4, (T - 4) >> 2, std::true_type{});
