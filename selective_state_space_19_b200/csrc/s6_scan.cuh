@@ -588,7 +588,7 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                     c1s = n1s;
                 };
                 if (FULL) {
-#pragma unroll 2
+#pragma unroll
                     for (int p = 0; p < T - 4; p += 4)
                         quad(p, p >> 2, std::false_type{});
                     quad(T - 4, (T - 4) >> 2, std::true_type{});
