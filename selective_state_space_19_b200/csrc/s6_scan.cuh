@@ -557,10 +557,16 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                     // the next quad's scalars (none after a chunk's last quad: its
                     // last token issues no further decays)
                     f2_t u2n = u2c, d2n = d2c, g2n = g2c;
-                    float4 n0s = c0s, n1s = c1s;
+                    float dnext = 0.f;
                     if (!LAST) {
                         quad_scalars(p + 4, u2n, d2n, g2n);
-                        exchange((q + 1) & 1, u2n, d2n, n0s, n1s);
+                        // Delta of the next quad's first token (thread `base` owns
+                        // it) for this quad's last update; the full exchange of the
+                        // next quad waits until after the updates, so that no warp
+                        // barrier separates the scalar work from the state updates
+                        float dlo, dhi;
+                        f2_unpack(d2n, dlo, dhi);
+                        dnext = __shfl_sync(0xffffffffu, dlo, base);
                     }
                     const float acc0 = update_pipe(bc[p], c0s.x, c0s.y, c1s.y, std::true_type{});
                     float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
@@ -569,7 +575,7 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                     if (FULL || p + 2 < tc)
                         acc2 = update_pipe(bc[p + 2], c0s.z, c0s.w, c1s.w, std::true_type{});
                     if (FULL || p + 3 < tc)
-                        acc3 = update_pipe(bc[p + 3], c1s.z, c1s.w, n0s.y, std::integral_constant<bool, !LAST>{});
+                        acc3 = update_pipe(bc[p + 3], c1s.z, c1s.w, dnext, std::integral_constant<bool, !LAST>{});
                     // each thread finishes its own tokens: own partial + the partner's
                     const float ra = __shfl_xor_sync(0xffffffffu, half ? acc0 : acc1, 1);
                     const float rb = __shfl_xor_sync(0xffffffffu, half ? acc2 : acc3, 1);
@@ -582,10 +588,10 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                         yw[p + half][cw] = tr::from_f(ya);
                     if (FULL || p + 2 + half < tc)
                         yw[p + 2 + half][cw] = tr::from_f(yb);
+                    if (!LAST)
+                        exchange((q + 1) & 1, u2n, d2n, c0s, c1s);
                     u2c = u2n;
                     g2c = g2n;
-                    c0s = n0s;
-                    c1s = n1s;
                 };
                 if (FULL) {
 #pragma unroll
