@@ -169,7 +169,7 @@ template <typename IO, int NS, int TPC, bool CONV, bool ZOH>
 int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, ScanArgs a,
                   cudaStream_t stream, const FixedScratch *fixed = nullptr) {
     constexpr int T = sizeof(IO) == 2 ? 32 : 16;
-    constexpr int STAGES = TPC == 4 ? 2 : 3;
+    constexpr int STAGES = 3;
     using Sh = s6::ScanShape<NS, TPC, T, CONV>;
     using Smem = s6::ScanSmem<IO, NS, TPC, T, STAGES, CONV>;
     constexpr int CPB = Sh::CPB;
@@ -279,7 +279,7 @@ int launch_scan_n(const s6_dims *dims, const void *x, const void *dt, const void
         return launch_scan_t<IO, 4, 1, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
     if (dims->d_state <= 8)
         return launch_scan_t<IO, 8, 1, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
-    return launch_scan_t<IO, 16, 4, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
+    return launch_scan_t<IO, 16, 2, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
 }
 
 template <typename IO>

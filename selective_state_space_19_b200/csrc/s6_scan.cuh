@@ -61,6 +61,10 @@ constexpr int kConsumerWarps = 4;
 constexpr int kScanThreads = 32 * kConsumerWarps;  // consumer threads
 constexpr int kScanBlock = kScanThreads + 32;      // + one producer warp
 constexpr int kHalo = 3;                           // conv history rows (taps padded to 4)
+#ifndef S6_SCAN_YBUF
+#define S6_SCAN_YBUF 3
+#endif
+constexpr int kYBuf = S6_SCAN_YBUF;  // y tiles per consumer warp
 
 constexpr int kMetaFirst = 1;  // first chunk of its unit
 constexpr int kMetaLast = 2;   // last chunk of its unit
@@ -97,7 +101,7 @@ struct ScanShape {
     static constexpr int XR = T + (CONV ? kHalo : 0);
     static constexpr int XPAD = 4;  // rows after the x tile read only for tokens past the chunk
     static_assert(NH % 4 == 0, "states per thread must be a multiple of 4");
-    static_assert(TPC == 1 || TPC == 2 || TPC == 4, "one, two or four threads per channel");
+    static_assert(TPC == 1 || TPC == 2, "one or two threads per channel");
     static_assert(T % (2 * TPC) == 0, "chunks hold whole token groups");
 };
 
@@ -113,7 +117,7 @@ struct ScanSmem {
     Tile<IO, Sh::XR + Sh::XPAD, Sh::CPB> x[STAGES];
     Tile<IO, T + Sh::XPAD, Sh::CPB> dt[STAGES];
     Tile<IO, T + Sh::XPAD, Sh::CPB> z[STAGES];
-    Tile<IO, T, Sh::CPW> y[kConsumerWarps][3];  // per consumer warp, triple-buffered
+    Tile<IO, T, Sh::CPW> y[kConsumerWarps][kYBuf];  // per consumer warp, rotating
     Tile<IO, 1, T * NS> braw[STAGES];
     Tile<IO, 1, T * NS> craw[STAGES];
     float bc[STAGES][T][2][NS];        // [stage][token][B|C][n], float32, zero-padded
@@ -142,7 +146,7 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
 constexpr uint32_t kWaitPolls = 1u << 24;
 
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, bool ZOH>
-__global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 2)
+__global__ void __launch_bounds__(kScanBlock, 2)
     s6_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
                    const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 2)
     const int cw = lane / TPC;       // channel within the warp
     const int cl = warp * CPW + cw;  // channel within the CTA tile
     const int sub = lane % TPC;  // which NH states of the channel this thread holds
-    const int half = (TPC == 2) ? sub : 0;  // used by TPC == 2
+    const int half = (TPC == 2) ? sub : 0;
     const int n0 = sub * NH;
 
     f2_t hp[NP], A2p[NP], nrAp[NP];
@@ -478,140 +482,10 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 2)
         const IO(*xs)[CPB] = sm.x[s].v;
         const IO(*dts)[CPB] = sm.dt[s].v;
         const IO(*zs)[CPB] = sm.z[s].v;
-        IO(*yw)[CPW] = sm.y[warp][c % 3].v;
+        IO(*yw)[CPW] = sm.y[warp][c % kYBuf].v;
         const float(*bc)[2][NS] = sm.bc[s];
 
-        if constexpr (TPC == 4) {
-            // Tokens in octets (p .. p+7).  Thread r of a channel's four owns
-            // tokens ja = p + r and jb = ja + 4: it computes their scalars
-            // (packed), swaps (u, Delta) with the channel's other threads through
-            // per-lane shared slots, advances its 4 states token by token (each
-            // update also issuing the next token's decays), and after a
-            // reduce-scatter of the eight partial readouts writes its two outputs.
-            const int r = sub;
-            const int base = lane & ~3;
-            const IO *xq = &xs[r][cl];  // row k: x row r + k (token r + k - 3)
-            const IO *dq = &dts[r][cl];
-            const IO *zq = &zs[r][cl];
-            auto ld = [&](const IO *qq, int row) { return tr::to_f(qq[row * CPB]); };
-            const f2_t W0 = f2_pack(w0, w0), W1 = f2_pack(w1, w1), W2 = f2_pack(w2, w2), W3 = f2_pack(w3, w3);
-            const f2_t CB = f2_pack(cb, cb), BIAS = f2_pack(bias, bias);
-            auto silu2 = [&](f2_t v) {
-                if constexpr (sizeof(IO) == 2)
-                    return f2_silu_tanh(v);
-                else
-                    return f2_silu_fast(v);
-            };
-            auto oct_scalars = [&](int p, f2_t &u2, f2_t &d2, f2_t &g2) {
-                if (CONV) {
-                    // token ja reads x rows ja .. ja+3, token jb rows jb .. jb+3
-                    f2_t pre = f2_fma(W0, f2_pack(ld(xq, p), ld(xq, p + 4)), CB);
-                    pre = f2_fma(W1, f2_pack(ld(xq, p + 1), ld(xq, p + 5)), pre);
-                    pre = f2_fma(W2, f2_pack(ld(xq, p + 2), ld(xq, p + 6)), pre);
-                    pre = f2_fma(W3, f2_pack(ld(xq, p + 3), ld(xq, p + 7)), pre);
-                    u2 = silu2(pre);
-                } else {
-                    u2 = f2_pack(ld(xq, p), ld(xq, p + 4));
-                }
-                const f2_t gz = silu2(f2_pack(ld(zq, p), ld(zq, p + 4)));
-                g2 = a.has_z ? gz : f2_pack(1.0f, 1.0f);
-                d2 = f2_softplus_fast(f2_add(f2_pack(ld(dq, p), ld(dq, p + 4)), BIAS));
-            };
-            // slot of lane base+k: (u, Delta) of tokens p+k and p+4+k
-            auto exchange = [&](int buf, f2_t u2, f2_t d2, float4 (&sl)[4]) {
-                float ua, ub, da, db;
-                f2_unpack(u2, ua, ub);
-                f2_unpack(d2, da, db);
-                sm.xch[buf][warp][lane] = make_float4(ua, da, ub, db);
-                __syncwarp();
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    sl[k] = sm.xch[buf][warp][base + k];
-            };
-            auto run = [&](auto full_tag) {
-                constexpr bool FULL = decltype(full_tag)::value;
-                const int tc = FULL ? T : tcount;
-                f2_t u2c, d2c, g2c;
-                float4 sl[4];
-                oct_scalars(0, u2c, d2c, g2c);
-                exchange(0, u2c, d2c, sl);
-                decays(sl[0].y);  // the chunk's first token
-                auto octet = [&](int p, int q, auto last_tag) {
-                    constexpr bool LAST = decltype(last_tag)::value;
-                    f2_t u2n = u2c, d2n = d2c, g2n = g2c;
-                    float dnext = 0.f;
-                    if (!LAST) {
-                        oct_scalars(p + 8, u2n, d2n, g2n);
-                        float dlo, dhi;
-                        f2_unpack(d2n, dlo, dhi);
-                        dnext = __shfl_sync(0xffffffffu, dlo, base);  // Delta of token p+8
-                    }
-                    float acc[8];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float dn = k < 3 ? sl[k + 1].y : sl[0].w;
-                        acc[k] = (FULL || p + k < tc) ? update_pipe(bc[p + k], sl[k].x, sl[k].y, dn, std::true_type{})
-                                                       : 0.0f;
-                    }
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        if (k < 3)
-                            acc[4 + k] = (FULL || p + 4 + k < tc)
-                                             ? update_pipe(bc[p + 4 + k], sl[k].z, sl[k].w, sl[k + 1].w, std::true_type{})
-                                             : 0.0f;
-                        else
-                            acc[7] = (FULL || p + 7 < tc) ? update_pipe(bc[p + 7], sl[3].z, sl[3].w, dnext,
-                                                                        std::integral_constant<bool, !LAST>{})
-                                                          : 0.0f;
-                    }
-                    // reduce-scatter over the channel's four threads: thread r keeps
-                    // the totals of tokens r and 4 + r
-                    float t1[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float keep = (r & 1) ? acc[2 * i + 1] : acc[2 * i];
-                        const float send = (r & 1) ? acc[2 * i] : acc[2 * i + 1];
-                        t1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
-                    }
-                    float t2[2];
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const float keep = (r & 2) ? t1[2 * i + 1] : t1[2 * i];
-                        const float send = (r & 2) ? t1[2 * i] : t1[2 * i + 1];
-                        t2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-                    }
-                    float ua, ub, ga, gb;
-                    f2_unpack(u2c, ua, ub);
-                    f2_unpack(g2c, ga, gb);
-                    if (FULL || p + r < tc)
-                        yw[p + r][cw] = tr::from_f(fmaf(Dd, ua, t2[0]) * ga);
-                    if (FULL || p + 4 + r < tc)
-                        yw[p + 4 + r][cw] = tr::from_f(fmaf(Dd, ub, t2[1]) * gb);
-                    if (!LAST)
-                        exchange((q + 1) & 1, u2n, d2n, sl);
-                    u2c = u2n;
-                    g2c = g2n;
-                };
-                if (FULL) {
-#pragma unroll
-                    for (int p = 0; p < T - 8; p += 8)
-                        octet(p, p >> 3, std::false_type{});
-                    octet(T - 8, (T - 8) >> 3, std::true_type{});
-                } else {
-#pragma unroll 1
-                    for (int p = 0; p < tc; p += 8) {
-                        if (p + 8 < tc)
-                            octet(p, p >> 3, std::false_type{});
-                        else
-                            octet(p, p >> 3, std::true_type{});
-                    }
-                }
-            };
-            if (tcount == T)
-                run(std::true_type{});
-            else
-                run(std::false_type{});
-        } else if constexpr (TPC == 2) {
+        if constexpr (TPC == 2) {
             // Tokens in quads (p .. p+3).  This thread owns tokens ja = p + half
             // and jb = ja + 2: it computes their scalars (packed, one pair of
             // values per instruction), publishes (u, Delta) of both in a per-lane
@@ -876,11 +750,12 @@ __global__ void __launch_bounds__(kScanBlock, TPC == 4 ? 4 : 2)
         if (lane == 0) {
             mbar_arrive(&sm.empty[s]);
             if (c0 + warp * CPW < a.d) {  // a tile's last warps may lie past d
-                tma_store_3d(&tm_y, &sm.y[warp][c % 3].v[0][0], c0 + warp * CPW, m.y, bseq);
+                tma_store_3d(&tm_y, &sm.y[warp][c % kYBuf].v[0][0], c0 + warp * CPW, m.y, bseq);
                 bulk_commit_group();
             }
-            // the buffer written next-but-one chunk must be free again
-            bulk_wait_group_read<1>();
+            // the buffer this warp writes next chunk (stored kYBuf-1 chunks
+            // ago) must have been read by its store
+            bulk_wait_group_read<kYBuf - 1>();
         }
         __syncwarp();
     }
