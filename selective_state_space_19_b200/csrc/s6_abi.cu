@@ -168,8 +168,12 @@ size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
 template <typename IO, int NS, int TPC, bool CONV, bool ZOH>
 int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, ScanArgs a,
                   cudaStream_t stream, const FixedScratch *fixed = nullptr) {
-    constexpr int T = sizeof(IO) == 2 ? 32 : 16;
-    constexpr int STAGES = 3;
+    // Tokens per chunk: 64 (bf16) / 32 (f32).  A
+    // chunk's first decays and first token quad are not overlapped with other
+    // work, so long chunks amortise them; two stages of such chunks (about
+    // 104 KB of shared memory) still leave room for two CTAs per SM.
+    constexpr int T = sizeof(IO) == 2 ? 64 : 32;
+    constexpr int STAGES = 2;
     using Sh = s6::ScanShape<NS, TPC, T, CONV>;
     using Smem = s6::ScanSmem<IO, NS, TPC, T, STAGES, CONV>;
     constexpr int CPB = Sh::CPB;

@@ -62,7 +62,7 @@ constexpr int kScanThreads = 32 * kConsumerWarps;  // consumer threads
 constexpr int kScanBlock = kScanThreads + 32;      // + one producer warp
 constexpr int kHalo = 3;                           // conv history rows (taps padded to 4)
 #ifndef S6_SCAN_YBUF
-#define S6_SCAN_YBUF 3
+#define S6_SCAN_YBUF 2
 #endif
 constexpr int kYBuf = S6_SCAN_YBUF;  // y tiles per consumer warp
 
@@ -598,7 +598,7 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                     g2c = g2n;
                 };
                 if (FULL) {
-#pragma unroll
+#pragma unroll 3
                     for (int p = 0; p < T - 4; p += 4)
                         quad(p, p >> 2, std::false_type{});
                     quad(T - 4, (T - 4) >> 2, std::true_type{});

@@ -65,7 +65,9 @@ def test_noalloc_rejects_problems_beyond_the_array():
     S6_ERR_SCRATCH_LIMIT before anything is enqueued."""
     import torch
     import selective_state_space_19_b200 as S
-    Bt, L, d, N = 16, 256, 4096, 16  # 1024 channel tiles of 64: ~4.2 MB of carries
+    # 1024 (sequence, 64-channel tile) chains, each long enough to be split into
+    # segments: ~4.2 MB of carries
+    Bt, L, d, N = 16, 1024, 4096, 16
     x = torch.zeros(Bt, L, d, dtype=torch.bfloat16, device="cuda")
     Bm = torch.zeros(Bt, L, N, dtype=torch.bfloat16, device="cuda")
     w = torch.zeros(d, 4, device="cuda")
