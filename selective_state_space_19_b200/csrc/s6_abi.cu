@@ -234,8 +234,11 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     const int64_t workers = sms * per_sm;
     int64_t nseg = 1, seg_len = round_up(static_cast<size_t>(L), T);
     if (chains < 4 * workers && L > 4 * T) {
+        // about 16 units per worker: the last, partly filled wave of units is
+        // short next to the whole run (a chain's segments run one after the
+        // other, so at most `chains` units are ever in flight)
         const int64_t grid = chains < workers ? chains : workers;
-        int64_t want = (8 * grid + chains - 1) / chains;
+        int64_t want = (16 * grid + chains - 1) / chains;
         const int64_t max_seg = L / (4 * T);
         if (want > max_seg)
             want = max_seg;
@@ -371,11 +374,69 @@ int launch_step_t(const s6::StepArgs &a, cudaStream_t st) {
     return launch_status(cudaGetLastError());
 }
 
+// N in {4, 8, 16}: the pipelined kernel over persistent CTAs, each walking one
+// contiguous range of (channel tile, sequence) tiles.  BIO: the per-token rows
+// also move by bulk copies (all their runs 16-byte aligned).
+template <typename IO, int NS, bool ZOH, bool BIO>
+int launch_step_bulk(const s6::StepArgs &a, cudaStream_t st) {
+    constexpr int CT = s6::kStepThreads;  // channels per tile
+    static int occ[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return S6_ERR_CUDA;
+    if (!occ[dev]) {
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, s6::s6_step_bulk_kernel<IO, NS, ZOH, BIO>,
+                                                          s6::kStepThreads, 0) != cudaSuccess ||
+            nb < 1)
+            return S6_ERR_CUDA;
+        occ[dev] = nb;
+    }
+    const long long ctiles = (a.d + CT - 1) / CT;
+    const long long ntiles = ctiles * a.Bt;
+    if (ntiles == 0)
+        return S6_OK;
+    const long long max_grid = static_cast<long long>(device_sm_count()) * occ[dev];
+    const long long per = (ntiles + max_grid - 1) / max_grid;  // tiles per CTA, balanced
+    const long long grid = (ntiles + per - 1) / per;
+    if (grid > 0x7fffffffLL || per > 0x7fffffffLL)
+        return S6_ERR_UNSUPPORTED;
+    s6::s6_step_bulk_kernel<IO, NS, ZOH, BIO><<<static_cast<unsigned>(grid), s6::kStepThreads, 0, st>>>(
+        a, static_cast<int>(ctiles), static_cast<int>(per));
+    return launch_status(cudaGetLastError());
+}
+
+// Whether every per-token run of a tile starts and ends on 16 bytes: the rows
+// of u, Delta, z, y and the conv history are [batch, d_inner(, K-1)] with
+// element size es, so d_inner * es must be a multiple of 16 and the base
+// pointers 16-byte aligned.
+bool step_rows_bulk(const s6::StepArgs &a, size_t es) {
+    if ((static_cast<size_t>(a.d) * es) % 16 != 0)
+        return false;
+    const void *p[] = {a.u, a.dt, a.z, a.conv_state, a.y};
+    for (const void *q : p)
+        if (q && !aligned_to(q, 16))
+            return false;
+    return true;
+}
+
+template <typename IO, int NS, bool ZOH>
+int launch_step_bulk_io(const s6::StepArgs &a, cudaStream_t st) {
+    return step_rows_bulk(a, sizeof(IO)) ? launch_step_bulk<IO, NS, ZOH, true>(a, st)
+                                         : launch_step_bulk<IO, NS, ZOH, false>(a, st);
+}
+
 template <typename IO, bool ZOH>
 int launch_step_n(const s6::StepArgs &a, cudaStream_t st) {
-    if (a.N <= 4)
+    if (a.N == 4)
+        return launch_step_bulk_io<IO, 4, ZOH>(a, st);
+    if (a.N == 8)
+        return launch_step_bulk_io<IO, 8, ZOH>(a, st);
+    if (a.N == 16)
+        return launch_step_bulk_io<IO, 16, ZOH>(a, st);
+    if (a.N < 4)
         return launch_step_t<IO, 4, ZOH>(a, st);
-    if (a.N <= 8)
+    if (a.N < 8)
         return launch_step_t<IO, 8, ZOH>(a, st);
     return launch_step_t<IO, 16, ZOH>(a, st);
 }

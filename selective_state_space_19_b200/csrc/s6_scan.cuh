@@ -507,8 +507,7 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                 r4 = ld(xq, 4);
                 r5 = ld(xq, 5);
             }
-            const f2_t W0 = f2_pack(w0, w0), W1 = f2_pack(w1, w1), W2 = f2_pack(w2, w2), W3 = f2_pack(w3, w3);
-            const f2_t CB = f2_pack(cb, cb), BIAS = f2_pack(bias, bias);
+            const f2_t BIAS = f2_pack(bias, bias);
             auto silu2 = [&](f2_t v) {
                 if constexpr (sizeof(IO) == 2)
                     return f2_silu_tanh(v);
@@ -517,10 +516,11 @@ __global__ void __launch_bounds__(kScanBlock, 2)
             };
             auto quad_scalars = [&](int p, f2_t &u2, f2_t &d2, f2_t &g2) {
                 if (CONV) {
-                    f2_t pre = f2_fma(W0, f2_pack(r0, r2), CB);
-                    pre = f2_fma(W1, f2_pack(r1, r3), pre);
-                    pre = f2_fma(W2, f2_pack(r2, r4), pre);
-                    pre = f2_fma(W3, f2_pack(r3, r5), pre);
+                    // the two tokens' taps as scalar FMAs (packing the window
+                    // rows into pairs would cost register moves)
+                    const float pa = fmaf(w3, r3, fmaf(w2, r2, fmaf(w1, r1, fmaf(w0, r0, cb))));
+                    const float pb = fmaf(w3, r5, fmaf(w2, r4, fmaf(w1, r3, fmaf(w0, r2, cb))));
+                    const f2_t pre = f2_pack(pa, pb);
                     r0 = r4;
                     r1 = r5;
                     r2 = ld(xq, p + 6);
