@@ -475,6 +475,44 @@ int noalloc_scratch(cudaStream_t stream, FixedScratch *out) {
 }  // namespace
 
 // ======================================================================= ABI
+// Persistent CTAs (as many as fit on the SMs) over balanced contiguous ranges
+// of (channel tile, sequence, token tile) tiles.
+template <typename IO>
+int launch_conv(const s6_dims *dims, const void *x, s6::ConvArgs a, cudaStream_t st) {
+    using Sh = s6::ConvShape<IO>;
+    auto kern = s6::s6_conv_silu_kernel<IO>;
+    constexpr size_t smem = sizeof(s6::ConvSmem<IO>);
+    static int occ[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return S6_ERR_CUDA;
+    if (!occ[dev]) {
+        int nb = 0;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+                cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, 32 * s6::kConvWarps, smem) != cudaSuccess ||
+            nb < 1)
+            return S6_ERR_CUDA;
+        occ[dev] = nb;
+    }
+    CUtensorMap tx;
+    if (!make_map_3d(&tx, x, dims->io_dtype, dims->batch, dims->seqlen, dims->d_inner, Sh::CC, s6::kConvT + 3))
+        return S6_ERR_CUDA;
+    const long long ctiles = (dims->d_inner + Sh::CC - 1) / Sh::CC;
+    const long long ttiles = (dims->seqlen + s6::kConvT - 1) / s6::kConvT;
+    const long long ntiles = ctiles * dims->batch * ttiles;
+    const long long max_grid = static_cast<long long>(device_sm_count()) * occ[dev];
+    const long long per = (ntiles + max_grid - 1) / max_grid;  // tiles per CTA, balanced
+    const long long grid = (ntiles + per - 1) / per;
+    if (grid > 0x7fffffffLL || per > 0x7fffffffLL || ttiles > 0x7fffffffLL)
+        return S6_ERR_UNSUPPORTED;
+    a.ctiles = static_cast<int>(ctiles);
+    a.ttiles = static_cast<int>(ttiles);
+    a.per_cta = static_cast<int>(per);
+    kern<<<static_cast<unsigned>(grid), 32 * s6::kConvWarps, smem, st>>>(tx, a);
+    return launch_status(cudaGetLastError());
+}
+
 extern "C" {
 
 int s6_version(void) { return (1 << 16) | 0; }
@@ -541,20 +579,10 @@ int causal_conv1d_silu_fwd(const s6_dims *dims, const void *x, const float *conv
     a.conv_w = conv_w;
     a.conv_b = conv_b;
     a.out = out;
-    const int vec = static_cast<int>(16 / io_size(dims->io_dtype));
-    const long long cols = (dims->d_inner + 32LL * vec - 1) / (32LL * vec);
-    const long long rows = (dims->seqlen + 1LL * s6::kConvWarps * s6::kConvRun - 1) / (s6::kConvWarps * s6::kConvRun);
-    if (rows > 65535 || dims->batch > 65535)
-        return S6_ERR_UNSUPPORTED;
-    dim3 grid(static_cast<unsigned>(cols), static_cast<unsigned>(rows), static_cast<unsigned>(dims->batch));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (use_stream_device(s) != S6_OK)
         return S6_ERR_CUDA;
-    if (dims->io_dtype == S6_BF16)
-        s6::s6_conv_silu_kernel<__nv_bfloat16><<<grid, 32 * s6::kConvWarps, 0, s>>>(a);
-    else
-        s6::s6_conv_silu_kernel<float><<<grid, 32 * s6::kConvWarps, 0, s>>>(a);
-    return launch_status(cudaGetLastError());
+    return dims->io_dtype == S6_BF16 ? launch_conv<__nv_bfloat16>(dims, x, a, s) : launch_conv<float>(dims, x, a, s);
 }
 
 int s6_step(const s6_dims *dims, const float *A_log, const float *D, const float *dt_bias, const float *conv_w,
