@@ -415,7 +415,7 @@ def run_ours(args):
             "frac": ex2_per_s / peak_ex2, "traffic": traffic,
             "pipe": "MUFU ex2 (148 SMs x 16/clk x max SM clock)",
             "peak_at_measured_clock": (SMS * MUFU_PER_SM_CLK * ck["sm_mhz"] * 1e6 / 1e12) if ck.get("sm_mhz") else None,
-            "algorithmic_ex2_per_elem": N, "kernel": "s6_scan_kernel<bf16,16,32,3,conv,simplified>",
+            "algorithmic_ex2_per_elem": N, "kernel": "s6_scan_kernel<bf16,16,2,64,2,conv,simplified>",
             "kernel_source_sha": kernel_source_sha(),
             "hbm": {"achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
                     "algorithmic_bytes_per_elem": bpe, "peak_source": pk["source"]}}

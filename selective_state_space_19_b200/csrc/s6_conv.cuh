@@ -28,8 +28,8 @@
 namespace s6 {
 
 constexpr int kConvWarps = 4;
-constexpr int kConvT = 64;      // tokens per tile
-constexpr int kConvStages = 3;
+constexpr int kConvT = 48;      // tokens per tile
+constexpr int kConvStages = 4;
 constexpr uint32_t kConvWaitPolls = 1u << 22;
 
 template <typename IO>
