@@ -74,6 +74,56 @@ def test_streaming_equals_full_forward(io, zoh, cfg):
     np.testing.assert_array_equal(as_f64(from_dev(cs)), rhist)
 
 
+def _shifted(tensor, shift):
+    """A copy of `tensor` placed `shift` elements into a larger buffer: aligned to
+    its element size but not to 16 bytes."""
+    import torch
+    flat = torch.empty(tensor.numel() + shift, dtype=tensor.dtype, device=tensor.device)
+    view = flat[shift:].view(tensor.shape)
+    view.copy_(tensor)
+    return view
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("zoh", [False, True])
+@pytest.mark.parametrize("case", ["n4_bulk_rows", "rows_not_16B_multiple", "rows_misaligned_k2", "n8_k3_ragged"])
+def test_step_row_paths(io, zoh, case):
+    """The step's ways of moving a tile's per-token rows, against the oracle's full
+    forward: N = 4 with bulk-copied rows; d * sizeof(io) not a multiple of 16
+    (rows read with plain loads, results written directly); rows and conv history
+    at element-aligned but not 16-byte-aligned addresses, K = 2 (plain loads
+    again); N = 8, K = 3 with a ragged last channel tile."""
+    import selective_state_space_19_b200 as S
+    import torch
+    cfg = {"n4_bulk_rows": dict(Bt=3, L=12, d=136, N=4, K=4),
+           "rows_not_16B_multiple": dict(Bt=2, L=10, d=202, N=16, K=3),
+           "rows_misaligned_k2": dict(Bt=2, L=10, d=160, N=16, K=2),
+           "n8_k3_ragged": dict(Bt=5, L=9, d=300, N=8, K=3)}[case]
+    shift = 1 if case == "rows_misaligned_k2" else 0
+    inp = SI.scan_inputs("mamba_mini", io=io, seed=71 + cfg["d"], **cfg)
+    Bt, L, d, N, K = (cfg[k] for k in ("Bt", "L", "d", "N", "K"))
+    ry, rh, rhist = O.scan(inp["x"], inp["dt"], inp["A_log"], inp["B"], inp["C"], inp["D"], z=inp["z"],
+                           dt_bias=inp["dt_bias"], zoh=zoh, conv_w=inp["conv_w"], conv_b=inp["conv_b"],
+                           return_state=True)
+    t = dev_inputs(inp)
+    h = torch.zeros(Bt, d, N, device="cuda")
+    cs = torch.zeros(Bt, d, K - 1, device="cuda", dtype=t["x"].dtype)
+    if shift:
+        cs = _shifted(cs, shift)
+    ys = []
+    for s in range(L):
+        tok = {k: t[k][:, s].contiguous() for k in ("x", "dt", "z", "B", "C")}
+        if shift:
+            tok = {k: _shifted(v, shift) for k, v in tok.items()}
+        ys.append(from_dev(_step_gpu(S, t, tok, h, cs, zoh)))
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    y = np.stack([as_f64(v) for v in ys], axis=1)
+    assert_close(y, ry, io, "y")
+    assert_close(h.cpu().numpy(), rh, io, "h_ssm")
+    np.testing.assert_array_equal(as_f64(from_dev(cs)), rhist)
+
+
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_scan_then_step_resume(io):
     """Checkpoint/resume: scan tokens [0, L1) with h_final, then continue with the
