@@ -514,6 +514,8 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                 else
                     return f2_silu_fast(v);
             };
+            float za = ld(zq, 0), zb = ld(zq, 2), da = ld(dq, 0), db = ld(dq, 2);
+            float xa = CONV ? 0.f : ld(xq, 0), xb = CONV ? 0.f : ld(xq, 2);
             auto quad_scalars = [&](int p, f2_t &u2, f2_t &d2, f2_t &g2) {
                 if (CONV) {
                     // the two tokens' taps as scalar FMAs (packing the window
@@ -529,11 +531,20 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                     r5 = ld(xq, p + 9);
                     u2 = silu2(pre);
                 } else {
-                    u2 = f2_pack(ld(xq, p), ld(xq, p + 2));
+                    u2 = f2_pack(xa, xb);
+                    xa = ld(xq, p + 4);
+                    xb = ld(xq, p + 6);
                 }
-                const f2_t gz = silu2(f2_pack(ld(zq, p), ld(zq, p + 2)));
+                const f2_t gz = silu2(f2_pack(za, zb));
                 g2 = a.has_z ? gz : f2_pack(1.0f, 1.0f);
-                d2 = f2_softplus_fast(f2_add(f2_pack(ld(dq, p), ld(dq, p + 2)), BIAS));
+                d2 = f2_softplus_fast(f2_add(f2_pack(da, db), BIAS));
+                // this thread's z and dt rows of the next quad, read one quad
+                // ahead like the conv window (rows past the chunk lie in the
+                // tiles' padding)
+                za = ld(zq, p + 4);
+                zb = ld(zq, p + 6);
+                da = ld(dq, p + 4);
+                db = ld(dq, p + 6);
             };
             const int base = lane & ~1;
             // publish this thread's (u, Delta) of its two tokens; read the quad's
