@@ -251,6 +251,45 @@ def row_decode(device, stream, pk, steps=96, pool=8):
                          "frac": gbs / pk["hbm_gbs"], "algorithmic_bytes_per_elem": bytes_per}}
 
 
+def row_prefill(device, stream, pk, inp_dev, cfg, chunks=4, iters=10):
+    """Chunked prefill of the long_seq workload: the sequence in `chunks` equal
+    parts, each part a s6_conv_scan_fwd_from_state call started from the previous
+    part's h_final and its last K-1 inputs (the first part from zeros)."""
+    import selective_state_space_19_b200 as S
+    import torch
+    Bt, L, d, N, K = cfg["Bt"], cfg["L"], cfg["d"], cfg["N"], cfg["K"]
+    zoh = int(bool(cfg["zoh"]))
+    cuts = [L * i // chunks for i in range(chunks + 1)]
+    t = inp_dev
+    parts, hists = [], []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        parts.append({k: t[k][:, lo:hi].contiguous() for k in ("x", "dt", "z", "B", "C")})
+        hists.append(t["x"][:, hi - (K - 1):hi].transpose(1, 2).contiguous())
+    ys = [torch.empty_like(p["x"]) for p in parts]
+    hs = [torch.empty(Bt, d, N, device=device) for _ in parts]
+
+    def prefill():
+        for i, p in enumerate(parts):
+            S.s6_conv_scan_fwd_from_state(p["x"], t["conv_w"], t["conv_b"], p["dt"], t["A_log"], p["B"], p["C"],
+                                          t["D"], z=p["z"], dt_bias=t["dt_bias"], zoh_mode=zoh,
+                                          h_init=hs[i - 1] if i else None, conv_hist=hists[i - 1] if i else None,
+                                          y=ys[i], h_final=hs[i], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            prefill()
+        ms = time_events(prefill, iters, stream)
+    assert S.s6_device_status(stream=stream, device=device) == 0
+    elems = Bt * L * d
+    ex2_per_s = elems * N / (ms * 1e-3)
+    peak_ex2 = SMS * MUFU_PER_SM_CLK * pk["sm_max_mhz"] * 1e6
+    return {"workload": f"chunked prefill: long_seq in {chunks} parts of {L // chunks} tokens, each started from "
+                        "the previous part's (h, last K-1 inputs) by s6_conv_scan_fwd_from_state",
+            "value": elems / (ms * 1e-3) / 1e9, "unit": "Gelem/s", "ms_per_prefill": ms, "launches": chunks,
+            "roofline": {"bound": "alu", "achieved": ex2_per_s / 1e12, "peak": peak_ex2 / 1e12, "unit": "Tex2/s",
+                         "frac": ex2_per_s / peak_ex2}}
+
+
 def row_conv(device, stream, pk, inp_dev, cfg, iters=20):
     import selective_state_space_19_b200 as S
     import torch
@@ -451,6 +490,7 @@ def run_ours(args):
     if not args.no_rows and rank == 0:
         rows["s6_step"] = row_decode(device, stream, pk)
         rows["causal_conv1d_silu_fwd"] = row_conv(device, stream, pk, t, cfg)
+        rows["s6_conv_scan_fwd_from_state"] = row_prefill(device, stream, pk, t, cfg)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

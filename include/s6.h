@@ -47,8 +47,10 @@
  *     a failed check returns a negative s6_status and enqueues nothing.  A
  *     launch failure returns S6_ERR_CUDA.  No call aborts, traps or prints.
  *  Start state: a full-sequence call starts from h = 0 and a zero conv
- *     history (the conv is left-padded with zeros).
- *  Scratch: s6_scan_fwd and s6_conv_scan_fwd may use a library-owned device
+ *     history (the conv is left-padded with zeros); the _from_state calls
+ *     take both as arguments.
+ *  Scratch: s6_scan_fwd, s6_conv_scan_fwd and their _from_state forms may
+ *     use a library-owned device
  *     buffer for carries between thread blocks (allocated with cudaMalloc on
  *     the first call on a device that needs it, grown on demand, kept until
  *     process exit).  Make that first call before capturing a stream.  Calls
@@ -167,6 +169,35 @@ S6_API int s6_conv_scan_fwd_noalloc(const s6_dims *dims, const void *x, const fl
                                     const void *B, const void *C, const float *D, const void *z,
                                     const float *dt_bias, int zoh_mode, void *y, float *h_final,
                                     s6_stream_t stream);
+
+/*
+ * s6_scan_fwd_from_state, s6_conv_scan_fwd_from_state -- s6_scan_fwd and
+ * s6_conv_scan_fwd continued from a given state instead of zeros: the chunked
+ * form of a prefill, and the bridge between the scan and s6_step.  The state
+ * is what the streaming page carries between tokens ("mamba, live": the
+ * model's memory is h_ssm plus a (K-1)-token conv history per channel;
+ * "Carry context through a selective state", token streaming matching the full
+ * forward): scanning tokens [0, L1) and then [L1, L) from (h_final, the last
+ * K-1 inputs) equals one scan over [0, L).
+ *
+ *  h_init    [Bt,d,N]   f32  state before token 0; NULL = zeros
+ *  conv_hist [Bt,d,K-1] io   the K-1 inputs before token 0, oldest first (the
+ *                            layout of conv_state); NULL = zeros.  Fused form
+ *                            only.
+ *  the rest as s6_scan_fwd / s6_conv_scan_fwd.  h_init and conv_hist need
+ *  only element alignment and must not alias outputs.  With L = 0, h_final
+ *  receives h_init.
+ */
+S6_API int s6_scan_fwd_from_state(const s6_dims *dims, const void *u, const void *dt, const float *A_log,
+                                  const void *B, const void *C, const float *D, const void *z,
+                                  const float *dt_bias, int zoh_mode, const float *h_init, void *y,
+                                  float *h_final, s6_stream_t stream);
+S6_API int s6_conv_scan_fwd_from_state(const s6_dims *dims, const void *x, const float *conv_w,
+                                       const float *conv_b, const void *dt, const float *A_log,
+                                       const void *B, const void *C, const float *D, const void *z,
+                                       const float *dt_bias, int zoh_mode, const float *h_init,
+                                       const void *conv_hist, void *y, float *h_final,
+                                       s6_stream_t stream);
 
 /*
  * causal_conv1d_silu_fwd -- the conv + SiLU alone ("mamba, live":

@@ -7,8 +7,9 @@ hands raw device pointers plus the current CUDA stream to the C ABI declared in
 There is no CPU fallback: if the library is missing, the first call raises.
 
 Functions (same names as the C ABI):
-    s6_scan_fwd, s6_conv_scan_fwd, s6_conv_scan_fwd_noalloc, causal_conv1d_silu_fwd,
-    s6_step, s6_device_status, s6_status_string, s6_version
+    s6_scan_fwd, s6_conv_scan_fwd, s6_conv_scan_fwd_noalloc, s6_scan_fwd_from_state,
+    s6_conv_scan_fwd_from_state, causal_conv1d_silu_fwd, s6_step, s6_device_status,
+    s6_status_string, s6_version
 """
 from __future__ import annotations
 
@@ -16,7 +17,8 @@ import ctypes
 import os
 
 __all__ = [
-    "S6Error", "lib", "s6_scan_fwd", "s6_conv_scan_fwd", "s6_conv_scan_fwd_noalloc", "causal_conv1d_silu_fwd", "s6_step",
+    "S6Error", "lib", "s6_scan_fwd", "s6_conv_scan_fwd", "s6_conv_scan_fwd_noalloc", "s6_scan_fwd_from_state",
+    "s6_conv_scan_fwd_from_state", "causal_conv1d_silu_fwd", "s6_step",
     "s6_device_status", "s6_status_string", "s6_version", "S6_F32", "S6_BF16", "Dims",
 ]
 
@@ -58,14 +60,17 @@ def lib() -> ctypes.CDLL:
         L.s6_scan_fwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P]
         L.s6_conv_scan_fwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P]
         L.s6_conv_scan_fwd_noalloc.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P]
+        L.s6_scan_fwd_from_state.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]
+        L.s6_conv_scan_fwd_from_state.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]
         L.causal_conv1d_silu_fwd.argtypes = [DP, _P, _P, _P, _P, _P]
         L.s6_step.argtypes = [DP, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.s6_device_status.argtypes = [_P]
         L.s6_status_string.argtypes = [_I]
         L.s6_status_string.restype = ctypes.c_char_p
         L.s6_version.argtypes = []
-        for f in (L.s6_scan_fwd, L.s6_conv_scan_fwd, L.s6_conv_scan_fwd_noalloc, L.causal_conv1d_silu_fwd, L.s6_step,
-                  L.s6_device_status, L.s6_version):
+        for f in (L.s6_scan_fwd, L.s6_conv_scan_fwd, L.s6_conv_scan_fwd_noalloc, L.s6_scan_fwd_from_state,
+                  L.s6_conv_scan_fwd_from_state, L.causal_conv1d_silu_fwd, L.s6_step, L.s6_device_status,
+                  L.s6_version):
             f.restype = _I
         _lib = L
     return _lib
@@ -124,7 +129,8 @@ def _check(status, where):
         raise S6Error(status, where)
 
 
-def _scan(fn, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w, conv_b, want_h, stream):
+def _scan(fn, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w, conv_b, want_h, stream,
+          from_state=False, h_init=None, conv_hist=None):
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x/u must be [batch, seqlen, d_inner]")
@@ -149,8 +155,12 @@ def _scan(fn, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w, c
     args += [_ptr(dt, "dt", x.dtype, seq, dev), _ptr(A_log, "A_log", f32, (d, N), dev),
              _ptr(B, "B", x.dtype, (Bt, L, N), dev), _ptr(C, "C", x.dtype, (Bt, L, N), dev),
              _ptr(D, "D", f32, (d,), dev), _ptr(z, "z", x.dtype, seq, dev),
-             _ptr(dt_bias, "dt_bias", f32, (d,), dev), int(zoh_mode), _ptr(y, "y", x.dtype, seq, dev),
-             _ptr(h_final, "h_final", f32, (Bt, d, N), dev), _stream(stream, dev)]
+             _ptr(dt_bias, "dt_bias", f32, (d,), dev), int(zoh_mode)]
+    if from_state:
+        args += [_ptr(h_init, "h_init", f32, (Bt, d, N), dev)]
+        if conv_w is not None:
+            args += [_ptr(conv_hist, "conv_hist", x.dtype, (Bt, d, K - 1), dev)]
+    args += [_ptr(y, "y", x.dtype, seq, dev), _ptr(h_final, "h_final", f32, (Bt, d, N), dev), _stream(stream, dev)]
     _check(fn(*args), fn.__name__)
     return y, h_final
 
@@ -176,6 +186,22 @@ def s6_conv_scan_fwd_noalloc(x, conv_w, conv_b, dt, A_log, B, C, D, z=None, dt_b
     y and h_final to keep this call free of allocations on the torch side too."""
     return _scan(lib().s6_conv_scan_fwd_noalloc, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w,
                  conv_b, want_h_final, stream)
+
+
+def s6_scan_fwd_from_state(u, dt, A_log, B, C, D, z=None, dt_bias=None, zoh_mode=0, h_init=None, y=None,
+                           h_final=None, want_h_final=True, stream=None):
+    """s6_scan_fwd started from the state h_init [Bt, d, N] (None = zeros).  Returns (y, h_final)."""
+    return _scan(lib().s6_scan_fwd_from_state, u, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, None, None,
+                 want_h_final, stream, from_state=True, h_init=h_init)
+
+
+def s6_conv_scan_fwd_from_state(x, conv_w, conv_b, dt, A_log, B, C, D, z=None, dt_bias=None, zoh_mode=0,
+                                h_init=None, conv_hist=None, y=None, h_final=None, want_h_final=True, stream=None):
+    """s6_conv_scan_fwd started from the state h_init [Bt, d, N] and the conv history
+    conv_hist [Bt, d, K-1] (the K-1 inputs before token 0, oldest first; None = zeros).
+    Returns (y, h_final)."""
+    return _scan(lib().s6_conv_scan_fwd_from_state, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w,
+                 conv_b, want_h_final, stream, from_state=True, h_init=h_init, conv_hist=conv_hist)
 
 
 def causal_conv1d_silu_fwd(x, conv_w, conv_b=None, out=None, stream=None):

@@ -165,7 +165,7 @@ int device_sm_count() {
 
 size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
 
-template <typename IO, int NS, int TPC, bool CONV, bool ZOH>
+template <typename IO, int NS, int TPC, bool CONV, bool ZOH, bool INIT>
 int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, ScanArgs a,
                   cudaStream_t stream, const FixedScratch *fixed = nullptr) {
     // Tokens per chunk: 64 (bf16) / 32 (f32).  A
@@ -207,7 +207,7 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     } else {
         tB = tC = tdt;  // never read
     }
-    auto kern = s6::s6_scan_kernel<IO, NS, TPC, T, STAGES, CONV, ZOH>;
+    auto kern = s6::s6_scan_kernel<IO, NS, TPC, T, STAGES, CONV, ZOH, INIT>;
     const size_t smem = sizeof(Smem);
     static int occ = 0;  // resident CTAs per SM for this instantiation
     if (!occ) {
@@ -279,43 +279,55 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     return launch_status(cudaGetLastError());
 }
 
-template <typename IO, bool CONV, bool ZOH>
+template <typename IO, bool CONV, bool ZOH, bool INIT>
 int launch_scan_n(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, const ScanArgs &a,
                   cudaStream_t st, const FixedScratch *fixed = nullptr) {
     if (dims->d_state <= 4)
-        return launch_scan_t<IO, 4, 1, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
+        return launch_scan_t<IO, 4, 1, CONV, ZOH, INIT>(dims, x, dt, z, y, a, st, fixed);
     if (dims->d_state <= 8)
-        return launch_scan_t<IO, 8, 1, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
-    return launch_scan_t<IO, 16, 2, CONV, ZOH>(dims, x, dt, z, y, a, st, fixed);
+        return launch_scan_t<IO, 8, 1, CONV, ZOH, INIT>(dims, x, dt, z, y, a, st, fixed);
+    return launch_scan_t<IO, 16, 2, CONV, ZOH, INIT>(dims, x, dt, z, y, a, st, fixed);
 }
 
 template <typename IO>
 int launch_scan_io(const s6_dims *dims, bool conv, bool zoh, const void *x, const void *dt, const void *z, void *y,
                    const ScanArgs &a, cudaStream_t st, const FixedScratch *fixed = nullptr) {
+    if (a.h_init || a.conv_hist) {
+        if (conv)
+            return zoh ? launch_scan_n<IO, true, true, true>(dims, x, dt, z, y, a, st, fixed)
+                       : launch_scan_n<IO, true, false, true>(dims, x, dt, z, y, a, st, fixed);
+        return zoh ? launch_scan_n<IO, false, true, true>(dims, x, dt, z, y, a, st, fixed)
+                   : launch_scan_n<IO, false, false, true>(dims, x, dt, z, y, a, st, fixed);
+    }
     if (conv)
-        return zoh ? launch_scan_n<IO, true, true>(dims, x, dt, z, y, a, st, fixed)
-                   : launch_scan_n<IO, true, false>(dims, x, dt, z, y, a, st, fixed);
-    return zoh ? launch_scan_n<IO, false, true>(dims, x, dt, z, y, a, st, fixed)
-               : launch_scan_n<IO, false, false>(dims, x, dt, z, y, a, st, fixed);
+        return zoh ? launch_scan_n<IO, true, true, false>(dims, x, dt, z, y, a, st, fixed)
+                   : launch_scan_n<IO, true, false, false>(dims, x, dt, z, y, a, st, fixed);
+    return zoh ? launch_scan_n<IO, false, true, false>(dims, x, dt, z, y, a, st, fixed)
+               : launch_scan_n<IO, false, false, false>(dims, x, dt, z, y, a, st, fixed);
 }
 
 int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv_w, const float *conv_b,
                 const void *dt, const float *A_log, const void *B, const void *C, const float *D, const void *z,
                 const float *dt_bias, int zoh_mode, void *y, float *h_final, s6_stream_t stream,
-                const FixedScratch *fixed = nullptr) {
+                const FixedScratch *fixed = nullptr, const float *h_init = nullptr,
+                const void *conv_hist = nullptr) {
     int st = check_dims(dims, true, conv);
     if (st != S6_OK)
         return st;
     if (zoh_mode != 0 && zoh_mode != 1)
         return S6_ERR_INVALID_ARG;
+    if ((h_init && !aligned_to(h_init, 4)) || (conv_hist && !aligned_to(conv_hist, io_size(dims->io_dtype))))
+        return S6_ERR_ALIGNMENT;
     if (dims->batch == 0 || dims->seqlen == 0) {
-        // nothing to scan; h_final of an empty sequence is the zero start state
+        // nothing to scan; h_final of an empty sequence is the start state
         if (h_final && dims->batch > 0) {
-            if (use_stream_device(reinterpret_cast<cudaStream_t>(stream)) != S6_OK)
+            cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+            if (use_stream_device(s) != S6_OK)
                 return S6_ERR_CUDA;
-            return launch_status(cudaMemsetAsync(h_final, 0,
-                                                 sizeof(float) * dims->batch * dims->d_inner * dims->d_state,
-                                                 reinterpret_cast<cudaStream_t>(stream)));
+            const size_t bytes = sizeof(float) * dims->batch * dims->d_inner * dims->d_state;
+            if (h_init)
+                return launch_status(cudaMemcpyAsync(h_final, h_init, bytes, cudaMemcpyDeviceToDevice, s));
+            return launch_status(cudaMemsetAsync(h_final, 0, bytes, s));
         }
         return S6_OK;
     }
@@ -355,6 +367,8 @@ int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv
     a.conv_b = conv ? conv_b : nullptr;
     a.K = conv ? static_cast<int>(dims->conv_width) : 0;
     a.h_final = h_final;
+    a.h_init = h_init;
+    a.conv_hist = conv ? conv_hist : nullptr;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (use_stream_device(s) != S6_OK)
         return S6_ERR_CUDA;
@@ -555,6 +569,21 @@ int s6_conv_scan_fwd_noalloc(const s6_dims *dims, const void *x, const float *co
         return st;
     return scan_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, stream,
                        &fx);
+}
+
+int s6_scan_fwd_from_state(const s6_dims *dims, const void *u, const void *dt, const float *A_log, const void *B,
+                           const void *C, const float *D, const void *z, const float *dt_bias, int zoh_mode,
+                           const float *h_init, void *y, float *h_final, s6_stream_t stream) {
+    return scan_common(dims, false, u, nullptr, nullptr, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final,
+                       stream, nullptr, h_init, nullptr);
+}
+
+int s6_conv_scan_fwd_from_state(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b,
+                                const void *dt, const float *A_log, const void *B, const void *C, const float *D,
+                                const void *z, const float *dt_bias, int zoh_mode, const float *h_init,
+                                const void *conv_hist, void *y, float *h_final, s6_stream_t stream) {
+    return scan_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, stream,
+                       nullptr, h_init, conv_hist);
 }
 
 int causal_conv1d_silu_fwd(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b, void *out,

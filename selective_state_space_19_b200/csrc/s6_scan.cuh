@@ -69,7 +69,7 @@ constexpr int kYBuf = S6_SCAN_YBUF;  // y tiles per consumer warp
 constexpr int kMetaFirst = 1;  // first chunk of its unit
 constexpr int kMetaLast = 2;   // last chunk of its unit
 constexpr int kMetaEnd = 4;    // no more work
-constexpr int kMetaCarry = 8;  // the unit starts from a published carry
+constexpr int kMetaCarry = 8;  // the unit starts from a published carry or the given start state
 
 struct ScanArgs {
     int Bt, L, d, N, K;
@@ -91,6 +91,8 @@ struct ScanArgs {
     unsigned int *counter;  // dynamic: next unit to hand out (zeroed before launch)
     unsigned int *flags;    // dynamic: [Bt*tiles][consumer warps] last published segment + 1
     float *carry;           // dynamic: [Bt*tiles][CPB][NS] published end states
+    const float *h_init;    // [Bt, d, N] start state, or null (zeros)
+    const void *conv_hist;  // [Bt, d, K-1] io conv history before token 0 (oldest first), or null (zeros)
 };
 
 template <int NS, int TPC, int T, bool CONV>
@@ -145,7 +147,9 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
 
 constexpr uint32_t kWaitPolls = 1u << 24;
 
-template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, bool ZOH>
+// INIT: the scan may start from a given state (h_init, conv_hist); a separate
+// instantiation, so that the plain scan's code is not touched by it.
+template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, bool ZOH, bool INIT>
 __global__ void __launch_bounds__(kScanBlock, 2)
     s6_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
@@ -207,6 +211,20 @@ __global__ void __launch_bounds__(kScanBlock, 2)
             }
             const int4 m = sm.meta[sp];
             const UnitPos up = unit_pos(m.x, a);
+            if (INIT && CONV && got && a.conv_hist && m.y == 0) {
+                // the sequence's first chunk: its halo rows before token 0 (zeros
+                // from the tensor copy) take the given conv history instead
+                const int K1 = a.K - 1;
+                const IO *hsrc = static_cast<const IO *>(a.conv_hist) + static_cast<size_t>(up.b) * a.d * K1;
+                const int c0 = up.tile * CPB;
+                for (int i = lane; i < CPB * K1; i += 32) {
+                    const int ch = i / K1;
+                    const int kk = i - ch * K1;
+                    if (c0 + ch < a.d)
+                        sm.x[sp].v[kHalo - K1 + kk][ch] = hsrc[static_cast<size_t>(c0 + ch) * K1 + kk];
+                }
+                fence_proxy_async_smem();  // before the stage is refilled by the tensor unit
+            }
             constexpr int kSlots = 2 * T * NS;
             if (got && a.bc_tma && a.N == NS) {
                 // whole rows: four values per lane step
@@ -305,7 +323,9 @@ __global__ void __launch_bounds__(kScanBlock, 2)
             const UnitPos up = unit_pos(unit, a);
             const int t0 = tlo + k * T;
             const bool carry_in = a.dynamic && k == 0 && up.seg > 0;
-            const int fl = (k == 0 ? kMetaFirst : 0) | (k == nk - 1 ? kMetaLast : 0) | (carry_in ? kMetaCarry : 0);
+            const bool given_in = INIT && a.h_init && k == 0 && up.seg == 0;  // a chain's start state is given
+            const int fl = (k == 0 ? kMetaFirst : 0) | (k == nk - 1 ? kMetaLast : 0) |
+                           (carry_in || given_in ? kMetaCarry : 0);
             if (lane == 0) {
                 sm.meta[s] = make_int4(unit, t0, min(T, thi - t0), fl);
                 const int c0 = up.tile * CPB;
@@ -320,6 +340,17 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                 if (a.bc_tma) {
                     tma_load_3d(&sm.braw[s].v[0][0], &tm_B, &sm.full[s], 0, t0, up.b);
                     tma_load_3d(&sm.craw[s].v[0][0], &tm_C, &sm.full[s], 0, t0, up.b);
+                }
+            }
+            if (given_in) {
+                // rows of h_init for this tile's channels, zero past d and N
+                const float *src = a.h_init + static_cast<size_t>(up.b) * a.d * a.N;
+                const int c0 = up.tile * CPB;
+                for (int i = lane; i < CPB * NS; i += 32) {
+                    const int ch = i / NS;
+                    const int n = i - ch * NS;
+                    const int cc = c0 + ch;
+                    sm.hinit[s][ch][n] = (cc < a.d && n < a.N) ? __ldg(src + static_cast<size_t>(cc) * a.N + n) : 0.0f;
                 }
             }
             if (carry_in) {
