@@ -174,6 +174,15 @@ __global__ void __launch_bounds__(kStepThreads) s6_step_bulk_kernel(const StepAr
     static_assert((CT * NS * 4) % 16 == 0 && (CT * sizeof(IO)) % 16 == 0, "runs start 16-byte aligned");
 
     const int tid = threadIdx.x;
+    // A thread's N states are NS/4 16-byte chunks of its channel's row in the
+    // stage; rows of neighbouring threads are NS*4 bytes apart, so walking the
+    // chunks in the same order on every thread would put several threads of a
+    // warp on the same banks.  Register chunk j of this thread holds row chunk
+    // j ^ rot, with rot chosen so that the 8 threads sharing a 128-byte span
+    // use 8 different 16-byte bank groups; the thread's A rates and its reads
+    // of B and C use the same order.
+    constexpr int kChunks = NS / 4;
+    const int rot = (tid / (8 / kChunks)) & (kChunks - 1);
     const long long ntiles = static_cast<long long>(ctiles) * a.Bt;
     const long long t_begin = static_cast<long long>(blockIdx.x) * per_cta;
     const long long t_end = t_begin + per_cta < ntiles ? t_begin + per_cta : ntiles;
@@ -283,7 +292,7 @@ __global__ void __launch_bounds__(kStepThreads) s6_step_bulk_kernel(const StepAr
                 const float4 *al4 = reinterpret_cast<const float4 *>(a.A_log + static_cast<size_t>(c) * NS);
 #pragma unroll
                 for (int v = 0; v < NS / 4; ++v) {
-                    const float4 al = __ldg(al4 + v);
+                    const float4 al = __ldg(al4 + (v ^ rot));
                     const float alv[4] = {al.x, al.y, al.z, al.w};
                     float A2v[4], nrv[4];
 #pragma unroll
@@ -357,7 +366,8 @@ __global__ void __launch_bounds__(kStepThreads) s6_step_bulk_kernel(const StepAr
             f2_t acc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
             for (int v = 0; v < NS / 4; ++v) {
-                const float4 h4 = hrow[v], B = B4[v], C = C4[v];
+                const int vr = v ^ rot;  // the row chunk in register chunk v
+                const float4 h4 = hrow[vr], B = B4[vr], C = C4[vr];
                 f2_t hp[2] = {f2_pack(h4.x, h4.y), f2_pack(h4.z, h4.w)};
                 const f2_t Bp[2] = {f2_pack(B.x, B.y), f2_pack(B.z, B.w)};
                 const f2_t Cp[2] = {f2_pack(C.x, C.y), f2_pack(C.z, C.w)};
@@ -378,7 +388,7 @@ __global__ void __launch_bounds__(kStepThreads) s6_step_bulk_kernel(const StepAr
                 float h0v, h1v, h2v, h3v;
                 f2_unpack(hp[0], h0v, h1v);
                 f2_unpack(hp[1], h2v, h3v);
-                hrow[v] = make_float4(h0v, h1v, h2v, h3v);
+                hrow[vr] = make_float4(h0v, h1v, h2v, h3v);
             }
             float a0, a1, a2, a3;
             f2_unpack(acc2[0], a0, a1);
