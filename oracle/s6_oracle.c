@@ -209,6 +209,139 @@ void s6o_conv_silu_channels(int64_t n_ch, int64_t L, int K, const double *x,
     }
 }
 
+/* ------------------------------------------------------------ gradients
+ * The backward pass of the scan (no conv: u given), for training through the
+ * block ("Carry context through a selective state": the recurrence is what
+ * makes training slow, since every timestep touches N states).  Reverse-mode
+ * differentiation of exactly the forward steps above, for the loss
+ * sum_t dy[t] * y[t]; no reading of the pages is needed beyond the forward.
+ */
+
+/* sigmoid(v) = 1 / (1 + e^-v), the derivative of softplus. */
+double s6o_sigmoid(double v)
+{
+    if (v >= 0.0)
+        return 1.0 / (1.0 + exp(-v));
+    double e = exp(v);
+    return e / (1.0 + e);
+}
+
+/* d SiLU(v) / dv = sigmoid(v) * (1 + v * (1 - sigmoid(v))). */
+double s6o_dsilu(double v)
+{
+    double s = s6o_sigmoid(v);
+    return s * (1.0 + v * (1.0 - s));
+}
+
+/*
+ * One channel's gradients.  Inputs as s6o_scan_channel with K = 0, plus
+ *   dy      [L]     gradient of the loss with respect to y
+ *   hs      [(L+1)*N]  work: the states h_{-1} .. h_{L-1}
+ * Outputs, written:     du[L], ddt[L] (with respect to dt_raw), dz[L] (if z)
+ * Outputs, accumulated: dB[L*N], dC[L*N] (this channel's share of the
+ *   sequence's rows), dA_log[N], dD[0], ddt_bias[0], dh_in[N] (if not NULL).
+ */
+void s6o_scan_bwd_channel(int64_t L, int N, int zoh,
+                          const double *u, const double *dt_raw, const double *z,
+                          const double *Bm, const double *Cm,
+                          const double *A_log, double D, double dt_bias,
+                          const double *h_in, const double *dy,
+                          double *du, double *ddt, double *dz,
+                          double *dB, double *dC, double *dA_log, double *dD, double *ddt_bias,
+                          double *dh_in, double *hs)
+{
+    /* forward, keeping every state: hs[(t+1)*N + n] = h_t[n] */
+    for (int n = 0; n < N; ++n)
+        hs[n] = h_in ? h_in[n] : 0.0;
+    for (int64_t t = 0; t < L; ++t) {
+        double delta = s6o_softplus(dt_raw[t] + dt_bias);
+        for (int n = 0; n < N; ++n) {
+            double a_bar = s6o_decay(delta, A_log[n]);
+            double write = s6o_write_gain(delta, A_log[n], zoh) * Bm[t * N + n] * u[t];
+            hs[(t + 1) * N + n] = s6o_update(hs[t * N + n], a_bar, write);
+        }
+    }
+
+    /* reverse: g[n] = dLoss/dh_t[n] arriving from tokens after t */
+    double g[64];
+    for (int n = 0; n < N; ++n)
+        g[n] = 0.0;
+    for (int64_t t = L - 1; t >= 0; --t) {
+        const double *h_t = hs + (t + 1) * N;
+        const double *h_prev = hs + t * N;
+        double v = dt_raw[t] + dt_bias;
+        double delta = s6o_softplus(v);
+        double s = D * u[t];
+        for (int n = 0; n < N; ++n)
+            s += h_t[n] * Cm[t * N + n];
+        double gate = z ? s6o_silu(z[t]) : 1.0;
+        double ds = dy[t] * gate;  /* d/ds of y = s * gate */
+        if (z)
+            dz[t] = dy[t] * s * s6o_dsilu(z[t]);
+        *dD += ds * u[t];
+        double dut = ds * D;
+        double ddelta = 0.0;
+        for (int n = 0; n < N; ++n) {
+            double A = s6o_A(A_log[n]);
+            double a_bar = s6o_decay(delta, A_log[n]);
+            double gain = s6o_write_gain(delta, A_log[n], zoh);
+            double b = Bm[t * N + n];
+            dC[t * N + n] += ds * h_t[n];
+            double dh = ds * Cm[t * N + n] + g[n];  /* total dLoss/dh_t[n] */
+            /* h_t = a_bar h_{t-1} + gain * b * u */
+            double da = dh * h_prev[n];
+            double dgain = dh * b * u[t];
+            dB[t * N + n] += dh * gain * u[t];
+            dut += dh * gain * b;
+            /* a_bar = exp(delta * A) */
+            ddelta += da * a_bar * A;
+            double dA = da * a_bar * delta;
+            if (zoh) {
+                /* gain = expm1(delta A) / A */
+                ddelta += dgain * a_bar;
+                dA += dgain * (delta * a_bar * A - expm1(delta * A)) / (A * A);
+            } else {
+                /* gain = delta */
+                ddelta += dgain;
+            }
+            dA_log[n] += dA * A; /* A = -exp(A_log): dA/dA_log = A */
+            g[n] = dh * a_bar;   /* to h_{t-1} */
+        }
+        du[t] = dut;
+        double dv = ddelta * s6o_sigmoid(v);  /* softplus'(v) = sigmoid(v) */
+        ddt[t] = dv;
+        *ddt_bias += dv;
+    }
+    if (dh_in)
+        for (int n = 0; n < N; ++n)
+            dh_in[n] += g[n];
+}
+
+/*
+ * Many channels: channel c reads u + c*L etc. and its B/C rows at
+ * Bm + bc_row[c]*L*N; it accumulates into dB/dC at dBm + c*L*N (one private
+ * block per channel; the caller sums the channels of a sequence), its
+ * parameter gradients at dA_log + c*N, dD[c], ddt_bias[c], dh_in + c*N.
+ */
+void s6o_scan_bwd_channels(int64_t n_ch, int64_t L, int N, int zoh,
+                           const double *u, const double *dt_raw, const double *z,
+                           const double *Bm, const double *Cm, const int64_t *bc_row,
+                           const double *A_log, const double *D, const double *dt_bias,
+                           const double *h_in, const double *dy,
+                           double *du, double *ddt, double *dz, double *dBm, double *dCm,
+                           double *dA_log, double *dD, double *ddt_bias, double *dh_in, double *work)
+{
+    for (int64_t c = 0; c < n_ch; ++c) {
+        s6o_scan_bwd_channel(L, N, zoh, u + c * L, dt_raw + c * L, z ? z + c * L : NULL,
+                             Bm + bc_row[c] * L * N, Cm + bc_row[c] * L * N,
+                             A_log + c * N, D[c], dt_bias ? dt_bias[c] : 0.0,
+                             h_in ? h_in + c * N : NULL, dy + c * L,
+                             du + c * L, ddt + c * L, z ? dz + c * L : NULL,
+                             dBm + c * L * N, dCm + c * L * N, dA_log + c * N, dD + c,
+                             ddt_bias + c, dh_in ? dh_in + c * N : NULL, work);
+    }
+}
+
 /* Streaming state size of a block stack: channels x states x blocks
  * ("mamba, live": 1,536 x 16 x 6 = 147,456; the TinyMamba example: 8 x 3 = 24). */
 int64_t s6o_ssm_state_values(int64_t d_inner, int64_t d_state, int64_t blocks)

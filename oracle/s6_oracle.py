@@ -18,6 +18,9 @@ What the oracle computes (page titles and sections):
   model manifest, ``steps`` *local/select/state/read*) -- exact diagonal
   zero-order hold ``B_bar = (exp(dt*A) - 1)/A * B``, a zero-left-padded causal
   conv, C reading the updated state, D multiplying the conv output.
+* ``scan_bwd`` -- the gradients of that scan (no conv), by reverse-mode
+  differentiation of the same steps; pinned by central differences of the
+  forward oracle.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` to values the
 pages print or to closed forms; none is "parity unpinned".
@@ -57,7 +60,7 @@ def bind(path: str):
     d, i, i64 = ctypes.c_double, ctypes.c_int, ctypes.c_int64
     for name, args in (("s6o_softplus", [d]), ("s6o_silu", [d]), ("s6o_A", [d]),
                        ("s6o_decay", [d, d]), ("s6o_write_gain", [d, d, i]),
-                       ("s6o_update", [d, d, d])):
+                       ("s6o_update", [d, d, d]), ("s6o_sigmoid", [d]), ("s6o_dsilu", [d])):
         f = getattr(lib, name)
         f.argtypes, f.restype = args, d
     lib.s6o_conv_pre.argtypes = [i, _c_double_p, d, _c_double_p, d]
@@ -68,6 +71,9 @@ def bind(path: str):
     lib.s6o_conv_silu_channels.argtypes = [i64, i64, i, _c_double_p, _c_double_p, _c_double_p,
                                            _c_double_p]
     lib.s6o_conv_silu_channels.restype = None
+    lib.s6o_scan_bwd_channels.argtypes = [i64, i64, i, i] + [_c_double_p] * 5 + [_c_i64_p] + \
+        [_c_double_p] * 15
+    lib.s6o_scan_bwd_channels.restype = None
     for name in ("s6o_ssm_state_values", "s6o_conv_history_values"):
         f = getattr(lib, name)
         f.argtypes, f.restype = [i64, i64, i64], i64
@@ -121,6 +127,14 @@ def write_gain(delta: float, A_log: float, zoh: bool) -> float:
 
 def update(h: float, a_bar: float, write: float) -> float:
     return _load().s6o_update(float(h), float(a_bar), float(write))
+
+
+def sigmoid(v: float) -> float:
+    return _load().s6o_sigmoid(float(v))
+
+
+def dsilu(v: float) -> float:
+    return _load().s6o_dsilu(float(v))
 
 
 def conv_pre(w, bias: float, hist, x_t: float) -> float:
@@ -240,6 +254,66 @@ def scan(x, dt_raw, A_log, B, C, D, z=None, dt_bias=None, zoh=False, conv_w=None
         hs = histout[:, :km1].reshape(Bt, d, km1)
         return (y_full, h_full, hs) if return_state else (y_full, h_full)
     return (y, hout, histout[:, :km1]) if return_state else (y, hout)
+
+
+def scan_bwd(u, dt_raw, A_log, B, C, D, dy, z=None, dt_bias=None, zoh=False, h_init=None, threads=None):
+    """Gradients of the scan without conv (u given) for the loss sum(dy * y).
+
+    u, dt_raw, z, dy: [Bt, L, d]; B, C: [Bt, L, N]; A_log: [d, N]; D, dt_bias:
+    [d]; h_init: [Bt, d, N] or None (zeros).  Returns a dict of float64 arrays:
+    du, ddt, dz (None without z) [Bt, L, d]; dB, dC [Bt, L, N]; dA_log [d, N];
+    dD, ddt_bias [d]; dh_init [Bt, d, N].
+    """
+    u = np.asarray(u)
+    Bt, L, d = u.shape
+    N = np.asarray(A_log).shape[1]
+    bb, dd = np.meshgrid(np.arange(Bt), np.arange(d), indexing="ij")
+    cb, cd = bb.ravel(), dd.ravel()
+    n = Bt * d
+
+    def seq(a):
+        return np.ascontiguousarray(np.transpose(_f64(a), (0, 2, 1))).reshape(n, L)
+
+    us, dts, dys = seq(u), seq(dt_raw), seq(dy)
+    zs = seq(z) if z is not None else None
+    Bm = np.ascontiguousarray(_f64(B)).reshape(-1)
+    Cm = np.ascontiguousarray(_f64(C)).reshape(-1)
+    bc_row = np.ascontiguousarray(cb.astype(np.int64))
+    Al = np.ascontiguousarray(_f64(A_log)[cd])
+    Dv = np.ascontiguousarray(_f64(D)[cd])
+    bias = np.ascontiguousarray(_f64(dt_bias)[cd]) if dt_bias is not None else None
+    hin = np.ascontiguousarray(_f64(h_init).reshape(n, N)) if h_init is not None else None
+    du, ddt = np.zeros((n, L)), np.zeros((n, L))
+    dz = np.zeros((n, L)) if z is not None else None
+    dBc, dCc = np.zeros((n, L, N)), np.zeros((n, L, N))
+    dAl, dDc, dbc, dh = np.zeros((n, N)), np.zeros(n), np.zeros(n), np.zeros((n, N))
+    lib = _load()
+    nt = _threads(n, threads)
+    bounds = np.linspace(0, n, nt + 1).astype(np.int64)
+
+    def run(i):
+        lo, hi = int(bounds[i]), int(bounds[i + 1])
+        sl = slice(lo, hi)
+
+        def p(a):
+            return None if a is None else _ptr(a[sl])
+
+        work = np.zeros((L + 1) * N)
+        lib.s6o_scan_bwd_channels(hi - lo, L, N, int(bool(zoh)), p(us), p(dts), p(zs), _ptr(Bm), _ptr(Cm),
+                                  bc_row[sl].ctypes.data_as(_c_i64_p), p(Al), p(Dv), p(bias), p(hin), p(dys),
+                                  p(du), p(ddt), p(dz), p(dBc), p(dCc), p(dAl), p(dDc), p(dbc), p(dh), _ptr(work))
+
+    with ThreadPoolExecutor(nt) as ex:
+        list(ex.map(run, range(nt)))
+
+    def back(a):
+        return np.transpose(a.reshape(Bt, d, L), (0, 2, 1))
+
+    return {"du": back(du), "ddt": back(ddt), "dz": back(dz) if dz is not None else None,
+            # B and C rows are shared by the d channels of a sequence: sum their shares
+            "dB": dBc.reshape(Bt, d, L, N).sum(axis=1), "dC": dCc.reshape(Bt, d, L, N).sum(axis=1),
+            "dA_log": dAl.reshape(Bt, d, N).sum(axis=0), "dD": dDc.reshape(Bt, d).sum(axis=0),
+            "ddt_bias": dbc.reshape(Bt, d).sum(axis=0), "dh_init": dh.reshape(Bt, d, N)}
 
 
 def conv_silu(x, conv_w, conv_b=None, threads=None):

@@ -10,6 +10,7 @@ import subprocess
 import pytest
 
 from oracle import s6_oracle as O
+import test_oracle_bwd as TB
 import test_oracle_pins as P
 
 SRC = os.path.join(os.path.dirname(O.__file__), "s6_oracle.c")
@@ -37,6 +38,9 @@ ALL_PINS = [
     P.test_future_changes_leave_past_unchanged,
     P.test_conv_window_width3,
     lambda: P.test_streaming_equals_full_forward(True),
+    TB.test_sigmoid_and_dsilu_closed_forms,
+    lambda: TB.check_gradients_by_central_differences(False, True),
+    lambda: TB.check_gradients_by_central_differences(True, True),
 ]
 
 MUTATIONS = {
@@ -61,6 +65,17 @@ MUTATIONS = {
     "conv_no_bias": ("double acc = bias;", "double acc = 0.0 * bias;"),
     "conv_history_not_shifted": ("hist[k] = hist[k + 1];", "hist[k] = hist[k];"),
     "state_count_wrong": ("return d_inner * d_state * blocks;", "return d_inner * d_state;"),
+    # the backward pass
+    "bwd_carry_no_decay": ("g[n] = dh * a_bar;   /* to h_{t-1} */", "g[n] = dh;   /* to h_{t-1} */"),
+    "bwd_zoh_explicit_dA_missing": ("dA += dgain * (delta * a_bar * A - expm1(delta * A)) / (A * A);",
+                                    "dA += 0.0 * dgain;"),
+    "bwd_no_softplus_derivative": ("double dv = ddelta * s6o_sigmoid(v);", "double dv = ddelta;"),
+    "bwd_dA_log_chain_missing": ("dA_log[n] += dA * A;", "dA_log[n] += dA;"),
+    "bwd_dsilu_as_sigmoid": ("return s * (1.0 + v * (1.0 - s));", "return s;"),
+    "bwd_dC_old_state": ("dC[t * N + n] += ds * h_t[n];", "dC[t * N + n] += ds * h_prev[n];"),
+    "bwd_du_misses_D": ("double dut = ds * D;", "double dut = 0.0 * ds;"),
+    "bwd_gate_not_applied": ("double ds = dy[t] * gate;", "double ds = dy[t];"),
+    "bwd_write_gain_missing_in_dB": ("dB[t * N + n] += dh * gain * u[t];", "dB[t * N + n] += dh * u[t];"),
 }
 
 
