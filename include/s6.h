@@ -200,6 +200,34 @@ S6_API int s6_conv_scan_fwd_from_state(const s6_dims *dims, const void *x, const
                                        s6_stream_t stream);
 
 /*
+ * s6_scan_bwd -- gradients of s6_scan_fwd (no conv: u given) for the loss
+ * sum(dy * y): reverse-mode differentiation of the same steps (the recurrence
+ * the pages single out as what makes training slow, "Carry context through a
+ * selective state"; "mamba, live" for the forward).  Inputs as
+ * s6_scan_fwd_from_state, plus
+ *
+ *  dy        [Bt,L,d] io   gradient with respect to y
+ *  h_init    [Bt,d,N] f32  start state of the forward, NULL = zeros
+ * Written (float32):
+ *  du, ddt   [Bt,L,d]      with respect to u and the raw dt
+ *  dz        [Bt,L,d]      with respect to z (required when z is given)
+ *  dB, dC    [Bt,L,N]      summed over the d channels of each sequence
+ *  dA_log    [d,N], dD [d], ddt_bias [d] (NULL = not wanted)
+ *                          summed over the sequences and tokens
+ *  dh_init   [Bt,d,N]      with respect to h_init (NULL = not wanted)
+ * dB, dC, dA_log, dD and ddt_bias are zeroed by the call, then accumulated
+ * with atomics, so their last bits depend on the order of the additions.  The
+ * call uses the library-owned scratch buffer (state checkpoints every 64
+ * tokens plus one chunk of states: (ceil(L/64) + 64) * Bt * d * 16 floats at
+ * N = 16).  Pointers need only element alignment.
+ */
+S6_API int s6_scan_bwd(const s6_dims *dims, const void *u, const void *dt, const float *A_log,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *dt_bias, int zoh_mode, const float *h_init, const void *dy,
+                       float *du, float *ddt, float *dz, float *dB, float *dC, float *dA_log,
+                       float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream);
+
+/*
  * causal_conv1d_silu_fwd -- the conv + SiLU alone ("mamba, live":
  * depthwise_conv4 then SiLU; "Carry context ...", step "local").
  *
