@@ -541,7 +541,7 @@ int launch_bwd_t(s6::BwdArgs a, cudaStream_t st) {
         return rc;
     a.ck = static_cast<float *>(scr);
     a.hb = a.ck + ckf;
-    const long long grid = (G + s6::kBwdThreads - 1) / s6::kBwdThreads;
+    const long long grid = (G * s6::kBwdTPC + s6::kBwdThreads - 1) / s6::kBwdThreads;
     if (grid > 0x7fffffffLL)
         return S6_ERR_UNSUPPORTED;
     s6::s6_scan_bwd_kernel<IO, NS, ZOH><<<static_cast<unsigned>(grid), s6::kBwdThreads, 0, st>>>(a);

@@ -14,14 +14,15 @@
 //     dA      += dh_t h_{t-1} a_t Delta_t (+ ZOH: dh_t B_t u_t dgain/dA)
 //     ddt_t = dDelta_t sigmoid(v_t);  dA_log = dA * A;  dD += ds_t u_t
 //
-// One thread owns one (sequence, channel) and all of its N states.  The
-// reverse pass needs h_{t-1} at every t: a first forward pass saves the state
+// Four threads share a (sequence, channel), each owning N/4 of its states;
+// the sums over the states (readout, du, dDelta) go through two shuffles.
+// The reverse pass needs h_{t-1} at every t: a first forward pass saves the state
 // at the start of every chunk of kBwdChunk tokens (checkpoints), then the
 // chunks are walked last to first, each recomputed forward from its
 // checkpoint into a scratch buffer and then walked backwards.  Scratch layouts
 // put consecutive threads at consecutive addresses.  dB and dC are shared by
 // all channels of a sequence: a warp whose lanes all belong to one sequence
-// sums its 32 channels' shares with shuffles and adds them with one atomic
+// sums its 8 channels' shares with shuffles and adds them with one atomic
 // per value, otherwise every lane adds its own.  The parameter gradients
 // (dA_log, dD, ddt_bias) are summed over the sequences with atomics.
 #pragma once
@@ -32,14 +33,15 @@ namespace s6 {
 
 constexpr int kBwdThreads = 128;
 constexpr int kBwdChunk = 64;  // tokens between checkpoints
+constexpr int kBwdTPC = 4;     // threads per channel (N/4 states each)
 
 struct BwdArgs {
     int Bt, L, d, N, has_z, nck;
     const void *u, *dt, *B, *C, *z, *dy;
     const float *A_log, *D, *dt_bias, *h_init;
     float *du, *ddt, *dz, *dB, *dC, *dA_log, *dD, *ddt_bias, *dh_init;
-    float *ck;  // [nck][NS][Bt*d] state at the start of each chunk
-    float *hb;  // [kBwdChunk][NS][Bt*d] the states of the chunk being reversed
+    float *ck;  // [nck][NS/4][Bt*d*4] state at the start of each chunk
+    float *hb;  // [kBwdChunk][NS/4][Bt*d*4] the states of the chunk being reversed
 };
 
 // ZOH write gain (e^x - 1)/A with x = Delta*A, and its derivative in A at
@@ -60,22 +62,36 @@ template <typename IO, int NS, bool ZOH>
 __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs a) {
     using tr = io_traits<IO>;
     constexpr int T = kBwdChunk;
-    const long long G = static_cast<long long>(a.Bt) * a.d;
-    const long long g = static_cast<long long>(blockIdx.x) * kBwdThreads + threadIdx.x;
-    const bool live = g < G;
-    const long long gc = live ? g : 0;
+    constexpr int TPC = kBwdTPC;      // threads per channel
+    constexpr int NH = NS / TPC;      // states per thread
+    const long long G = static_cast<long long>(a.Bt) * a.d;  // channels
+    const long long GT = G * TPC;                            // threads with work
+    const long long gt = static_cast<long long>(blockIdx.x) * kBwdThreads + threadIdx.x;
+    const bool live = gt < GT;
+    const long long gtc = live ? gt : 0;
+    const long long gc = gtc / TPC;  // channel
+    const int q = static_cast<int>(gtc - gc * TPC);
+    const int n0 = q * NH;           // this thread's first state
     const int b = static_cast<int>(gc / a.d);
     const int c = static_cast<int>(gc - static_cast<long long>(b) * a.d);
     const unsigned full = 0xffffffffu;
     // every lane of the warp in the same sequence: dB/dC can be summed in the warp
     const bool one_seq = __all_sync(full, b == __shfl_sync(full, b, 0));
-
-    float A[NS], A2[NS];
+    // sum over the TPC threads of a channel
+    auto chan_sum = [&](float v) {
 #pragma unroll
-    for (int n = 0; n < NS; ++n) {
+        for (int off = 1; off < TPC; off <<= 1)
+            v += __shfl_xor_sync(full, v, off);
+        return v;
+    };
+
+    float A[NH], A2[NH];
+#pragma unroll
+    for (int j = 0; j < NH; ++j) {
+        const int n = n0 + j;
         const float Av = (n < a.N) ? -expf(a.A_log[static_cast<size_t>(c) * a.N + n]) : 0.0f;  // A = -exp(A_log)
-        A[n] = Av;
-        A2[n] = Av * kLog2e;
+        A[j] = Av;
+        A2[j] = Av * kLog2e;
     }
     const float Dd = a.D[c];
     const float bias = a.dt_bias ? a.dt_bias[c] : 0.0f;
@@ -83,34 +99,36 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
     auto seq = [&](const void *p, int t) -> float {
         return tr::to_f(static_cast<const IO *>(p)[(static_cast<size_t>(b) * a.L + t) * a.d + c]);
     };
-    auto row = [&](const void *p, int t, int n) -> float {
+    auto row = [&](const void *p, int t, int j) -> float {
+        const int n = n0 + j;
         return (n < a.N) ? tr::to_f(static_cast<const IO *>(p)[(static_cast<size_t>(b) * a.L + t) * a.N + n]) : 0.0f;
     };
-    auto slot = [&](float *base, int i, int n) -> float * {
-        return base + (static_cast<size_t>(i) * NS + n) * G + gc;
+    // scratch slot of this thread's state j at checkpoint / chunk row i
+    auto slot = [&](float *base, int i, int j) -> float * {
+        return base + (static_cast<size_t>(i) * NH + j) * GT + gtc;
     };
     // one forward token: h <- a h + gain B u
-    auto step = [&](int t, float (&h)[NS]) {
+    auto step = [&](int t, float (&h)[NH]) {
         const float delta = softplus_f(seq(a.dt, t) + bias);
         const float uu = seq(a.u, t);
 #pragma unroll
-        for (int n = 0; n < NS; ++n) {
-            const float ab = ex2_approx(delta * A2[n]);
-            const float gain = ZOH ? ((n < a.N) ? zoh_gain(delta * A[n], A[n]) : 0.0f) : delta;
-            h[n] = fmaf(ab, h[n], gain * row(a.B, t, n) * uu);
+        for (int j = 0; j < NH; ++j) {
+            const float ab = ex2_approx(delta * A2[j]);
+            const float gain = ZOH ? ((n0 + j < a.N) ? zoh_gain(delta * A[j], A[j]) : 0.0f) : delta;
+            h[j] = fmaf(ab, h[j], gain * row(a.B, t, j) * uu);
         }
     };
 
     // ---- pass 1: forward, checkpoint at every chunk start
-    float h[NS];
+    float h[NH];
 #pragma unroll
-    for (int n = 0; n < NS; ++n)
-        h[n] = (live && a.h_init && n < a.N) ? a.h_init[gc * a.N + n] : 0.0f;
+    for (int j = 0; j < NH; ++j)
+        h[j] = (live && a.h_init && n0 + j < a.N) ? a.h_init[gc * a.N + n0 + j] : 0.0f;
     for (int k = 0; k < a.nck; ++k) {
         if (live) {
 #pragma unroll
-            for (int n = 0; n < NS; ++n)
-                *slot(a.ck, k, n) = h[n];
+            for (int j = 0; j < NH; ++j)
+                *slot(a.ck, k, j) = h[j];
         }
         const int t1 = min(a.L, (k + 1) * T);
         for (int t = k * T; t < t1; ++t)
@@ -118,124 +136,133 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
     }
 
     // ---- pass 2: chunks last to first
-    float gcar[NS], dA[NS];  // dLoss/dh from later tokens (times their decay); dLoss/dA
+    float gcar[NH], dA[NH];  // dLoss/dh from later tokens (times their decay); dLoss/dA
 #pragma unroll
-    for (int n = 0; n < NS; ++n)
-        gcar[n] = dA[n] = 0.0f;
-    float dDa = 0.0f, dba = 0.0f;
+    for (int j = 0; j < NH; ++j)
+        gcar[j] = dA[j] = 0.0f;
+    float dDa = 0.0f, dba = 0.0f;  // kept by the channel's first thread
     for (int k = a.nck - 1; k >= 0; --k) {
         const int t0 = k * T, t1 = min(a.L, t0 + T);
-        float hc[NS];
+        float hc[NH];
 #pragma unroll
-        for (int n = 0; n < NS; ++n)
-            hc[n] = live ? *slot(a.ck, k, n) : 0.0f;
+        for (int j = 0; j < NH; ++j)
+            hc[j] = live ? *slot(a.ck, k, j) : 0.0f;
         for (int t = t0; t < t1; ++t) {
             step(t, hc);
             if (live) {
 #pragma unroll
-                for (int n = 0; n < NS; ++n)
-                    *slot(a.hb, t - t0, n) = hc[n];
+                for (int j = 0; j < NH; ++j)
+                    *slot(a.hb, t - t0, j) = hc[j];
             }
         }
-        for (int t = t1 - 1; t >= t0; --t) {
-            float ht[NS], hp[NS];
+        float ht[NH];  // h_t; the state after the chunk's last token is still in hc
 #pragma unroll
-            for (int n = 0; n < NS; ++n) {
-                ht[n] = live ? *slot(a.hb, t - t0, n) : 0.0f;
-                hp[n] = live ? (t > t0 ? *slot(a.hb, t - t0 - 1, n) : *slot(a.ck, k, n)) : 0.0f;
-            }
+        for (int j = 0; j < NH; ++j)
+            ht[j] = live ? hc[j] : 0.0f;
+        for (int t = t1 - 1; t >= t0; --t) {
+            float hp[NH];  // h_{t-1}
+#pragma unroll
+            for (int j = 0; j < NH; ++j)
+                hp[j] = live ? (t > t0 ? *slot(a.hb, t - t0 - 1, j) : *slot(a.ck, k, j)) : 0.0f;
             const float v = seq(a.dt, t) + bias;
             const float delta = softplus_f(v);
             const float uu = seq(a.u, t);
             const float dyv = live ? seq(a.dy, t) : 0.0f;
-            float s = Dd * uu;
+            float sp = 0.0f;
 #pragma unroll
-            for (int n = 0; n < NS; ++n)
-                s = fmaf(ht[n], row(a.C, t, n), s);
+            for (int j = 0; j < NH; ++j)
+                sp = fmaf(ht[j], row(a.C, t, j), sp);
+            const float s = fmaf(Dd, uu, chan_sum(sp));
             float gate = 1.0f;
+            const size_t o = (static_cast<size_t>(b) * a.L + t) * a.d + c;
             if (a.has_z) {
                 const float zv = seq(a.z, t);
                 const float sg = 1.0f / (1.0f + expf(-zv));
                 gate = zv * sg;
-                if (live)
-                    a.dz[(static_cast<size_t>(b) * a.L + t) * a.d + c] = dyv * s * sg * (1.0f + zv * (1.0f - sg));
+                if (live && q == 0)
+                    a.dz[o] = dyv * s * sg * (1.0f + zv * (1.0f - sg));
             }
             const float ds = dyv * gate;
-            dDa = fmaf(ds, uu, dDa);
-            float dut = ds * Dd, ddelta = 0.0f;
-            float dBn[NS], dCn[NS];
+            float dup = 0.0f, ddp = 0.0f;  // this thread's shares of du and dDelta
+            float dBn[NH], dCn[NH];
 #pragma unroll
-            for (int n = 0; n < NS; ++n) {
-                const float ab = ex2_approx(delta * A2[n]);
-                const float Bn = row(a.B, t, n), Cn = row(a.C, t, n);
-                const float gain = ZOH ? ((n < a.N) ? zoh_gain(delta * A[n], A[n]) : 0.0f) : delta;
-                dCn[n] = ds * ht[n];
-                const float dh = fmaf(ds, Cn, gcar[n]);
-                const float da = dh * hp[n];
+            for (int j = 0; j < NH; ++j) {
+                const float ab = ex2_approx(delta * A2[j]);
+                const float Bn = row(a.B, t, j), Cn = row(a.C, t, j);
+                const bool inN = n0 + j < a.N;
+                const float gain = ZOH ? (inN ? zoh_gain(delta * A[j], A[j]) : 0.0f) : delta;
+                dCn[j] = ds * ht[j];
+                const float dh = fmaf(ds, Cn, gcar[j]);
+                const float da = dh * hp[j];
                 const float dgain = dh * Bn * uu;
-                dBn[n] = dh * gain * uu;
-                dut = fmaf(dh * gain, Bn, dut);
-                ddelta = fmaf(da * ab, A[n], ddelta);
+                dBn[j] = dh * gain * uu;
+                dup = fmaf(dh * gain, Bn, dup);
+                ddp = fmaf(da * ab, A[j], ddp);
                 float dAn = da * ab * delta;
                 if (ZOH) {
-                    ddelta = fmaf(dgain, ab, ddelta);
-                    if (n < a.N)
-                        dAn += dgain * zoh_dgain_dA(delta * A[n], delta, A[n]);
-                } else {
-                    ddelta += dgain;
+                    ddp = fmaf(dgain, ab, ddp);
+                    if (inN)
+                        dAn += dgain * zoh_dgain_dA(delta * A[j], delta, A[j]);
+                } else if (inN) {
+                    ddp += dgain;
                 }
-                dA[n] += dAn;
-                gcar[n] = dh * ab;
+                dA[j] += dAn;
+                gcar[j] = dh * ab;
             }
-            const float dv = ddelta / (1.0f + expf(-v));  // softplus'(v) = sigmoid(v)
-            dba += dv;
-            if (live) {
-                const size_t o = (static_cast<size_t>(b) * a.L + t) * a.d + c;
-                a.du[o] = dut;
-                a.ddt[o] = dv;
+            const float dut = fmaf(ds, Dd, chan_sum(dup));
+            const float dv = chan_sum(ddp) / (1.0f + expf(-v));  // softplus'(v) = sigmoid(v)
+            if (q == 0) {
+                dDa = fmaf(ds, uu, dDa);
+                dba += dv;
+                if (live) {
+                    a.du[o] = dut;
+                    a.ddt[o] = dv;
+                }
             }
-            // dB, dC rows of (b, t): sum over the channels
-            float *dBr = a.dB + (static_cast<size_t>(b) * a.L + t) * a.N;
-            float *dCr = a.dC + (static_cast<size_t>(b) * a.L + t) * a.N;
+            // dB, dC rows of (b, t): sum over the warp's 8 channels
+            float *dBr = a.dB + (static_cast<size_t>(b) * a.L + t) * a.N + n0;
+            float *dCr = a.dC + (static_cast<size_t>(b) * a.L + t) * a.N + n0;
             if (one_seq) {
 #pragma unroll
-                for (int n = 0; n < NS; ++n) {
-                    float vb = dBn[n], vc = dCn[n];
+                for (int j = 0; j < NH; ++j) {
+                    float vb = dBn[j], vc = dCn[j];
 #pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) {
+                    for (int off = TPC; off < 32; off <<= 1) {
                         vb += __shfl_xor_sync(full, vb, off);
                         vc += __shfl_xor_sync(full, vc, off);
                     }
-                    if ((threadIdx.x & 31) == 0 && n < a.N) {
-                        atomicAdd(dBr + n, vb);
-                        atomicAdd(dCr + n, vc);
+                    if ((threadIdx.x & 31) < TPC && n0 + j < a.N) {
+                        atomicAdd(dBr + j, vb);
+                        atomicAdd(dCr + j, vc);
                     }
                 }
             } else if (live) {
 #pragma unroll
-                for (int n = 0; n < NS; ++n)
-                    if (n < a.N) {
-                        atomicAdd(dBr + n, dBn[n]);
-                        atomicAdd(dCr + n, dCn[n]);
+                for (int j = 0; j < NH; ++j)
+                    if (n0 + j < a.N) {
+                        atomicAdd(dBr + j, dBn[j]);
+                        atomicAdd(dCr + j, dCn[j]);
                     }
             }
+#pragma unroll
+            for (int j = 0; j < NH; ++j)
+                ht[j] = hp[j];
         }
     }
     if (!live)
         return;
-    if (a.dh_init) {
 #pragma unroll
-        for (int n = 0; n < NS; ++n)
-            if (n < a.N)
-                a.dh_init[gc * a.N + n] = gcar[n];
+    for (int j = 0; j < NH; ++j)
+        if (n0 + j < a.N) {
+            if (a.dh_init)
+                a.dh_init[gc * a.N + n0 + j] = gcar[j];
+            atomicAdd(a.dA_log + static_cast<size_t>(c) * a.N + n0 + j, dA[j] * A[j]);  // dA/dA_log = A
+        }
+    if (q == 0) {
+        atomicAdd(a.dD + c, dDa);
+        if (a.ddt_bias)
+            atomicAdd(a.ddt_bias + c, dba);
     }
-#pragma unroll
-    for (int n = 0; n < NS; ++n)
-        if (n < a.N)
-            atomicAdd(a.dA_log + static_cast<size_t>(c) * a.N + n, dA[n] * A[n]);  // dA/dA_log = A
-    atomicAdd(a.dD + c, dDa);
-    if (a.ddt_bias)
-        atomicAdd(a.ddt_bias + c, dba);
 }
 
 }  // namespace s6
