@@ -106,6 +106,38 @@ def test_conv_and_step_host_checks(lib):
                        None) == S.S6_ERR_ALIGNMENT
 
 
+def test_from_state_and_backward_host_checks(lib):
+    import selective_state_space_19_b200 as S
+    P = ctypes.c_void_p
+    d = ctypes.byref(_dims())
+    ok = P(16)
+
+    def fs(zoh=0, h_init=ok, hist=ok):  # s6_conv_scan_fwd_from_state
+        return lib.s6_conv_scan_fwd_from_state(d, ok, ok, None, ok, ok, ok, ok, ok, None, None, zoh, h_init, hist,
+                                               ok, None, None)
+    assert fs(zoh=2) == S.S6_ERR_INVALID_ARG
+    assert fs(h_init=P(18)) == S.S6_ERR_ALIGNMENT   # float32 start state
+    assert fs(hist=P(18)) == S.S6_ERR_ALIGNMENT     # float32 I/O conv history
+    assert lib.s6_scan_fwd_from_state(d, ok, ok, ok, ok, ok, ok, None, None, 0, P(2), ok, None,
+                                      None) == S.S6_ERR_ALIGNMENT
+
+    def bwd(zoh=0, **kw):  # s6_scan_bwd
+        a = dict(u=ok, dt=ok, A_log=ok, B=ok, C=ok, D=ok, z=None, dt_bias=None, h_init=None, dy=ok, du=ok,
+                 ddt=ok, dz=None, dB=ok, dC=ok, dA_log=ok, dD=ok, ddt_bias=None, dh_init=None)
+        a.update(kw)
+        return lib.s6_scan_bwd(kw.pop("dims", d), a["u"], a["dt"], a["A_log"], a["B"], a["C"], a["D"], a["z"],
+                               a["dt_bias"], zoh, a["h_init"], a["dy"], a["du"], a["ddt"], a["dz"], a["dB"],
+                               a["dC"], a["dA_log"], a["dD"], a["ddt_bias"], a["dh_init"], None)
+    assert bwd(zoh=5) == S.S6_ERR_INVALID_ARG
+    assert bwd(dy=None) == S.S6_ERR_INVALID_ARG
+    assert bwd(dB=None) == S.S6_ERR_INVALID_ARG
+    assert bwd(z=ok) == S.S6_ERR_INVALID_ARG        # a gate needs dz
+    assert bwd(u=P(18)) == S.S6_ERR_ALIGNMENT
+    assert bwd(dA_log=P(2)) == S.S6_ERR_ALIGNMENT
+    assert bwd(dims=ctypes.byref(_dims(d_state=17))) == S.S6_ERR_UNSUPPORTED
+    assert bwd(dims=ctypes.byref(_dims(batch=0))) == S.S6_OK  # nothing to do, nothing touched
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     import selective_state_space_19_b200 as S
