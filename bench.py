@@ -132,10 +132,16 @@ def to_pinned(a):
 
 
 def kernel_source_sha():
+    """Hash of the scan kernel's sources with comments and blank lines removed, so
+    that an edit of a comment does not orphan the recorded capture."""
     h = hashlib.sha256()
     for f in ("s6_common.cuh", "s6_scan.cuh"):
-        with open(os.path.join(ROOT, "selective_state_space_19_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "selective_state_space_19_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+        h.update(code.encode())
     return h.hexdigest()[:16]
 
 

@@ -37,15 +37,22 @@
 //
 // Arithmetic.  The 16 decays per element are the binding work (one live
 // exponential per state per token, "the s6 cell") and go to the MUFU ex2
-// pipe.  SiLU and softplus take one MUFU op each, their reciprocal and log1p
-// run on the FMA pipe.  With TPC = 2 the two threads of a channel walk the
-// tokens in pairs: each computes every per-token scalar (conv, both SiLUs,
-// softplus) of one token of the pair and the two swap u and Delta with
-// shuffles, so no scalar is computed twice; each then updates its NH states
-// for both tokens, and the partial readouts are swapped so that each thread
-// finishes and writes the output of its own token.  State arithmetic runs on
-// packed float32 pairs (f32x2); the scalars of the next pair are computed
-// before the state update of the current one.
+// pipe.  SiLU and softplus take one MUFU op each (SiLU by tanh for bfloat16
+// I/O); the reciprocal and log1p run on the FMA pipe.  With TPC = 2 the two
+// threads of a channel walk the tokens in quads: each computes the per-token
+// scalars (conv, both SiLUs, softplus) of two of the four tokens in packed
+// form, and the pair swaps (u, Delta) through per-lane shared-memory slots, so
+// no scalar is computed twice; each thread then updates its NH states token
+// by token, issuing the next token's decays among the current token's FMAs,
+// and the partial readouts are swapped with one shuffle so that each thread
+// finishes and writes its own tokens.  The next quad's scalars are computed
+// at the start of a quad, its (u, Delta) exchanged after the updates, and the
+// rows they read (conv window, z, dt) fetched one quad ahead.  State
+// arithmetic runs on packed float32 pairs (f32x2).
+//
+// The INIT instantiations also start a chain from a given state (h_init, and
+// for the fused form the conv history before token 0); they are separate so
+// that the plain scan's code is untouched by that support.
 //
 // No tensor cores: the recurrence is diagonal (an elementwise product with a
 // data-dependent decay), not a contraction.
