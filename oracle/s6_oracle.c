@@ -342,6 +342,45 @@ void s6o_scan_bwd_channels(int64_t n_ch, int64_t L, int N, int zoh,
     }
 }
 
+/*
+ * Backward of the causal conv + SiLU in front of the scan, one channel at a
+ * time: given dxc[t] (the gradient with respect to the conv output u_t, e.g.
+ * du of s6o_scan_bwd_channels), pre_t = bias + sum_k w[k] x[t-K+1+k] with
+ * zero left padding, u_t = SiLU(pre_t):
+ *   dpre_t = dxc[t] * SiLU'(pre_t);  dx[t-K+1+k] += w[k] dpre_t (in range);
+ *   dw[k] += dpre_t x[t-K+1+k];  db += dpre_t.
+ * dx is written; dw (K values per channel) and db are accumulated.
+ */
+void s6o_conv_silu_bwd_channels(int64_t n_ch, int64_t L, int K, const double *x,
+                                const double *conv_w, const double *conv_b, const double *dxc,
+                                double *dx, double *dw, double *db)
+{
+    for (int64_t c = 0; c < n_ch; ++c) {
+        const double *xc = x + c * L;
+        const double *w = conv_w + c * K;
+        double *dxo = dx + c * L;
+        for (int64_t t = 0; t < L; ++t)
+            dxo[t] = 0.0;
+        double hist[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int64_t t = 0; t < L; ++t) {
+            double pre = s6o_conv_pre(K, w, conv_b ? conv_b[c] : 0.0, hist, xc[t]);
+            double dpre = dxc[c * L + t] * s6o_dsilu(pre);
+            for (int k = 0; k < K; ++k) {
+                int64_t src = t - (K - 1) + k;
+                if (src >= 0) {
+                    dxo[src] += w[k] * dpre;
+                    dw[c * K + k] += dpre * xc[src];
+                }
+            }
+            db[c] += dpre;
+            for (int k = 0; k + 1 < K - 1; ++k)
+                hist[k] = hist[k + 1];
+            if (K > 1)
+                hist[K - 2] = xc[t];
+        }
+    }
+}
+
 /* Streaming state size of a block stack: channels x states x blocks
  * ("mamba, live": 1,536 x 16 x 6 = 147,456; the TinyMamba example: 8 x 3 = 24). */
 int64_t s6o_ssm_state_values(int64_t d_inner, int64_t d_state, int64_t blocks)

@@ -74,6 +74,8 @@ def bind(path: str):
     lib.s6o_scan_bwd_channels.argtypes = [i64, i64, i, i] + [_c_double_p] * 5 + [_c_i64_p] + \
         [_c_double_p] * 15
     lib.s6o_scan_bwd_channels.restype = None
+    lib.s6o_conv_silu_bwd_channels.argtypes = [i64, i64, i] + [_c_double_p] * 7
+    lib.s6o_conv_silu_bwd_channels.restype = None
     for name in ("s6o_ssm_state_values", "s6o_conv_history_values"):
         f = getattr(lib, name)
         f.argtypes, f.restype = [i64, i64, i64], i64
@@ -314,6 +316,31 @@ def scan_bwd(u, dt_raw, A_log, B, C, D, dy, z=None, dt_bias=None, zoh=False, h_i
             "dB": dBc.reshape(Bt, d, L, N).sum(axis=1), "dC": dCc.reshape(Bt, d, L, N).sum(axis=1),
             "dA_log": dAl.reshape(Bt, d, N).sum(axis=0), "dD": dDc.reshape(Bt, d).sum(axis=0),
             "ddt_bias": dbc.reshape(Bt, d).sum(axis=0), "dh_init": dh.reshape(Bt, d, N)}
+
+
+def conv_scan_bwd(x, conv_w, conv_b, dt_raw, A_log, B, C, D, dy, z=None, dt_bias=None, zoh=False, h_init=None,
+                  threads=None):
+    """Gradients of the fused path (causal conv + SiLU, then the scan) for the loss
+    sum(dy * y): the scan's backward on u = SiLU(conv(x)), then the conv's
+    backward on du.  Returns the dict of scan_bwd with du replaced by dx
+    [Bt, L, d], plus dconv_w [d, K] and dconv_b [d]."""
+    x = np.asarray(x)
+    Bt, L, d = x.shape
+    K = np.asarray(conv_w).shape[1]
+    u = conv_silu(x, conv_w, conv_b, threads=threads)
+    g = scan_bwd(u, dt_raw, A_log, B, C, D, dy, z=z, dt_bias=dt_bias, zoh=zoh, h_init=h_init, threads=threads)
+    n = Bt * d
+    xs = np.ascontiguousarray(np.transpose(_f64(x), (0, 2, 1))).reshape(n, L)
+    dxc = np.ascontiguousarray(np.transpose(g.pop("du"), (0, 2, 1))).reshape(n, L)
+    cw = np.ascontiguousarray(np.tile(_f64(conv_w), (Bt, 1)))
+    cbias = np.ascontiguousarray(np.tile(_f64(conv_b), Bt)) if conv_b is not None else None
+    dx, dw, db = np.zeros((n, L)), np.zeros((n, K)), np.zeros(n)
+    _load().s6o_conv_silu_bwd_channels(n, L, K, _ptr(xs), _ptr(cw), _ptr(cbias), _ptr(dxc), _ptr(dx), _ptr(dw),
+                                      _ptr(db))
+    g["dx"] = np.transpose(dx.reshape(Bt, d, L), (0, 2, 1))
+    g["dconv_w"] = dw.reshape(Bt, d, K).sum(axis=0)
+    g["dconv_b"] = db.reshape(Bt, d).sum(axis=0)
+    return g
 
 
 def conv_silu(x, conv_w, conv_b=None, threads=None):

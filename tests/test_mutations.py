@@ -41,6 +41,7 @@ ALL_PINS = [
     TB.test_sigmoid_and_dsilu_closed_forms,
     lambda: TB.check_gradients_by_central_differences(False, True),
     lambda: TB.check_gradients_by_central_differences(True, True),
+    lambda: TB.check_fused_gradients_by_central_differences(False),
 ]
 
 MUTATIONS = {
@@ -76,6 +77,9 @@ MUTATIONS = {
     "bwd_du_misses_D": ("double dut = ds * D;", "double dut = 0.0 * ds;"),
     "bwd_gate_not_applied": ("double ds = dy[t] * gate;", "double ds = dy[t];"),
     "bwd_write_gain_missing_in_dB": ("dB[t * N + n] += dh * gain * u[t];", "dB[t * N + n] += dh * u[t];"),
+    "cbwd_no_dsilu": ("double dpre = dxc[c * L + t] * s6o_dsilu(pre);", "double dpre = dxc[c * L + t];"),
+    "cbwd_dx_taps_reversed": ("dxo[src] += w[k] * dpre;", "dxo[src] += w[K - 1 - k] * dpre;"),
+    "cbwd_dw_wrong_input": ("dw[c * K + k] += dpre * xc[src];", "dw[c * K + k] += dpre * xc[t];"),
 }
 
 

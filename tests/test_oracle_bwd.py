@@ -92,3 +92,44 @@ def test_gradient_of_linear_readout_is_state():
         _, h_t = O.scan(p["u"][:, :t + 1], p["dt"][:, :t + 1], p["A_log"], p["B"][:, :t + 1], p["C"][:, :t + 1],
                         p["D"], dt_bias=p["dt_bias"], h_init=p["h_init"], threads=1)
         np.testing.assert_allclose(g["dC"][0, t], dy[0, t, 0] * h_t[0, 0], rtol=1e-14, atol=1e-15)
+
+
+def check_fused_gradients_by_central_differences(zoh, seed=4):
+    """The fused path (conv + SiLU, then the scan): every gradient, including
+    those of x, conv_w and conv_b, equals the central difference of the fused
+    forward oracle."""
+    p, dy = _problem(seed, Bt=2, L=6, d=2, N=3)
+    rng = np.random.default_rng(seed + 9)
+    K = 3
+    p["x"] = p.pop("u")
+    p["conv_w"] = rng.uniform(-0.8, 0.8, (2, K))
+    p["conv_b"] = rng.uniform(-0.3, 0.3, 2)
+
+    def loss(q):
+        y, _ = O.scan(q["x"], q["dt"], q["A_log"], q["B"], q["C"], q["D"], z=q["z"], dt_bias=q["dt_bias"], zoh=zoh,
+                      conv_w=q["conv_w"], conv_b=q["conv_b"], h_init=q["h_init"], threads=1)
+        return float(np.sum(y * dy))
+
+    g = O.conv_scan_bwd(p["x"], p["conv_w"], p["conv_b"], p["dt"], p["A_log"], p["B"], p["C"], p["D"], dy,
+                        z=p["z"], dt_bias=p["dt_bias"], zoh=zoh, h_init=p["h_init"], threads=1)
+    an = {"x": g["dx"], "conv_w": g["dconv_w"], "conv_b": g["dconv_b"], "dt": g["ddt"], "z": g["dz"], "B": g["dB"],
+          "C": g["dC"], "A_log": g["dA_log"], "D": g["dD"], "dt_bias": g["ddt_bias"], "h_init": g["dh_init"]}
+    for name, ref in an.items():
+        base = p[name]
+        fd = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            eps = 1e-6 * max(1.0, abs(base[idx]))
+            q = dict(p)
+            q[name] = base.copy()
+            q[name][idx] = base[idx] + eps
+            lp = loss(q)
+            q[name][idx] = base[idx] - eps
+            lm = loss(q)
+            fd[idx] = (lp - lm) / (2 * eps)
+        err = np.max(np.abs(fd - ref) / (1.0 + np.abs(fd)))
+        assert err < 1e-6, f"{name} (zoh={zoh}): max rel diff {err:.2e}"
+
+
+@pytest.mark.parametrize("zoh", [False, True])
+def test_fused_gradients_equal_central_differences(zoh):
+    check_fused_gradients_by_central_differences(zoh)
