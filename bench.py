@@ -296,9 +296,10 @@ def row_prefill(device, stream, pk, inp_dev, cfg, chunks=4, iters=10):
                          "frac": ex2_per_s / peak_ex2}}
 
 
-def row_bwd(device, stream, pk, inp_dev, cfg, iters=3):
-    """Backward pass of the scan (s6_scan_bwd) on the long_seq workload's
-    (u, dt, z, B, C): the gradients of sum(dy * y) for a random dy."""
+def row_bwd(device, stream, pk, inp_dev, cfg, iters=3, fused=False):
+    """Backward pass of the scan (s6_scan_bwd; with `fused`, of the conv + scan,
+    s6_conv_scan_bwd) on the long_seq workload's inputs: the gradients of
+    sum(dy * y) for a random dy."""
     import selective_state_space_19_b200 as S
     import torch
     Bt, L, d, N = cfg["Bt"], cfg["L"], cfg["d"], cfg["N"]
@@ -308,8 +309,12 @@ def row_bwd(device, stream, pk, inp_dev, cfg, iters=3):
     zoh = int(bool(cfg["zoh"]))
 
     def bwd():
-        S.s6_scan_bwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], t["D"], dy, z=t["z"], dt_bias=t["dt_bias"],
-                      zoh_mode=zoh, stream=stream)
+        if fused:
+            S.s6_conv_scan_bwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"], dy,
+                               z=t["z"], dt_bias=t["dt_bias"], zoh_mode=zoh, stream=stream)
+        else:
+            S.s6_scan_bwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], t["D"], dy, z=t["z"], dt_bias=t["dt_bias"],
+                          zoh_mode=zoh, stream=stream)
 
     with torch.cuda.stream(stream):
         bwd()
@@ -319,7 +324,8 @@ def row_bwd(device, stream, pk, inp_dev, cfg, iters=3):
     elems = Bt * L * d
     ex2_per_s = elems * N / (ms * 1e-3)
     peak_ex2 = SMS * MUFU_PER_SM_CLK * pk["sm_max_mhz"] * 1e6
-    return {"workload": "s6_scan_bwd on long_seq (Bt16 L8192 d1536 N16, bf16 in, float32 gradients, gate, "
+    name = "s6_conv_scan_bwd (conv4 + SiLU + scan)" if fused else "s6_scan_bwd"
+    return {"workload": f"{name} on long_seq (Bt16 L8192 d1536 N16, bf16 in, float32 gradients, gate, "
                         "simplified write): all gradients of sum(dy * y)",
             "value": elems / (ms * 1e-3) / 1e9, "unit": "Gelem/s", "ms_per_launch": ms,
             "roofline": {"bound": "alu", "achieved": ex2_per_s / 1e12, "peak": peak_ex2 / 1e12, "unit": "Tex2/s",
@@ -530,6 +536,7 @@ def run_ours(args):
         rows["causal_conv1d_silu_fwd"] = row_conv(device, stream, pk, t, cfg)
         rows["s6_conv_scan_fwd_from_state"] = row_prefill(device, stream, pk, t, cfg)
         rows["s6_scan_bwd"] = row_bwd(device, stream, pk, t, cfg)
+        rows["s6_conv_scan_bwd"] = row_bwd(device, stream, pk, t, cfg, fused=True)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

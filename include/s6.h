@@ -228,6 +228,25 @@ S6_API int s6_scan_bwd(const s6_dims *dims, const void *u, const void *dt, const
                        float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream);
 
 /*
+ * s6_conv_scan_bwd -- gradients of the fused path (s6_conv_scan_fwd_from_state
+ * with a zero conv history) for the loss sum(dy * y): the scan's gradients as
+ * in s6_scan_bwd, carried through SiLU and the causal conv.  In addition to
+ * s6_scan_bwd's arguments (with x, the pre-conv input, in place of u):
+ *
+ *  conv_w  [d,K] f32, conv_b [d] f32 (NULL = zeros)   as in the forward
+ *  dx      [Bt,L,d]  f32  with respect to x (written; replaces du)
+ *  dconv_w [d,K]     f32  with respect to conv_w (zeroed, then accumulated)
+ *  dconv_b [d]       f32  with respect to conv_b (NULL = not wanted)
+ */
+S6_API int s6_conv_scan_bwd(const s6_dims *dims, const void *x, const float *conv_w,
+                            const float *conv_b, const void *dt, const float *A_log,
+                            const void *B, const void *C, const float *D, const void *z,
+                            const float *dt_bias, int zoh_mode, const float *h_init,
+                            const void *dy, float *dx, float *dconv_w, float *dconv_b,
+                            float *ddt, float *dz, float *dB, float *dC, float *dA_log,
+                            float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream);
+
+/*
  * causal_conv1d_silu_fwd -- the conv + SiLU alone ("mamba, live":
  * depthwise_conv4 then SiLU; "Carry context ...", step "local").
  *

@@ -8,7 +8,7 @@ There is no CPU fallback: if the library is missing, the first call raises.
 
 Functions (same names as the C ABI):
     s6_scan_fwd, s6_conv_scan_fwd, s6_conv_scan_fwd_noalloc, s6_scan_fwd_from_state,
-    s6_conv_scan_fwd_from_state, s6_scan_bwd, causal_conv1d_silu_fwd, s6_step,
+    s6_conv_scan_fwd_from_state, s6_scan_bwd, s6_conv_scan_bwd, causal_conv1d_silu_fwd, s6_step,
     s6_device_status, s6_status_string, s6_version
 """
 from __future__ import annotations
@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "S6Error", "lib", "s6_scan_fwd", "s6_conv_scan_fwd", "s6_conv_scan_fwd_noalloc", "s6_scan_fwd_from_state",
-    "s6_conv_scan_fwd_from_state", "s6_scan_bwd", "causal_conv1d_silu_fwd", "s6_step",
+    "s6_conv_scan_fwd_from_state", "s6_scan_bwd", "s6_conv_scan_bwd", "causal_conv1d_silu_fwd", "s6_step",
     "s6_device_status", "s6_status_string", "s6_version", "S6_F32", "S6_BF16", "Dims",
 ]
 
@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
         L.s6_scan_fwd_from_state.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]
         L.s6_conv_scan_fwd_from_state.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]
         L.s6_scan_bwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P] + [_P] * 9 + [_P]
+        L.s6_conv_scan_bwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P] + [_P] * 11 + [_P]
         L.causal_conv1d_silu_fwd.argtypes = [DP, _P, _P, _P, _P, _P]
         L.s6_step.argtypes = [DP, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.s6_device_status.argtypes = [_P]
@@ -70,7 +71,7 @@ def lib() -> ctypes.CDLL:
         L.s6_status_string.restype = ctypes.c_char_p
         L.s6_version.argtypes = []
         for f in (L.s6_scan_fwd, L.s6_conv_scan_fwd, L.s6_conv_scan_fwd_noalloc, L.s6_scan_fwd_from_state,
-                  L.s6_conv_scan_fwd_from_state, L.s6_scan_bwd, L.causal_conv1d_silu_fwd, L.s6_step,
+                  L.s6_conv_scan_fwd_from_state, L.s6_scan_bwd, L.s6_conv_scan_bwd, L.causal_conv1d_silu_fwd, L.s6_step,
                   L.s6_device_status, L.s6_version):
             f.restype = _I
         _lib = L
@@ -235,6 +236,44 @@ def s6_scan_bwd(u, dt, A_log, B, C, D, dy, z=None, dt_bias=None, zoh_mode=0, h_i
                                                      "dh_init")],
                            _stream(stream, dev))
     _check(st, "s6_scan_bwd")
+    return g
+
+
+def s6_conv_scan_bwd(x, conv_w, conv_b, dt, A_log, B, C, D, dy, z=None, dt_bias=None, zoh_mode=0, h_init=None,
+                     want_dh_init=False, stream=None):
+    """Gradients of s6_conv_scan_fwd for the loss sum(dy * y).  Returns the dict of
+    s6_scan_bwd with dx [Bt, L, d] in place of du, plus dconv_w [d, K] and dconv_b
+    [d] (None without conv_b)."""
+    torch = _torch()
+    if x.dim() != 3:
+        raise ValueError("x must be [batch, seqlen, d_inner]")
+    Bt, L, d = x.shape
+    N = A_log.shape[-1]
+    K = conv_w.shape[-1]
+    dev = x.device
+    f32 = torch.float32
+    seq = (Bt, L, d)
+    g = {"dx": torch.empty(seq, dtype=f32, device=dev),
+         "dconv_w": torch.empty((d, K), dtype=f32, device=dev),
+         "dconv_b": torch.empty((d,), dtype=f32, device=dev) if conv_b is not None else None,
+         "ddt": torch.empty(seq, dtype=f32, device=dev),
+         "dz": torch.empty(seq, dtype=f32, device=dev) if z is not None else None,
+         "dB": torch.empty((Bt, L, N), dtype=f32, device=dev), "dC": torch.empty((Bt, L, N), dtype=f32, device=dev),
+         "dA_log": torch.empty((d, N), dtype=f32, device=dev), "dD": torch.empty((d,), dtype=f32, device=dev),
+         "ddt_bias": torch.empty((d,), dtype=f32, device=dev) if dt_bias is not None else None,
+         "dh_init": torch.empty((Bt, d, N), dtype=f32, device=dev) if want_dh_init else None}
+    dims = Dims(Bt, L, d, N, K, _io_code(x))
+    io = x.dtype
+    st = lib().s6_conv_scan_bwd(ctypes.byref(dims), _ptr(x, "x", io, seq, dev), _ptr(conv_w, "conv_w", f32, (d, K), dev),
+                                _ptr(conv_b, "conv_b", f32, (d,), dev), _ptr(dt, "dt", io, seq, dev),
+                                _ptr(A_log, "A_log", f32, (d, N), dev), _ptr(B, "B", io, (Bt, L, N), dev),
+                                _ptr(C, "C", io, (Bt, L, N), dev), _ptr(D, "D", f32, (d,), dev),
+                                _ptr(z, "z", io, seq, dev), _ptr(dt_bias, "dt_bias", f32, (d,), dev), int(zoh_mode),
+                                _ptr(h_init, "h_init", f32, (Bt, d, N), dev), _ptr(dy, "dy", io, seq, dev),
+                                *[_ptr(g[k], k) for k in ("dx", "dconv_w", "dconv_b", "ddt", "dz", "dB", "dC",
+                                                          "dA_log", "dD", "ddt_bias", "dh_init")],
+                                _stream(stream, dev))
+    _check(st, "s6_conv_scan_bwd")
     return g
 
 

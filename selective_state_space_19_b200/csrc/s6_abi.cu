@@ -530,7 +530,7 @@ int launch_conv(const s6_dims *dims, const void *x, s6::ConvArgs a, cudaStream_t
 
 // ------------------------------------------------------------ backward dispatch
 // Checkpoints and chunk states live in the library-owned scratch buffer.
-template <typename IO, int NS, bool ZOH>
+template <typename IO, int NS, bool ZOH, bool CONV>
 int launch_bwd_t(s6::BwdArgs a, cudaStream_t st) {
     const long long G = static_cast<long long>(a.Bt) * a.d;
     const size_t ckf = static_cast<size_t>(a.nck) * NS * G;
@@ -544,17 +544,108 @@ int launch_bwd_t(s6::BwdArgs a, cudaStream_t st) {
     const long long grid = (G * s6::kBwdTPC + s6::kBwdThreads - 1) / s6::kBwdThreads;
     if (grid > 0x7fffffffLL)
         return S6_ERR_UNSUPPORTED;
-    s6::s6_scan_bwd_kernel<IO, NS, ZOH><<<static_cast<unsigned>(grid), s6::kBwdThreads, 0, st>>>(a);
+    s6::s6_scan_bwd_kernel<IO, NS, ZOH, CONV><<<static_cast<unsigned>(grid), s6::kBwdThreads, 0, st>>>(a);
     return launch_status(cudaGetLastError());
 }
 
-template <typename IO, bool ZOH>
+template <typename IO, bool ZOH, bool CONV>
 int launch_bwd_n(const s6::BwdArgs &a, cudaStream_t st) {
     if (a.N <= 4)
-        return launch_bwd_t<IO, 4, ZOH>(a, st);
+        return launch_bwd_t<IO, 4, ZOH, CONV>(a, st);
     if (a.N <= 8)
-        return launch_bwd_t<IO, 8, ZOH>(a, st);
-    return launch_bwd_t<IO, 16, ZOH>(a, st);
+        return launch_bwd_t<IO, 8, ZOH, CONV>(a, st);
+    return launch_bwd_t<IO, 16, ZOH, CONV>(a, st);
+}
+
+template <typename IO>
+int launch_bwd_io(const s6::BwdArgs &a, bool zoh, bool conv, cudaStream_t st) {
+    if (conv)
+        return zoh ? launch_bwd_n<IO, true, true>(a, st) : launch_bwd_n<IO, false, true>(a, st);
+    return zoh ? launch_bwd_n<IO, true, false>(a, st) : launch_bwd_n<IO, false, false>(a, st);
+}
+
+// The backward entry points share their checks and set-up; `conv` selects the
+// fused form (x, conv_w, conv_b in; dx, dconv_w, dconv_b out).
+int bwd_common(const s6_dims *dims, bool conv, const void *x, const float *conv_w, const float *conv_b,
+               const void *dt, const float *A_log, const void *B, const void *C, const float *D, const void *z,
+               const float *dt_bias, int zoh_mode, const float *h_init, const void *dy, float *dx,
+               float *dconv_w, float *dconv_b, float *ddt, float *dz, float *dB, float *dC, float *dA_log, float *dD,
+               float *ddt_bias, float *dh_init, s6_stream_t stream) {
+    int st = check_dims(dims, true, conv);
+    if (st != S6_OK)
+        return st;
+    if (zoh_mode != 0 && zoh_mode != 1)
+        return S6_ERR_INVALID_ARG;
+    if (dims->batch == 0)
+        return S6_OK;
+    if (!x || !dt || !A_log || !B || !C || !D || !dy || !dx || !ddt || !dB || !dC || !dA_log || !dD || (z && !dz) ||
+        (conv && (!conv_w || !dconv_w)))
+        return S6_ERR_INVALID_ARG;
+    const size_t es = io_size(dims->io_dtype);
+    const void *io_ptrs[] = {x, dt, B, C, z, dy};
+    for (const void *p : io_ptrs)
+        if (p && !aligned_to(p, es))
+            return S6_ERR_ALIGNMENT;
+    const void *f32_ptrs[] = {A_log, D, dt_bias, h_init, conv_w, conv_b, dx, ddt, dz, dB, dC, dA_log, dD,
+                              ddt_bias, dh_init, dconv_w, dconv_b};
+    for (const void *p : f32_ptrs)
+        if (p && !aligned_to(p, 4))
+            return S6_ERR_ALIGNMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (use_stream_device(s) != S6_OK)
+        return S6_ERR_CUDA;
+    // the summed gradients start from zero
+    const int64_t Bt = dims->batch, L = dims->seqlen, d = dims->d_inner, N = dims->d_state;
+    const int64_t K = conv ? dims->conv_width : 0;
+    if (cudaMemsetAsync(dB, 0, sizeof(float) * Bt * L * N, s) != cudaSuccess ||
+        cudaMemsetAsync(dC, 0, sizeof(float) * Bt * L * N, s) != cudaSuccess ||
+        cudaMemsetAsync(dA_log, 0, sizeof(float) * d * N, s) != cudaSuccess ||
+        cudaMemsetAsync(dD, 0, sizeof(float) * d, s) != cudaSuccess ||
+        (ddt_bias && cudaMemsetAsync(ddt_bias, 0, sizeof(float) * d, s) != cudaSuccess) ||
+        (conv && cudaMemsetAsync(dconv_w, 0, sizeof(float) * d * K, s) != cudaSuccess) ||
+        (conv && dconv_b && cudaMemsetAsync(dconv_b, 0, sizeof(float) * d, s) != cudaSuccess))
+        return S6_ERR_CUDA;
+    if (L == 0) {
+        // an empty sequence contributes nothing; the start state gets no gradient
+        if (dh_init && cudaMemsetAsync(dh_init, 0, sizeof(float) * Bt * d * N, s) != cudaSuccess)
+            return S6_ERR_CUDA;
+        return S6_OK;
+    }
+    s6::BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.Bt = static_cast<int>(Bt);
+    a.L = static_cast<int>(L);
+    a.d = static_cast<int>(d);
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.has_z = z != nullptr;
+    a.nck = static_cast<int>((L + s6::kBwdChunk - 1) / s6::kBwdChunk);
+    a.u = x;
+    a.dt = dt;
+    a.B = B;
+    a.C = C;
+    a.z = z;
+    a.dy = dy;
+    a.A_log = A_log;
+    a.D = D;
+    a.dt_bias = dt_bias;
+    a.h_init = h_init;
+    a.conv_w = conv_w;
+    a.conv_b = conv_b;
+    a.du = dx;
+    a.ddt = ddt;
+    a.dz = dz;
+    a.dB = dB;
+    a.dC = dC;
+    a.dA_log = dA_log;
+    a.dD = dD;
+    a.ddt_bias = ddt_bias;
+    a.dh_init = dh_init;
+    a.dconv_w = dconv_w;
+    a.dconv_b = dconv_b;
+    if (dims->io_dtype == S6_BF16)
+        return launch_bwd_io<__nv_bfloat16>(a, zoh_mode == 1, conv, s);
+    return launch_bwd_io<float>(a, zoh_mode == 1, conv, s);
 }
 
 extern "C" {
@@ -620,72 +711,17 @@ int s6_scan_bwd(const s6_dims *dims, const void *u, const void *dt, const float 
                 const float *D, const void *z, const float *dt_bias, int zoh_mode, const float *h_init, const void *dy,
                 float *du, float *ddt, float *dz, float *dB, float *dC, float *dA_log, float *dD, float *ddt_bias,
                 float *dh_init, s6_stream_t stream) {
-    int st = check_dims(dims, true, false);
-    if (st != S6_OK)
-        return st;
-    if (zoh_mode != 0 && zoh_mode != 1)
-        return S6_ERR_INVALID_ARG;
-    if (dims->batch == 0)
-        return S6_OK;
-    if (!u || !dt || !A_log || !B || !C || !D || !dy || !du || !ddt || !dB || !dC || !dA_log || !dD ||
-        (z && !dz))
-        return S6_ERR_INVALID_ARG;
-    const size_t es = io_size(dims->io_dtype);
-    const void *io_ptrs[] = {u, dt, B, C, z, dy};
-    for (const void *p : io_ptrs)
-        if (p && !aligned_to(p, es))
-            return S6_ERR_ALIGNMENT;
-    const void *f32_ptrs[] = {A_log, D, dt_bias, h_init, du, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init};
-    for (const void *p : f32_ptrs)
-        if (p && !aligned_to(p, 4))
-            return S6_ERR_ALIGNMENT;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (use_stream_device(s) != S6_OK)
-        return S6_ERR_CUDA;
-    // the summed gradients start from zero
-    const int64_t Bt = dims->batch, L = dims->seqlen, d = dims->d_inner, N = dims->d_state;
-    if (cudaMemsetAsync(dB, 0, sizeof(float) * Bt * L * N, s) != cudaSuccess ||
-        cudaMemsetAsync(dC, 0, sizeof(float) * Bt * L * N, s) != cudaSuccess ||
-        cudaMemsetAsync(dA_log, 0, sizeof(float) * d * N, s) != cudaSuccess ||
-        cudaMemsetAsync(dD, 0, sizeof(float) * d, s) != cudaSuccess ||
-        (ddt_bias && cudaMemsetAsync(ddt_bias, 0, sizeof(float) * d, s) != cudaSuccess))
-        return S6_ERR_CUDA;
-    if (L == 0) {
-        // an empty sequence contributes nothing; the start state gets no gradient
-        if (dh_init && cudaMemsetAsync(dh_init, 0, sizeof(float) * Bt * d * N, s) != cudaSuccess)
-            return S6_ERR_CUDA;
-        return S6_OK;
-    }
-    s6::BwdArgs a;
-    std::memset(&a, 0, sizeof(a));
-    a.Bt = static_cast<int>(Bt);
-    a.L = static_cast<int>(L);
-    a.d = static_cast<int>(d);
-    a.N = static_cast<int>(N);
-    a.has_z = z != nullptr;
-    a.nck = static_cast<int>((L + s6::kBwdChunk - 1) / s6::kBwdChunk);
-    a.u = u;
-    a.dt = dt;
-    a.B = B;
-    a.C = C;
-    a.z = z;
-    a.dy = dy;
-    a.A_log = A_log;
-    a.D = D;
-    a.dt_bias = dt_bias;
-    a.h_init = h_init;
-    a.du = du;
-    a.ddt = ddt;
-    a.dz = dz;
-    a.dB = dB;
-    a.dC = dC;
-    a.dA_log = dA_log;
-    a.dD = dD;
-    a.ddt_bias = ddt_bias;
-    a.dh_init = dh_init;
-    if (dims->io_dtype == S6_BF16)
-        return zoh_mode ? launch_bwd_n<__nv_bfloat16, true>(a, s) : launch_bwd_n<__nv_bfloat16, false>(a, s);
-    return zoh_mode ? launch_bwd_n<float, true>(a, s) : launch_bwd_n<float, false>(a, s);
+    return bwd_common(dims, false, u, nullptr, nullptr, dt, A_log, B, C, D, z, dt_bias, zoh_mode, h_init, dy, du,
+                      nullptr, nullptr, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, stream);
+}
+
+int s6_conv_scan_bwd(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b, const void *dt,
+                     const float *A_log, const void *B, const void *C, const float *D, const void *z,
+                     const float *dt_bias, int zoh_mode, const float *h_init, const void *dy, float *dx,
+                     float *dconv_w, float *dconv_b, float *ddt, float *dz, float *dB, float *dC, float *dA_log,
+                     float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream) {
+    return bwd_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, h_init, dy, dx,
+                      dconv_w, dconv_b, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, stream);
 }
 
 int causal_conv1d_silu_fwd(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b, void *out,

@@ -36,10 +36,12 @@ constexpr int kBwdChunk = 64;  // tokens between checkpoints
 constexpr int kBwdTPC = 4;     // threads per channel (N/4 states each)
 
 struct BwdArgs {
-    int Bt, L, d, N, has_z, nck;
-    const void *u, *dt, *B, *C, *z, *dy;
+    int Bt, L, d, N, K, has_z, nck;
+    const void *u, *dt, *B, *C, *z, *dy;  // u: the pre-conv x in the fused form
     const float *A_log, *D, *dt_bias, *h_init;
-    float *du, *ddt, *dz, *dB, *dC, *dA_log, *dD, *ddt_bias, *dh_init;
+    const float *conv_w, *conv_b;          // fused form: [d, K] taps oldest first, [d] or null
+    float *du, *ddt, *dz, *dB, *dC, *dA_log, *dD, *ddt_bias, *dh_init;  // du: dx in the fused form
+    float *dconv_w, *dconv_b;              // fused form: [d, K], [d] or null
     float *ck;  // [nck][NS/4][Bt*d*4] state at the start of each chunk
     float *hb;  // [kBwdChunk][NS/4][Bt*d*4] the states of the chunk being reversed
 };
@@ -58,7 +60,11 @@ __device__ __forceinline__ float zoh_dgain_dA(float x, float delta, float A) {
     return (x * expf(x) - expm1f(x)) / (A * A);
 }
 
-template <typename IO, int NS, bool ZOH>
+// CONV: the fused path -- u_t = SiLU(pre_t), pre_t = conv_b + sum_k w[k] x[t-K+1+k]
+// recomputed from x wherever it is needed; on the way back dpre_t =
+// du_t SiLU'(pre_t), and dx[s] = sum_k w[k] dpre_{s+K-1-k} collects the next
+// K-1 tokens' dpre from a sliding window, so each dx is final when written.
+template <typename IO, int NS, bool ZOH, bool CONV>
 __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs a) {
     using tr = io_traits<IO>;
     constexpr int T = kBwdChunk;
@@ -95,6 +101,16 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
     }
     const float Dd = a.D[c];
     const float bias = a.dt_bias ? a.dt_bias[c] : 0.0f;
+    // conv taps right-aligned into 4 slots (missing oldest taps are zero)
+    float w[4] = {0.f, 0.f, 0.f, 0.f}, cbv = 0.f;
+    if (CONV) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int src = k - (4 - a.K);
+            w[k] = src >= 0 ? a.conv_w[static_cast<size_t>(c) * a.K + src] : 0.0f;
+        }
+        cbv = a.conv_b ? a.conv_b[c] : 0.0f;
+    }
 
     auto seq = [&](const void *p, int t) -> float {
         return tr::to_f(static_cast<const IO *>(p)[(static_cast<size_t>(b) * a.L + t) * a.d + c]);
@@ -103,6 +119,23 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
         const int n = n0 + j;
         return (n < a.N) ? tr::to_f(static_cast<const IO *>(p)[(static_cast<size_t>(b) * a.L + t) * a.N + n]) : 0.0f;
     };
+    // the pre-conv input at token t (zero before the sequence)
+    auto xin = [&](int t) -> float { return t >= 0 ? seq(a.u, t) : 0.0f; };
+    auto conv_pre = [&](int t) -> float {
+        float p = cbv;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            p = fmaf(w[k], xin(t - 3 + k), p);
+        return p;
+    };
+    // the scan input u_t
+    auto uval = [&](int t) -> float {
+        if (CONV) {
+            const float p = conv_pre(t);
+            return p / (1.0f + expf(-p));  // SiLU
+        }
+        return seq(a.u, t);
+    };
     // scratch slot of this thread's state j at checkpoint / chunk row i
     auto slot = [&](float *base, int i, int j) -> float * {
         return base + (static_cast<size_t>(i) * NH + j) * GT + gtc;
@@ -110,7 +143,7 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
     // one forward token: h <- a h + gain B u
     auto step = [&](int t, float (&h)[NH]) {
         const float delta = softplus_f(seq(a.dt, t) + bias);
-        const float uu = seq(a.u, t);
+        const float uu = uval(t);
 #pragma unroll
         for (int j = 0; j < NH; ++j) {
             const float ab = ex2_approx(delta * A2[j]);
@@ -141,6 +174,8 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
     for (int j = 0; j < NH; ++j)
         gcar[j] = dA[j] = 0.0f;
     float dDa = 0.0f, dba = 0.0f;  // kept by the channel's first thread
+    float dW[4] = {0.f, 0.f, 0.f, 0.f}, dcb = 0.0f;  // conv taps, bias (first thread)
+    float dp1 = 0.f, dp2 = 0.f, dp3 = 0.f;            // dpre of tokens t+1, t+2, t+3
     for (int k = a.nck - 1; k >= 0; --k) {
         const int t0 = k * T, t1 = min(a.L, t0 + T);
         float hc[NH];
@@ -166,7 +201,13 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
                 hp[j] = live ? (t > t0 ? *slot(a.hb, t - t0 - 1, j) : *slot(a.ck, k, j)) : 0.0f;
             const float v = seq(a.dt, t) + bias;
             const float delta = softplus_f(v);
-            const float uu = seq(a.u, t);
+            float pre = 0.0f, uu;
+            if (CONV) {
+                pre = conv_pre(t);
+                uu = pre / (1.0f + expf(-pre));
+            } else {
+                uu = seq(a.u, t);
+            }
             const float dyv = live ? seq(a.dy, t) : 0.0f;
             float sp = 0.0f;
 #pragma unroll
@@ -214,8 +255,21 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
             if (q == 0) {
                 dDa = fmaf(ds, uu, dDa);
                 dba += dv;
+                float dxo = dut;
+                if (CONV) {
+                    const float sg = 1.0f / (1.0f + expf(-pre));
+                    const float dpre = dut * sg * (1.0f + pre * (1.0f - sg));  // SiLU'(pre)
+                    dxo = fmaf(w[3], dpre, fmaf(w[2], dp1, fmaf(w[1], dp2, w[0] * dp3)));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        dW[k] = fmaf(dpre, xin(t - 3 + k), dW[k]);
+                    dcb += dpre;
+                    dp3 = dp2;
+                    dp2 = dp1;
+                    dp1 = dpre;
+                }
                 if (live) {
-                    a.du[o] = dut;
+                    a.du[o] = dxo;
                     a.ddt[o] = dv;
                 }
             }
@@ -262,6 +316,16 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
         atomicAdd(a.dD + c, dDa);
         if (a.ddt_bias)
             atomicAdd(a.ddt_bias + c, dba);
+        if (CONV) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int src = k - (4 - a.K);
+                if (src >= 0)
+                    atomicAdd(a.dconv_w + static_cast<size_t>(c) * a.K + src, dW[k]);
+            }
+            if (a.dconv_b)
+                atomicAdd(a.dconv_b + c, dcb);
+        }
     }
 }
 

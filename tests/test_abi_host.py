@@ -137,6 +137,14 @@ def test_from_state_and_backward_host_checks(lib):
     assert bwd(dims=ctypes.byref(_dims(d_state=17))) == S.S6_ERR_UNSUPPORTED
     assert bwd(dims=ctypes.byref(_dims(batch=0))) == S.S6_OK  # nothing to do, nothing touched
 
+    def cbwd(dims=d, conv_w=ok, dconv_w=ok):  # s6_conv_scan_bwd
+        return lib.s6_conv_scan_bwd(dims, ok, conv_w, None, ok, ok, ok, ok, ok, None, None, 0, None, ok, ok,
+                                    dconv_w, None, ok, None, ok, ok, ok, ok, None, None, None)
+    assert cbwd(dims=ctypes.byref(_dims(conv_width=5))) == S.S6_ERR_UNSUPPORTED
+    assert cbwd(conv_w=None) == S.S6_ERR_INVALID_ARG
+    assert cbwd(dconv_w=None) == S.S6_ERR_INVALID_ARG
+    assert cbwd(conv_w=P(2)) == S.S6_ERR_ALIGNMENT
+
 
 def test_binding_refuses_cpu_tensors(lib):
     import torch
