@@ -15,6 +15,10 @@
  *       numerical example" and the manifest's steps "state"/"read": the exact
  *       zero-order hold B_bar = (exp(dt*A) - 1)/A * B, and C reading the
  *       UPDATED state.
+ * Entry points: the full-sequence scans (plain, fused with the conv, without
+ * allocation, or from a given state), the standalone conv, the single-token
+ * streaming step, and the gradients of the scans (reverse-mode
+ * differentiation of the same steps).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -79,7 +83,7 @@ typedef enum { S6_F32 = 0, S6_BF16 = 1 } s6_dtype;
 
 typedef struct {
     int64_t batch;      /* Bt >= 0 (0: nothing to do)                          */
-    int64_t seqlen;     /* L  >= 0 (0: nothing to do); ignored by s6_step      */
+    int64_t seqlen;     /* L  >= 0 (0: nothing to scan); ignored by s6_step    */
     int64_t d_inner;    /* d  >= 1                                             */
     int64_t d_state;    /* N  in [1, 16]                                       */
     int64_t conv_width; /* K  in [2, 4] for calls that apply the conv          */
