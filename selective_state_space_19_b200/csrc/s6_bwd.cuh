@@ -121,34 +121,82 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
     };
     // the pre-conv input at token t (zero before the sequence)
     auto xin = [&](int t) -> float { return t >= 0 ? seq(a.u, t) : 0.0f; };
-    auto conv_pre = [&](int t) -> float {
-        float p = cbv;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            p = fmaf(w[k], xin(t - 3 + k), p);
-        return p;
-    };
-    // the scan input u_t
-    auto uval = [&](int t) -> float {
-        if (CONV) {
-            const float p = conv_pre(t);
-            return p / (1.0f + expf(-p));  // SiLU
-        }
-        return seq(a.u, t);
-    };
     // scratch slot of this thread's state j at checkpoint / chunk row i
     auto slot = [&](float *base, int i, int j) -> float * {
         return base + (static_cast<size_t>(i) * NH + j) * GT + gtc;
     };
     // one forward token: h <- a h + gain B u
-    auto step = [&](int t, float (&h)[NH]) {
-        const float delta = softplus_f(seq(a.dt, t) + bias);
-        const float uu = uval(t);
+    // A token's inputs: raw dt, the conv window x[t-3..t] (x[3] alone is u
+    // without the conv), dy, z, and this thread's B and C values.  In the
+    // fused form (PF) they are read one token ahead of their use, so that the
+    // window's loads overlap the previous token's arithmetic; without the conv
+    // the extra registers cost more than the overlap gains (measured), and each
+    // token's inputs are read when it starts.
+    constexpr bool PF = CONV;
+    struct Tok {
+        float dt, x[4], dy, z, B[NH], C[NH];
+    };
+    auto load_tok = [&](int t, Tok &k, bool rev) {
+        k.dt = seq(a.dt, t);
+        if (CONV) {
+#pragma unroll
+            for (int i = 0; i < 3; ++i)
+                k.x[i] = xin(t - 3 + i);
+        }
+        k.x[3] = seq(a.u, t);
+#pragma unroll
+        for (int j = 0; j < NH; ++j)
+            k.B[j] = row(a.B, t, j);
+        if (rev) {
+            k.dy = live ? seq(a.dy, t) : 0.0f;
+            k.z = a.has_z ? seq(a.z, t) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < NH; ++j)
+                k.C[j] = row(a.C, t, j);
+        }
+    };
+    auto pre_of = [&](const Tok &k) {
+        float p = cbv;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            p = fmaf(w[i], k.x[i], p);
+        return p;
+    };
+    auto u_of = [&](const Tok &k) {
+        if (CONV) {
+            const float p = pre_of(k);
+            return p / (1.0f + expf(-p));  // SiLU
+        }
+        return k.x[3];
+    };
+    auto step = [&](const Tok &k, float (&h)[NH]) {
+        const float delta = softplus_f(k.dt + bias);
+        const float uu = u_of(k);
 #pragma unroll
         for (int j = 0; j < NH; ++j) {
             const float ab = ex2_approx(delta * A2[j]);
             const float gain = ZOH ? ((n0 + j < a.N) ? zoh_gain(delta * A[j], A[j]) : 0.0f) : delta;
-            h[j] = fmaf(ab, h[j], gain * row(a.B, t, j) * uu);
+            h[j] = fmaf(ab, h[j], gain * k.B[j] * uu);
+        }
+    };
+    // forward over tokens [ta, tb) from h; `keep` stores each state in the chunk buffer
+    auto walk = [&](int ta, int tb, float (&h)[NH], bool keep) {
+        Tok cur, nxt;
+        if (PF)
+            load_tok(ta, cur, false);
+        for (int t = ta; t < tb; ++t) {
+            if (!PF)
+                load_tok(t, cur, false);
+            else if (t + 1 < tb)
+                load_tok(t + 1, nxt, false);
+            step(cur, h);
+            if (keep && live) {
+#pragma unroll
+                for (int j = 0; j < NH; ++j)
+                    *slot(a.hb, t - ta, j) = h[j];
+            }
+            if (PF)
+                cur = nxt;
         }
     };
 
@@ -163,9 +211,7 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
             for (int j = 0; j < NH; ++j)
                 *slot(a.ck, k, j) = h[j];
         }
-        const int t1 = min(a.L, (k + 1) * T);
-        for (int t = k * T; t < t1; ++t)
-            step(t, h);
+        walk(k * T, min(a.L, (k + 1) * T), h, false);
     }
 
     // ---- pass 2: chunks last to first
@@ -182,42 +228,54 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
 #pragma unroll
         for (int j = 0; j < NH; ++j)
             hc[j] = live ? *slot(a.ck, k, j) : 0.0f;
-        for (int t = t0; t < t1; ++t) {
-            step(t, hc);
-            if (live) {
-#pragma unroll
-                for (int j = 0; j < NH; ++j)
-                    *slot(a.hb, t - t0, j) = hc[j];
-            }
-        }
+        walk(t0, t1, hc, true);
         float ht[NH];  // h_t; the state after the chunk's last token is still in hc
 #pragma unroll
         for (int j = 0; j < NH; ++j)
             ht[j] = live ? hc[j] : 0.0f;
-        for (int t = t1 - 1; t >= t0; --t) {
-            float hp[NH];  // h_{t-1}
+        // h_{t-1} of token t: the chunk buffer's previous row, or the checkpoint
+        auto load_prev = [&](int t, float (&hp)[NH]) {
 #pragma unroll
             for (int j = 0; j < NH; ++j)
                 hp[j] = live ? (t > t0 ? *slot(a.hb, t - t0 - 1, j) : *slot(a.ck, k, j)) : 0.0f;
-            const float v = seq(a.dt, t) + bias;
+        };
+        Tok cur, nxt;
+        float hpc[NH], hpn[NH];
+        if (PF) {
+            load_tok(t1 - 1, cur, true);
+            load_prev(t1 - 1, hpc);
+        }
+        for (int t = t1 - 1; t >= t0; --t) {
+            if (!PF) {
+                load_tok(t, cur, true);
+                load_prev(t, hpc);
+            } else if (t - 1 >= t0) {
+                load_tok(t - 1, nxt, true);
+                load_prev(t - 1, hpn);
+            }
+            float hp[NH];  // h_{t-1}
+#pragma unroll
+            for (int j = 0; j < NH; ++j)
+                hp[j] = hpc[j];
+            const float v = cur.dt + bias;
             const float delta = softplus_f(v);
             float pre = 0.0f, uu;
             if (CONV) {
-                pre = conv_pre(t);
+                pre = pre_of(cur);
                 uu = pre / (1.0f + expf(-pre));
             } else {
-                uu = seq(a.u, t);
+                uu = cur.x[3];
             }
-            const float dyv = live ? seq(a.dy, t) : 0.0f;
+            const float dyv = cur.dy;
             float sp = 0.0f;
 #pragma unroll
             for (int j = 0; j < NH; ++j)
-                sp = fmaf(ht[j], row(a.C, t, j), sp);
+                sp = fmaf(ht[j], cur.C[j], sp);
             const float s = fmaf(Dd, uu, chan_sum(sp));
             float gate = 1.0f;
             const size_t o = (static_cast<size_t>(b) * a.L + t) * a.d + c;
             if (a.has_z) {
-                const float zv = seq(a.z, t);
+                const float zv = cur.z;
                 const float sg = 1.0f / (1.0f + expf(-zv));
                 gate = zv * sg;
                 if (live && q == 0)
@@ -229,7 +287,7 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
 #pragma unroll
             for (int j = 0; j < NH; ++j) {
                 const float ab = ex2_approx(delta * A2[j]);
-                const float Bn = row(a.B, t, j), Cn = row(a.C, t, j);
+                const float Bn = cur.B[j], Cn = cur.C[j];
                 const bool inN = n0 + j < a.N;
                 const float gain = ZOH ? (inN ? zoh_gain(delta * A[j], A[j]) : 0.0f) : delta;
                 dCn[j] = ds * ht[j];
@@ -261,8 +319,8 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
                     const float dpre = dut * sg * (1.0f + pre * (1.0f - sg));  // SiLU'(pre)
                     dxo = fmaf(w[3], dpre, fmaf(w[2], dp1, fmaf(w[1], dp2, w[0] * dp3)));
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        dW[k] = fmaf(dpre, xin(t - 3 + k), dW[k]);
+                    for (int i = 0; i < 4; ++i)
+                        dW[i] = fmaf(dpre, cur.x[i], dW[i]);
                     dcb += dpre;
                     dp3 = dp2;
                     dp2 = dp1;
@@ -301,6 +359,12 @@ __global__ void __launch_bounds__(kBwdThreads) s6_scan_bwd_kernel(const BwdArgs 
 #pragma unroll
             for (int j = 0; j < NH; ++j)
                 ht[j] = hp[j];
+            if (PF) {
+#pragma unroll
+                for (int j = 0; j < NH; ++j)
+                    hpc[j] = hpn[j];
+                cur = nxt;
+            }
         }
     }
     if (!live)
