@@ -393,3 +393,51 @@ int64_t s6o_conv_history_values(int64_t d_inner, int64_t K, int64_t blocks)
 {
     return d_inner * (K - 1) * blocks;
 }
+
+/* ------------------------------------------------ constant-decay recurrence
+ * The diagonal recurrence cell of "the s6 cell", sections "one cell, two
+ * architectures" and "the difference that no engineering removes": the same
+ * line h <- a*h + b*u with a = 2^(negative), but the decay taken from a
+ * constant instead of computed per token.  With state width N per channel:
+ *   a[n] = 2^w[n]  (w[n] <= 0, a per-channel constant, precomputed once)
+ *   h[n] <- a[n] * h[n] + B_t[n] * u_t          (no step size: b = B_t)
+ *   y_t  = (<h, C_t> + D * u_t) * SiLU(z_t)     (the S6 cell's readout; z optional)
+ * RWKV's normaliser branch is not part of this cell (the pages give it no
+ * formula).
+ */
+void s6o_diag_const_channel(int64_t L, int N, const double *u, const double *z,
+                            const double *Bm, const double *Cm, const double *log2_decay,
+                            double D, const double *h_in, double *y, double *h_out)
+{
+    double h[64], a[64];
+    for (int n = 0; n < N; ++n) {
+        h[n] = h_in ? h_in[n] : 0.0;
+        a[n] = exp2(log2_decay[n]);
+    }
+    for (int64_t t = 0; t < L; ++t) {
+        double acc = 0.0;
+        for (int n = 0; n < N; ++n) {
+            h[n] = s6o_update(h[n], a[n], Bm[t * N + n] * u[t]);
+            acc += h[n] * Cm[t * N + n];
+        }
+        double out = acc + D * u[t];
+        if (z)
+            out *= s6o_silu(z[t]);
+        y[t] = out;
+    }
+    if (h_out)
+        for (int n = 0; n < N; ++n)
+            h_out[n] = h[n];
+}
+
+/* Many channels, laid out as in s6o_scan_channels (log2_decay + c*N). */
+void s6o_diag_const_channels(int64_t n_ch, int64_t L, int N, const double *u, const double *z,
+                             const double *Bm, const double *Cm, const int64_t *bc_row,
+                             const double *log2_decay, const double *D, const double *h_in,
+                             double *y, double *h_out)
+{
+    for (int64_t c = 0; c < n_ch; ++c)
+        s6o_diag_const_channel(L, N, u + c * L, z ? z + c * L : NULL, Bm + bc_row[c] * L * N,
+                               Cm + bc_row[c] * L * N, log2_decay + c * N, D[c],
+                               h_in ? h_in + c * N : NULL, y + c * L, h_out ? h_out + c * N : NULL);
+}

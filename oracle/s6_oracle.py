@@ -18,6 +18,9 @@ What the oracle computes (page titles and sections):
   model manifest, ``steps`` *local/select/state/read*) -- exact diagonal
   zero-order hold ``B_bar = (exp(dt*A) - 1)/A * B``, a zero-left-padded causal
   conv, C reading the updated state, D multiplying the conv output.
+* ``diag_const`` -- "the s6 cell", *one cell, two architectures*: the same
+  diagonal recurrence with a constant decay 2^w per (channel, state) instead of
+  a per-token one, written B_t * u_t.
 * ``scan_bwd`` -- the gradients of that scan (no conv), by reverse-mode
   differentiation of the same steps; pinned by central differences of the
   forward oracle.
@@ -76,6 +79,8 @@ def bind(path: str):
     lib.s6o_scan_bwd_channels.restype = None
     lib.s6o_conv_silu_bwd_channels.argtypes = [i64, i64, i] + [_c_double_p] * 7
     lib.s6o_conv_silu_bwd_channels.restype = None
+    lib.s6o_diag_const_channels.argtypes = [i64, i64, i] + [_c_double_p] * 4 + [_c_i64_p] + [_c_double_p] * 5
+    lib.s6o_diag_const_channels.restype = None
     for name in ("s6o_ssm_state_values", "s6o_conv_history_values"):
         f = getattr(lib, name)
         f.argtypes, f.restype = [i64, i64, i64], i64
@@ -256,6 +261,62 @@ def scan(x, dt_raw, A_log, B, C, D, z=None, dt_bias=None, zoh=False, conv_w=None
         hs = histout[:, :km1].reshape(Bt, d, km1)
         return (y_full, h_full, hs) if return_state else (y_full, h_full)
     return (y, hout, histout[:, :km1]) if return_state else (y, hout)
+
+
+def diag_const(u, log2_decay, B, C, D, z=None, channels=None, h_init=None, threads=None):
+    """The constant-decay diagonal recurrence ("the s6 cell", *one cell, two
+    architectures*): h <- 2^w * h + B_t * u_t per state, y = (<h, C_t> + D u) * SiLU(z).
+
+    u, z: [Bt, L, d]; B, C: [Bt, L, N]; log2_decay (w <= 0): [d, N]; D: [d];
+    h_init: [Bt, d, N] or None.  ``channels`` as in ``scan``.  Returns (y, h_final)
+    in float64: [Bt, L, d] / [Bt, d, N], or [n, L] / [n, N] for a channel list.
+    """
+    u = np.asarray(u)
+    Bt, L, d = u.shape
+    N = np.asarray(log2_decay).shape[1]
+    full = channels is None
+    if full:
+        bb, dd = np.meshgrid(np.arange(Bt), np.arange(d), indexing="ij")
+        channels = np.stack([bb.ravel(), dd.ravel()], axis=1)
+    channels = np.asarray(channels, dtype=np.int64).reshape(-1, 2)
+    n = channels.shape[0]
+    cb, cd = channels[:, 0], channels[:, 1]
+
+    def gather_seq(a):
+        return np.ascontiguousarray(_f64(np.asarray(a)[cb, :, cd]).reshape(n, L))
+
+    us = gather_seq(u)
+    zs = gather_seq(z) if z is not None else None
+    Bm = np.ascontiguousarray(_f64(B)).reshape(-1)
+    Cm = np.ascontiguousarray(_f64(C)).reshape(-1)
+    bc_row = np.ascontiguousarray(cb)
+    W = np.ascontiguousarray(_f64(log2_decay)[cd])
+    Dv = np.ascontiguousarray(_f64(D)[cd])
+    hin = None
+    if h_init is not None:
+        hin = np.ascontiguousarray(_f64(h_init)[cb, cd] if full else _f64(h_init)).reshape(n, N)
+    y = np.zeros((n, L))
+    hout = np.zeros((n, N))
+    lib = _load()
+
+    def run(lo, hi):
+        sl = slice(lo, hi)
+
+        def p(a):
+            return None if a is None else _ptr(a[sl])
+
+        lib.s6o_diag_const_channels(hi - lo, L, N, p(us), p(zs), _ptr(Bm), _ptr(Cm),
+                                    bc_row[sl].ctypes.data_as(_c_i64_p), p(W), p(Dv), p(hin), p(y), p(hout))
+
+    nt = _threads(n, threads)
+    bounds = np.linspace(0, n, nt + 1).astype(np.int64)
+    with ThreadPoolExecutor(nt) as ex:
+        list(ex.map(lambda i: run(int(bounds[i]), int(bounds[i + 1])), range(nt)))
+    if full:
+        y_full = np.zeros((Bt, L, d))
+        y_full[cb, :, cd] = y
+        return y_full, hout.reshape(Bt, d, N)
+    return y, hout
 
 
 def scan_bwd(u, dt_raw, A_log, B, C, D, dy, z=None, dt_bias=None, zoh=False, h_init=None, threads=None):

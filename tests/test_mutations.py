@@ -11,6 +11,7 @@ import pytest
 
 from oracle import s6_oracle as O
 import test_oracle_bwd as TB
+import test_oracle_diag as TD
 import test_oracle_pins as P
 
 SRC = os.path.join(os.path.dirname(O.__file__), "s6_oracle.c")
@@ -42,6 +43,11 @@ ALL_PINS = [
     lambda: TB.check_gradients_by_central_differences(False, True),
     lambda: TB.check_gradients_by_central_differences(True, True),
     lambda: TB.check_fused_gradients_by_central_differences(False),
+    TD.test_diag_bruteforce_decayed_sum,
+    TD.test_diag_geometric_series,
+    TD.test_diag_equals_selective_scan_at_unit_step,
+    TD.test_diag_decays_in_unit_interval_and_state_bounded,
+    TD.test_diag_streaming_continues_from_state,
 ]
 
 MUTATIONS = {
@@ -80,6 +86,14 @@ MUTATIONS = {
     "cbwd_no_dsilu": ("double dpre = dxc[c * L + t] * s6o_dsilu(pre);", "double dpre = dxc[c * L + t];"),
     "cbwd_dx_taps_reversed": ("dxo[src] += w[k] * dpre;", "dxo[src] += w[K - 1 - k] * dpre;"),
     "cbwd_dw_wrong_input": ("dw[c * K + k] += dpre * xc[src];", "dw[c * K + k] += dpre * xc[t];"),
+    # the constant-decay cell
+    "diag_decay_sign": ("a[n] = exp2(log2_decay[n]);", "a[n] = exp2(-log2_decay[n]);"),
+    "diag_decay_natural_base": ("a[n] = exp2(log2_decay[n]);", "a[n] = exp(log2_decay[n]);"),
+    "diag_write_without_u": ("Bm[t * N + n] * u[t]);", "Bm[t * N + n]);"),
+    "diag_readout_old_state": ("            h[n] = s6o_update(h[n], a[n], Bm[t * N + n] * u[t]);\n            acc += h[n] * Cm[t * N + n];",
+                               "            acc += h[n] * Cm[t * N + n];\n            h[n] = s6o_update(h[n], a[n], Bm[t * N + n] * u[t]);"),
+    "diag_no_skip": ("double out = acc + D * u[t];", "double out = acc;"),
+    "diag_B_is_C": ("h[n] = s6o_update(h[n], a[n], Bm[t * N + n] * u[t]);", "h[n] = s6o_update(h[n], a[n], Cm[t * N + n] * u[t]);"),
 }
 
 
