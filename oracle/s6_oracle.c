@@ -441,3 +441,125 @@ void s6o_diag_const_channels(int64_t n_ch, int64_t L, int N, const double *u, co
                                Cm + bc_row[c] * L * N, log2_decay + c * N, D[c],
                                h_in ? h_in + c * N : NULL, y + c * L, h_out ? h_out + c * N : NULL);
 }
+
+/* ------------------------------------------------------ the decode block
+ * One Mamba-mini block for one token of one sequence, in the streaming form of
+ * "mamba, live", section "what is actually running" (the per-block listing),
+ * with the weights stored as that page's "Weights" paragraph says: per-row
+ * symmetric int8, w = int8_row x scale_row, A_log kept in float32.
+ *
+ *   hn      = LayerNorm(x)                          (biased variance, eps, affine)
+ *   [xin,z] = in_proj(hn)                           dm -> 2 di  (rows 0..di-1: xin)
+ *   xc      = SiLU(conv_K(xin))                     with the (K-1)-token history
+ *   [dt,B,C]= x_proj(xc)                            di -> R + N + N
+ *   Delta   = softplus(dt_proj(dt) + dt_bias)       R -> di
+ *   h       = exp(Delta A) h + (Delta B) xc,  A = -exp(A_log)
+ *   y       = <h, C> + D xc
+ *   x      += out_proj(y SiLU(z))                   di -> dm
+ *
+ * Readings: in_proj, x_proj and out_proj carry no bias (the TinyMamba
+ * manifest's Linears say bias false); dt_proj's bias is dt_bias; LayerNorm is
+ * PyTorch's (weight and bias, biased variance).
+ */
+
+/* LayerNorm of one row: (x - mean) / sqrt(var + eps) * w + b. */
+void s6o_layernorm(int n, const double *x, const double *w, const double *b, double eps, double *out)
+{
+    double mean = 0.0;
+    for (int i = 0; i < n; ++i)
+        mean += x[i];
+    mean /= n;
+    double var = 0.0;
+    for (int i = 0; i < n; ++i)
+        var += (x[i] - mean) * (x[i] - mean);
+    var /= n;
+    double r = 1.0 / sqrt(var + eps);
+    for (int i = 0; i < n; ++i)
+        out[i] = (x[i] - mean) * r * w[i] + b[i];
+}
+
+/* y[o] = scale[o] * sum_i q[o][i] x[i]: a Linear with per-row int8 weights. */
+void s6o_linear_q8(int n_out, int n_in, const int8_t *q, const double *scale, const double *x, double *y)
+{
+    for (int o = 0; o < n_out; ++o) {
+        double acc = 0.0;
+        for (int i = 0; i < n_in; ++i)
+            acc += (double)q[(int64_t)o * n_in + i] * x[i];
+        y[o] = scale[o] * acc;
+    }
+}
+
+/* The block's weights (all row-major, [out][in]). */
+typedef struct {
+    int dm, di, N, R, K;
+    double eps;
+    const double *ln_w, *ln_b;             /* [dm] */
+    const int8_t *in_q;                    /* [2 di][dm] */
+    const double *in_s;                    /* [2 di] */
+    const double *conv_w, *conv_b;         /* [di][K], [di] */
+    const int8_t *xp_q;                    /* [R + 2N][di] */
+    const double *xp_s;                    /* [R + 2N] */
+    const int8_t *dt_q;                    /* [di][R] */
+    const double *dt_s, *dt_bias;          /* [di], [di] */
+    const double *A_log, *D;               /* [di][N], [di] */
+    const int8_t *out_q;                   /* [dm][di] */
+    const double *out_s;                   /* [dm] */
+} s6o_block;
+
+/* One token through one block.  x [dm] is updated in place (the residual
+ * stream); conv_state [di][K-1] (oldest first) and h [di][N] too.  work holds
+ * 6 di + dm + R + 2N doubles. */
+void s6o_block_step(const s6o_block *p, double *x, double *conv_state, double *h, double *work)
+{
+    int dm = p->dm, di = p->di, N = p->N, R = p->R, K = p->K;
+    double *hn = work;                 /* dm */
+    double *xz = hn + dm;              /* 2 di */
+    double *xc = xz + 2 * di;          /* di */
+    double *dbc = xc + di;             /* R + 2N */
+    double *dtr = dbc + R + 2 * N;     /* di */
+    double *g = dtr + di;              /* di */
+    s6o_layernorm(dm, x, p->ln_w, p->ln_b, p->eps, hn);
+    s6o_linear_q8(2 * di, dm, p->in_q, p->in_s, hn, xz);
+    for (int c = 0; c < di; ++c) {
+        double *hist = conv_state + (int64_t)c * (K - 1);
+        double pre = s6o_conv_pre(K, p->conv_w + (int64_t)c * K, p->conv_b ? p->conv_b[c] : 0.0, hist, xz[c]);
+        for (int k = 0; k + 1 < K - 1; ++k)
+            hist[k] = hist[k + 1];
+        if (K > 1)
+            hist[K - 2] = xz[c];
+        xc[c] = s6o_silu(pre);
+    }
+    s6o_linear_q8(R + 2 * N, di, p->xp_q, p->xp_s, xc, dbc);
+    s6o_linear_q8(di, R, p->dt_q, p->dt_s, dbc, dtr);
+    const double *Bt = dbc + R, *Ct = dbc + R + N;
+    for (int c = 0; c < di; ++c) {
+        double delta = s6o_softplus(dtr[c] + p->dt_bias[c]);
+        double acc = 0.0;
+        for (int n = 0; n < N; ++n) {
+            double a_bar = s6o_decay(delta, p->A_log[(int64_t)c * N + n]);
+            double *hc = h + (int64_t)c * N + n;
+            *hc = s6o_update(*hc, a_bar, delta * Bt[n] * xc[c]);
+            acc += *hc * Ct[n];
+        }
+        double yv = acc + p->D[c] * xc[c];
+        g[c] = yv * s6o_silu(xz[di + c]);
+    }
+    double *o = hn; /* reuse: dm outputs */
+    s6o_linear_q8(dm, di, p->out_q, p->out_s, g, o);
+    for (int i = 0; i < dm; ++i)
+        x[i] += o[i];
+}
+
+/* The block for n_seq independent sequences (x, conv_state, h per sequence). */
+void s6o_block_step_seqs(int64_t n_seq, int dm, int di, int N, int R, int K, double eps,
+                         const double *ln_w, const double *ln_b, const int8_t *in_q, const double *in_s,
+                         const double *conv_w, const double *conv_b, const int8_t *xp_q, const double *xp_s,
+                         const int8_t *dt_q, const double *dt_s, const double *dt_bias, const double *A_log,
+                         const double *D, const int8_t *out_q, const double *out_s,
+                         double *x, double *conv_state, double *h, double *work)
+{
+    s6o_block p = {dm, di, N, R, K, eps, ln_w, ln_b, in_q, in_s, conv_w, conv_b, xp_q, xp_s,
+                   dt_q, dt_s, dt_bias, A_log, D, out_q, out_s};
+    for (int64_t s = 0; s < n_seq; ++s)
+        s6o_block_step(&p, x + s * dm, conv_state + s * (int64_t)di * (K - 1), h + s * (int64_t)di * N, work);
+}

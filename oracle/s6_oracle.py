@@ -21,6 +21,10 @@ What the oracle computes (page titles and sections):
 * ``diag_const`` -- "the s6 cell", *one cell, two architectures*: the same
   diagonal recurrence with a constant decay 2^w per (channel, state) instead of
   a per-token one, written B_t * u_t.
+* ``block_step`` -- one token through one Mamba-mini block ("mamba, live",
+  the per-block listing and *Weights*): LayerNorm, int8 per-row in_proj,
+  conv + SiLU, x_proj, dt_proj + softplus, the recurrence, readout, gate,
+  out_proj and the residual add.
 * ``scan_bwd`` -- the gradients of that scan (no conv), by reverse-mode
   differentiation of the same steps; pinned by central differences of the
   forward oracle.
@@ -81,6 +85,16 @@ def bind(path: str):
     lib.s6o_conv_silu_bwd_channels.restype = None
     lib.s6o_diag_const_channels.argtypes = [i64, i64, i] + [_c_double_p] * 4 + [_c_i64_p] + [_c_double_p] * 5
     lib.s6o_diag_const_channels.restype = None
+    _c_i8_p = ctypes.POINTER(ctypes.c_int8)
+    lib.s6o_layernorm.argtypes = [i, _c_double_p, _c_double_p, _c_double_p, d, _c_double_p]
+    lib.s6o_layernorm.restype = None
+    lib.s6o_linear_q8.argtypes = [i, i, _c_i8_p, _c_double_p, _c_double_p, _c_double_p]
+    lib.s6o_linear_q8.restype = None
+    lib.s6o_block_step_seqs.argtypes = ([i64, i, i, i, i, i, d, _c_double_p, _c_double_p, _c_i8_p, _c_double_p,
+                                         _c_double_p, _c_double_p, _c_i8_p, _c_double_p, _c_i8_p, _c_double_p,
+                                         _c_double_p, _c_double_p, _c_double_p, _c_i8_p, _c_double_p] +
+                                        [_c_double_p] * 4)
+    lib.s6o_block_step_seqs.restype = None
     for name in ("s6o_ssm_state_values", "s6o_conv_history_values"):
         f = getattr(lib, name)
         f.argtypes, f.restype = [i64, i64, i64], i64
@@ -317,6 +331,70 @@ def diag_const(u, log2_decay, B, C, D, z=None, channels=None, h_init=None, threa
         y_full[cb, :, cd] = y
         return y_full, hout.reshape(Bt, d, N)
     return y, hout
+
+
+def layernorm(x, w, b, eps=1e-5):
+    """LayerNorm of each row of x (the last axis), biased variance, affine."""
+    x = np.ascontiguousarray(_f64(x))
+    rows = x.reshape(-1, x.shape[-1])
+    out = np.zeros_like(rows)
+    wv, bv = np.ascontiguousarray(_f64(w)), np.ascontiguousarray(_f64(b))
+    for r in range(rows.shape[0]):
+        _load().s6o_layernorm(rows.shape[1], _ptr(rows[r]), _ptr(wv), _ptr(bv), float(eps), _ptr(out[r]))
+    return out.reshape(x.shape)
+
+
+def linear_q8(q, scale, x):
+    """y = scale[o] * sum_i q[o, i] x[i] for each row of x: a Linear with per-row int8 weights."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    sc = np.ascontiguousarray(_f64(scale))
+    x = np.ascontiguousarray(_f64(x))
+    rows = x.reshape(-1, x.shape[-1])
+    out = np.zeros((rows.shape[0], q.shape[0]))
+    for r in range(rows.shape[0]):
+        _load().s6o_linear_q8(q.shape[0], q.shape[1], q.ctypes.data_as(ctypes.POINTER(ctypes.c_int8)), _ptr(sc),
+                              _ptr(rows[r]), _ptr(out[r]))
+    return out.reshape(x.shape[:-1] + (q.shape[0],))
+
+
+_BLOCK_KEYS = ("ln_w", "ln_b", "in_q", "in_s", "conv_w", "conv_b", "xp_q", "xp_s", "dt_q", "dt_s", "dt_bias",
+               "A_log", "D", "out_q", "out_s")
+
+
+def block_step(x, conv_state, h, w, eps=1e-5, threads=None):
+    """One token through one decode block ("mamba, live", the per-block listing)
+    for each sequence: x [Bt, dm], conv_state [Bt, di, K-1], h [Bt, di, N];
+    ``w`` the block's weights (s6_inputs.block_weights).  Returns new
+    (x, conv_state, h) as float64 arrays; the inputs are not modified."""
+    x = np.array(_f64(x), copy=True)
+    cs = np.array(_f64(conv_state), copy=True)
+    hh = np.array(_f64(h), copy=True)
+    Bt, dm = x.shape
+    di, N = np.asarray(w["A_log"]).shape
+    K = np.asarray(w["conv_w"]).shape[1]
+    R = np.asarray(w["dt_q"]).shape[1]
+    arrs = {}
+    for k in _BLOCK_KEYS:
+        v = np.asarray(w[k])
+        arrs[k] = np.ascontiguousarray(v, dtype=np.int8) if v.dtype == np.int8 else np.ascontiguousarray(_f64(v))
+    i8 = ctypes.POINTER(ctypes.c_int8)
+
+    def p(k):
+        a = arrs[k]
+        return a.ctypes.data_as(i8) if a.dtype == np.int8 else _ptr(a)
+
+    nt = _threads(Bt, threads)
+    bounds = np.linspace(0, Bt, nt + 1).astype(np.int64)
+
+    def run(i):
+        lo, hi = int(bounds[i]), int(bounds[i + 1])
+        work = np.zeros(6 * di + dm + R + 2 * N)
+        _load().s6o_block_step_seqs(hi - lo, dm, di, N, R, K, float(eps), *[p(k) for k in _BLOCK_KEYS],
+                                    _ptr(x[lo:hi]), _ptr(cs[lo:hi]), _ptr(hh[lo:hi]), _ptr(work))
+
+    with ThreadPoolExecutor(nt) as ex:
+        list(ex.map(run, range(nt)))
+    return x, cs, hh
 
 
 def scan_bwd(u, dt_raw, A_log, B, C, D, dy, z=None, dt_bias=None, zoh=False, h_init=None, threads=None):

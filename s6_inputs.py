@@ -20,6 +20,10 @@ the Mamba-mini block of "mamba, live" / "two recurrences"):
   decode     256 sequences x 6 blocks x d1536 x N16, K4, fp32 state, seed 3
   long_seq   Bt16 L8192 d1536 N16 K4, bf16 I/O, seed 4
   wide       Bt4 L2048 d5120 N16 K4, bf16 I/O, exact ZOH, seed 5
+
+The constant-decay cell ("the s6 cell", one cell, two architectures) reads the
+same u, z, B, C draws plus a per-(channel, state) constant decay drawn by
+``diag_log2_decay``.
 """
 from __future__ import annotations
 
@@ -141,3 +145,45 @@ def decode_tokens(step: int, block: int, *, Bt=256, d=1536, N=16, seed=3, io="f3
     dt = _normal(rng, (Bt, d), 0.5)
     return dict(x=to_storage(x, io), z=to_storage(z, io), B=to_storage(Bm, io), C=to_storage(Cm, io),
                 dt=to_storage(dt, io))
+
+
+def diag_log2_decay(d: int, N: int, seed: int = 6) -> np.ndarray:
+    """log2 of constant decays a[d, n] ~ U[0.2, 0.999] (float32 [d, N], <= 0)."""
+    rng = np.random.default_rng([seed, d, N])
+    return np.log2(rng.uniform(0.2, 0.999, size=(d, N))).astype(np.float32)
+
+
+# ------------------------------------------------------------ the decode block
+# Mamba-mini ("mamba, live", what is actually running): d_model 384, d_inner
+# 1536, N 16, dt rank 24, conv width 4, 6 blocks.  Weights are synthetic (no
+# trained ones exist here), stored as that page's Weights paragraph says:
+# per-row symmetric int8 with one float32 scale per output row; the scales
+# give unit-variance inputs unit-variance outputs.
+MAMBA_MINI_BLOCK = dict(dm=384, di=1536, N=16, R=24, K=4, blocks=6, eps=1e-5)
+
+
+def _q8_rows(rng, n_out, n_in, gain=1.0):
+    q = rng.integers(-127, 128, size=(n_out, n_in)).astype(np.int8)
+    # std of U{-127..127} is about 73.6; scale so that Var(w) = gain^2 / n_in
+    scale = (gain / (73.6 * np.sqrt(n_in)) * rng.uniform(0.8, 1.25, size=n_out)).astype(np.float32)
+    return q, scale
+
+
+def block_weights(block: int, *, dm=384, di=1536, N=16, R=24, K=4, seed=7):
+    """Synthetic weights of one decode block (int8 rows x float32 scales)."""
+    rng = np.random.default_rng([seed, block])
+    in_q, in_s = _q8_rows(rng, 2 * di, dm)
+    xp_q, xp_s = _q8_rows(rng, R + 2 * N, di)
+    dt_q, dt_s = _q8_rows(rng, di, R, gain=0.5)
+    out_q, out_s = _q8_rows(rng, dm, di, gain=0.5)
+    p = params(rng, di, N, K, "mamba_mini")
+    return dict(ln_w=(1.0 + 0.1 * rng.standard_normal(dm)).astype(np.float32),
+                ln_b=(0.1 * rng.standard_normal(dm)).astype(np.float32),
+                in_q=in_q, in_s=in_s, conv_w=p["conv_w"], conv_b=p["conv_b"], xp_q=xp_q, xp_s=xp_s,
+                dt_q=dt_q, dt_s=dt_s, dt_bias=p["dt_bias"], A_log=p["A_log"], D=p["D"], out_q=out_q, out_s=out_s)
+
+
+def block_tokens(step: int, *, Bt=256, dm=384, seed=8):
+    """Residual-stream input of one decode step: x [Bt, dm] ~ N(0, 1) (float32)."""
+    rng = np.random.default_rng([seed, step])
+    return rng.standard_normal((Bt, dm)).astype(np.float32)

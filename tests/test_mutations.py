@@ -10,6 +10,7 @@ import subprocess
 import pytest
 
 from oracle import s6_oracle as O
+import test_oracle_block as TK
 import test_oracle_bwd as TB
 import test_oracle_diag as TD
 import test_oracle_pins as P
@@ -48,6 +49,10 @@ ALL_PINS = [
     TD.test_diag_equals_selective_scan_at_unit_step,
     TD.test_diag_decays_in_unit_interval_and_state_bounded,
     TD.test_diag_streaming_continues_from_state,
+    TK.test_block_worked_example,
+    TK.test_block_streaming_equals_sequence_form,
+    TK.test_linear_q8_against_numpy,
+    TK.test_layernorm_against_numpy,
 ]
 
 MUTATIONS = {
@@ -94,6 +99,15 @@ MUTATIONS = {
                                "            acc += h[n] * Cm[t * N + n];\n            h[n] = s6o_update(h[n], a[n], Bm[t * N + n] * u[t]);"),
     "diag_no_skip": ("double out = acc + D * u[t];", "double out = acc;"),
     "diag_B_is_C": ("h[n] = s6o_update(h[n], a[n], Bm[t * N + n] * u[t]);", "h[n] = s6o_update(h[n], a[n], Cm[t * N + n] * u[t]);"),
+    # the decode block
+    "block_no_residual": ("        x[i] += o[i];", "        x[i] = o[i];"),
+    "block_ln_unbiased_variance": ("    var /= n;", "    var /= (n - 1);"),
+    "block_ln_no_affine_bias": ("out[i] = (x[i] - mean) * r * w[i] + b[i];", "out[i] = (x[i] - mean) * r * w[i];"),
+    "block_linear_scale_per_column": ("y[o] = scale[o] * acc;", "y[o] = scale[o % n_in] * acc;"),
+    "block_xproj_B_C_swapped": ("const double *Bt = dbc + R, *Ct = dbc + R + N;", "const double *Bt = dbc + R + N, *Ct = dbc + R;"),
+    "block_dt_bias_missing": ("double delta = s6o_softplus(dtr[c] + p->dt_bias[c]);", "double delta = s6o_softplus(dtr[c]);"),
+    "block_gate_from_xin": ("g[c] = yv * s6o_silu(xz[di + c]);", "g[c] = yv * s6o_silu(xz[c]);"),
+    "block_conv_history_not_updated": ("            hist[K - 2] = xz[c];", "            hist[K - 2] = hist[K - 2];"),
 }
 
 
