@@ -204,6 +204,41 @@ S6_API int s6_conv_scan_fwd_from_state(const s6_dims *dims, const void *x, const
                                        s6_stream_t stream);
 
 /*
+ * s6_diag_recurrence_fwd -- the diagonal recurrence cell with the decay source
+ * as a parameter ("the s6 cell", sections "one cell, two architectures" and
+ * "the difference that no engineering removes"): both recurrences reduce to
+ * h <- a*h + b*u with a = 2^(negative); the decay is either computed per token
+ * from the input (live, the selective scan) or a per-channel constant that is
+ * precomputed once (no exponential per token).  State width N = d_state.
+ *
+ *  decay_source  S6_DECAY_LIVE:  a = 2^(Delta*A*log2 e), Delta = softplus(dt +
+ *                                dt_bias), A = -exp(A_log), b = Delta*B_t --
+ *                                exactly s6_scan_fwd_from_state with
+ *                                zoh_mode = 0 (dt, A_log required; log2_decay
+ *                                ignored)
+ *                S6_DECAY_CONST: a[d,n] = 2^log2_decay[d,n] (log2_decay <= 0
+ *                                for a decay in (0, 1]), b = B_t: per state n,
+ *                                h[n] <- a[n] h[n] + B_t[n] u_t
+ *                                (dt, A_log and dt_bias ignored, may be NULL)
+ *  u        [Bt,L,d] io   input
+ *  log2_decay [d,N]  f32  log2 of the constant decays (S6_DECAY_CONST)
+ *  B, C     [Bt,L,N] io   per-token write and readout vectors
+ *  D        [d]      f32  y = (<h, C_t> + D*u) * SiLU(z)
+ *  z        [Bt,L,d] io   NULL = no gate
+ *  h_init   [Bt,d,N] f32  start state, NULL = zeros
+ *  y, h_final              as s6_scan_fwd
+ * RWKV's normaliser branch (the page's other difference) is not part of this
+ * cell: the pages give it no formula.  Alignment and scratch as s6_scan_fwd;
+ * an unknown decay_source returns S6_ERR_INVALID_ARG.
+ */
+#define S6_DECAY_LIVE 0
+#define S6_DECAY_CONST 1
+S6_API int s6_diag_recurrence_fwd(const s6_dims *dims, int decay_source, const void *u, const void *dt,
+                                  const float *A_log, const float *dt_bias, const float *log2_decay,
+                                  const void *B, const void *C, const float *D, const void *z,
+                                  const float *h_init, void *y, float *h_final, s6_stream_t stream);
+
+/*
  * s6_scan_bwd -- gradients of s6_scan_fwd (no conv: u given) for the loss
  * sum(dy * y): reverse-mode differentiation of the same steps (the recurrence
  * the pages single out as what makes training slow, "Carry context through a
@@ -285,12 +320,89 @@ S6_API int s6_step(const s6_dims *dims, const float *A_log, const float *D, cons
             void *conv_state, void *y_t, s6_stream_t stream);
 
 /*
+ * s6_block_step -- one token through one Mamba-mini decode block for Bt
+ * independent sequences ("mamba, live", section "what is actually running":
+ * the per-block listing; its "Weights" paragraph: per-row symmetric int8,
+ * w = int8_row x scale_row, A_log kept in float32):
+ *
+ *     hn = LayerNorm(x);  [xin, z] = in_proj(hn);  xc = SiLU(conv_K(xin))
+ *     [dt, B, C] = x_proj(xc);  Delta = softplus(dt_proj(dt) + dt_bias)
+ *     h = exp(Delta A) h + (Delta B) xc,  A = -exp(A_log);  y = <h, C> + D xc
+ *     x += out_proj(y * SiLU(z))
+ *
+ * Readings: in_proj, x_proj and out_proj have no bias; dt_proj's bias is
+ * dt_bias; LayerNorm uses the biased variance, eps = dims.eps, weight and bias.
+ *
+ *  dims      batch Bt >= 0, d_model dm >= 1, d_inner di >= 1, d_state N in
+ *            [1, 16], dt_rank R >= 1, conv_width K in [2, 4], eps
+ *  w         the block's weights (device pointers, row-major [out][in]):
+ *              ln_w, ln_b [dm] f32; in_q [2 di][dm] int8, in_s [2 di] f32
+ *              (rows 0..di-1 give xin, di..2di-1 give z); conv_w [di][K] f32,
+ *              conv_b [di] f32 (NULL = zeros); xp_q [R + 2N][di] int8, xp_s
+ *              [R + 2N] f32 (rows: dt, then B, then C); dt_q [di][R] int8, dt_s
+ *              [di] f32, dt_bias [di] f32; A_log [di][N] f32, D [di] f32;
+ *              out_q [dm][di] int8, out_s [dm] f32.  w_row = q_row * s_row.
+ *  x          [Bt][dm]      f32  the residual stream: read, and out_proj's
+ *                                output added in place
+ *  conv_state [Bt][di][K-1] f32  the K-1 previous xin, oldest first (in place)
+ *  h_ssm      [Bt][di][N]   f32  the state (in place)
+ * All float pointers need 4-byte alignment (A_log and h_ssm 16-byte when
+ * N = 16).  Uses a library-owned scratch buffer for the intermediate rows
+ * (xin|z, the x_proj rows, the gated readout): allocated on the first call on
+ * a device, grown on demand; make that call before capturing a stream.
+ * out_proj and x_proj add their partial sums with float atomics, so the last
+ * bits of x can vary between runs.
+ */
+typedef struct {
+    int64_t batch;      /* Bt >= 0 */
+    int64_t d_model;    /* dm */
+    int64_t d_inner;    /* di */
+    int64_t d_state;    /* N in [1, 16] */
+    int64_t dt_rank;    /* R */
+    int64_t conv_width; /* K in [2, 4] */
+    float eps;          /* LayerNorm epsilon */
+} s6_block_dims;
+
+typedef struct {
+    const float *ln_w, *ln_b;
+    const int8_t *in_q;
+    const float *in_s;
+    const float *conv_w, *conv_b;
+    const int8_t *xp_q;
+    const float *xp_s;
+    const int8_t *dt_q;
+    const float *dt_s, *dt_bias;
+    const float *A_log, *D;
+    const int8_t *out_q;
+    const float *out_s;
+} s6_block_weights;
+
+S6_API int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x, float *conv_state,
+                         float *h_ssm, s6_stream_t stream);
+
+/*
  * s6_device_status -- synchronises `stream`, then reads and clears the
  * library's device-side error word.  Returns S6_ERR_TIMEOUT if a kernel gave
  * up a bounded wait (its outputs are then incomplete), S6_ERR_CUDA if the
  * stream or the copy failed, else S6_OK.
  */
 S6_API int s6_device_status(s6_stream_t stream);
+
+/*
+ * s6_debug_carry_fault -- fault injection for tests of the failure path; the
+ * pages have no counterpart.  Off by default; a process that never calls it is
+ * unaffected.
+ *
+ * After the call, every scan that splits its sequences into segments gives up
+ * a wait for a predecessor's carry after `carry_polls` polls (0 restores the
+ * default, about 4M polls spaced by 64 ns sleeps), and the unit with index
+ * `skip_publish_unit` (-1: none) publishes no carry, so its successor's wait
+ * runs out: that kernel sets the device error word, continues from an
+ * undefined start state and exits normally, and s6_device_status then returns
+ * S6_ERR_TIMEOUT.  Nothing faults, traps or hangs.  Process-wide host state,
+ * read when a scan is enqueued; not for concurrent use with other scans.
+ */
+S6_API int s6_debug_carry_fault(int skip_publish_unit, unsigned int carry_polls);
 
 /* Human-readable name of an s6_status value (static string; never NULL). */
 S6_API const char *s6_status_string(int status);

@@ -8,8 +8,9 @@ There is no CPU fallback: if the library is missing, the first call raises.
 
 Functions (same names as the C ABI):
     s6_scan_fwd, s6_conv_scan_fwd, s6_conv_scan_fwd_noalloc, s6_scan_fwd_from_state,
-    s6_conv_scan_fwd_from_state, s6_scan_bwd, s6_conv_scan_bwd, causal_conv1d_silu_fwd, s6_step,
-    s6_device_status, s6_status_string, s6_version
+    s6_conv_scan_fwd_from_state, s6_diag_recurrence_fwd, s6_scan_bwd, s6_conv_scan_bwd,
+    causal_conv1d_silu_fwd, s6_step, s6_block_step, s6_device_status, s6_status_string, s6_version,
+    s6_debug_carry_fault (tests only)
 """
 from __future__ import annotations
 
@@ -18,8 +19,9 @@ import os
 
 __all__ = [
     "S6Error", "lib", "s6_scan_fwd", "s6_conv_scan_fwd", "s6_conv_scan_fwd_noalloc", "s6_scan_fwd_from_state",
-    "s6_conv_scan_fwd_from_state", "s6_scan_bwd", "s6_conv_scan_bwd", "causal_conv1d_silu_fwd", "s6_step",
-    "s6_device_status", "s6_status_string", "s6_version", "S6_F32", "S6_BF16", "Dims",
+    "s6_conv_scan_fwd_from_state", "s6_diag_recurrence_fwd", "S6_DECAY_LIVE", "S6_DECAY_CONST", "s6_scan_bwd", "s6_conv_scan_bwd", "causal_conv1d_silu_fwd", "s6_step",
+    "s6_block_step", "BlockDims", "BlockWeights", "BLOCK_WEIGHT_KEYS",
+    "s6_device_status", "s6_status_string", "s6_version", "s6_debug_carry_fault", "S6_F32", "S6_BF16", "Dims",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -28,12 +30,29 @@ LIB_PATH = os.path.join(_HERE, "libs6_b200.so")
 S6_F32, S6_BF16 = 0, 1
 S6_OK, S6_ERR_INVALID_ARG, S6_ERR_UNSUPPORTED, S6_ERR_ALIGNMENT, S6_ERR_CUDA, S6_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 S6_ERR_SCRATCH_LIMIT = -6
+S6_DECAY_LIVE, S6_DECAY_CONST = 0, 1
 
 
 class Dims(ctypes.Structure):
     """Mirror of ``s6_dims``."""
     _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("d_inner", ctypes.c_int64),
                 ("d_state", ctypes.c_int64), ("conv_width", ctypes.c_int64), ("io_dtype", ctypes.c_int32)]
+
+
+class BlockDims(ctypes.Structure):
+    """Mirror of ``s6_block_dims``."""
+    _fields_ = [("batch", ctypes.c_int64), ("d_model", ctypes.c_int64), ("d_inner", ctypes.c_int64),
+                ("d_state", ctypes.c_int64), ("dt_rank", ctypes.c_int64), ("conv_width", ctypes.c_int64),
+                ("eps", ctypes.c_float)]
+
+
+BLOCK_WEIGHT_KEYS = ("ln_w", "ln_b", "in_q", "in_s", "conv_w", "conv_b", "xp_q", "xp_s", "dt_q", "dt_s", "dt_bias",
+                     "A_log", "D", "out_q", "out_s")
+
+
+class BlockWeights(ctypes.Structure):
+    """Mirror of ``s6_block_weights`` (device pointers)."""
+    _fields_ = [(k, ctypes.c_void_p) for k in BLOCK_WEIGHT_KEYS]
 
 
 class S6Error(RuntimeError):
@@ -62,6 +81,7 @@ def lib() -> ctypes.CDLL:
         L.s6_conv_scan_fwd_noalloc.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P]
         L.s6_scan_fwd_from_state.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P]
         L.s6_conv_scan_fwd_from_state.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]
+        L.s6_diag_recurrence_fwd.argtypes = [DP, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.s6_scan_bwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P] + [_P] * 9 + [_P]
         L.s6_conv_scan_bwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P] + [_P] * 11 + [_P]
         L.causal_conv1d_silu_fwd.argtypes = [DP, _P, _P, _P, _P, _P]
@@ -70,8 +90,12 @@ def lib() -> ctypes.CDLL:
         L.s6_status_string.argtypes = [_I]
         L.s6_status_string.restype = ctypes.c_char_p
         L.s6_version.argtypes = []
+        L.s6_debug_carry_fault.argtypes = [_I, ctypes.c_uint]
+        L.s6_block_step.argtypes = [ctypes.POINTER(BlockDims), ctypes.POINTER(BlockWeights), _P, _P, _P, _P]
+        L.s6_block_step.restype = _I
+        L.s6_debug_carry_fault.restype = _I
         for f in (L.s6_scan_fwd, L.s6_conv_scan_fwd, L.s6_conv_scan_fwd_noalloc, L.s6_scan_fwd_from_state,
-                  L.s6_conv_scan_fwd_from_state, L.s6_scan_bwd, L.s6_conv_scan_bwd, L.causal_conv1d_silu_fwd, L.s6_step,
+                  L.s6_conv_scan_fwd_from_state, L.s6_diag_recurrence_fwd, L.s6_scan_bwd, L.s6_conv_scan_bwd, L.causal_conv1d_silu_fwd, L.s6_step,
                   L.s6_device_status, L.s6_version):
             f.restype = _I
         _lib = L
@@ -206,6 +230,40 @@ def s6_conv_scan_fwd_from_state(x, conv_w, conv_b, dt, A_log, B, C, D, z=None, d
                  conv_b, want_h_final, stream, from_state=True, h_init=h_init, conv_hist=conv_hist)
 
 
+def s6_diag_recurrence_fwd(u, B, C, D, decay_source=S6_DECAY_CONST, log2_decay=None, dt=None, A_log=None,
+                           dt_bias=None, z=None, h_init=None, y=None, h_final=None, want_h_final=True, stream=None):
+    """The diagonal recurrence with the decay source as a parameter: constant
+    (h <- 2^log2_decay * h + B_t u_t; log2_decay [d, N]) or live (the selective
+    scan, dt and A_log given).  Returns (y, h_final)."""
+    torch = _torch()
+    if u.dim() != 3:
+        raise ValueError("u must be [batch, seqlen, d_inner]")
+    Bt, L, d = u.shape
+    par = A_log if decay_source == S6_DECAY_LIVE else log2_decay
+    if par is None:
+        par = A_log if A_log is not None else log2_decay
+    if par is None:
+        raise ValueError("log2_decay (constant decay) or A_log (live decay) is required")
+    N = par.shape[-1]
+    dev = u.device
+    f32 = torch.float32
+    if y is None:
+        y = torch.empty_like(u)
+    if h_final is None and want_h_final:
+        h_final = torch.empty((Bt, d, N), dtype=f32, device=dev)
+    dims = Dims(Bt, L, d, N, 0, _io_code(u))
+    seq = (Bt, L, d)
+    st = lib().s6_diag_recurrence_fwd(
+        ctypes.byref(dims), int(decay_source), _ptr(u, "u", u.dtype, seq, dev), _ptr(dt, "dt", u.dtype, seq, dev),
+        _ptr(A_log, "A_log", f32, (d, N), dev), _ptr(dt_bias, "dt_bias", f32, (d,), dev),
+        _ptr(log2_decay, "log2_decay", f32, (d, N), dev), _ptr(B, "B", u.dtype, (Bt, L, N), dev),
+        _ptr(C, "C", u.dtype, (Bt, L, N), dev), _ptr(D, "D", f32, (d,), dev), _ptr(z, "z", u.dtype, seq, dev),
+        _ptr(h_init, "h_init", f32, (Bt, d, N), dev), _ptr(y, "y", u.dtype, seq, dev),
+        _ptr(h_final, "h_final", f32, (Bt, d, N), dev), _stream(stream, dev))
+    _check(st, "s6_diag_recurrence_fwd")
+    return y, h_final
+
+
 def s6_scan_bwd(u, dt, A_log, B, C, D, dy, z=None, dt_bias=None, zoh_mode=0, h_init=None, want_dh_init=False,
                 stream=None):
     """Gradients of s6_scan_fwd for the loss sum(dy * y).  Returns a dict of float32
@@ -319,8 +377,44 @@ def s6_step(u_t, dt_t, B_t, C_t, A_log, D, conv_w, h_ssm, conv_state, z_t=None, 
     return y_t
 
 
+def s6_block_step(x, conv_state, h_ssm, w, eps=1e-5, stream=None):
+    """One token through one decode block for every sequence of the batch:
+    x [Bt, dm] (the residual stream, updated in place), conv_state [Bt, di, K-1]
+    and h_ssm [Bt, di, N] (float32, in place); ``w`` a dict of the block's device
+    weights (BLOCK_WEIGHT_KEYS: int8 rows *_q with float32 row scales *_s).  The
+    weight structure is kept on the dict (key "_abi") for later calls."""
+    torch = _torch()
+    Bt, dm = x.shape
+    di, N = w["A_log"].shape
+    K = w["conv_w"].shape[1]
+    R = w["dt_q"].shape[1]
+    dev = x.device
+    f32, i8 = torch.float32, torch.int8
+    shapes = {"ln_w": ((dm,), f32), "ln_b": ((dm,), f32), "in_q": ((2 * di, dm), i8), "in_s": ((2 * di,), f32),
+              "conv_w": ((di, K), f32), "conv_b": ((di,), f32), "xp_q": ((R + 2 * N, di), i8),
+              "xp_s": ((R + 2 * N,), f32), "dt_q": ((di, R), i8), "dt_s": ((di,), f32), "dt_bias": ((di,), f32),
+              "A_log": ((di, N), f32), "D": ((di,), f32), "out_q": ((dm, di), i8), "out_s": ((dm,), f32)}
+    abi = w.get("_abi")
+    if abi is None:
+        abi = BlockWeights(*[_ptr(w.get(k), k, shapes[k][1], shapes[k][0], dev) for k in BLOCK_WEIGHT_KEYS])
+        w["_abi"] = abi
+    dims = BlockDims(Bt, dm, di, N, R, K, float(eps))
+    st = lib().s6_block_step(ctypes.byref(dims), ctypes.byref(abi), _ptr(x, "x", f32, (Bt, dm), dev),
+                             _ptr(conv_state, "conv_state", f32, (Bt, di, K - 1), dev),
+                             _ptr(h_ssm, "h_ssm", f32, (Bt, di, N), dev), _stream(stream, dev))
+    _check(st, "s6_block_step")
+    return x
+
+
 def s6_device_status(stream=None, device=None) -> int:
     """Synchronise and return (and clear) the library's device-side error status."""
     torch = _torch()
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
     return lib().s6_device_status(_stream(stream, dev))
+
+
+def s6_debug_carry_fault(skip_publish_unit: int = -1, carry_polls: int = 0) -> None:
+    """Test-only fault injection: unit `skip_publish_unit` of the next segmented
+    scans publishes no carry and carry waits give up after `carry_polls` polls
+    (0 = default).  ``s6_debug_carry_fault()`` switches it off again."""
+    _check(lib().s6_debug_carry_fault(int(skip_publish_unit), int(carry_polls)), "s6_debug_carry_fault")

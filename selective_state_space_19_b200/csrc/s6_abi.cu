@@ -7,7 +7,9 @@
 #include <cstddef>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
+#include <utility>
 
 #include "s6.h"
 #include "s6_common.cuh"
@@ -15,6 +17,8 @@
 #include "s6_scan.cuh"
 #include "s6_step.cuh"
 #include "s6_bwd.cuh"
+#include "s6_bwd_rev.cuh"
+#include "s6_block.cuh"
 
 namespace {
 
@@ -84,6 +88,23 @@ int check_dims(const s6_dims *dims, bool need_L, bool need_K) {
 
 int launch_status(cudaError_t e) { return e == cudaSuccess ? S6_OK : S6_ERR_CUDA; }
 
+// Every entry point restores the calling thread's current device before it
+// returns: use_stream_device below may switch it to the stream's device.
+struct DeviceRestore {
+    int prev = -1;
+    DeviceRestore() {
+        if (cudaGetDevice(&prev) != cudaSuccess)
+            prev = -1;
+    }
+    ~DeviceRestore() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev)
+            cudaSetDevice(prev);
+    }
+    DeviceRestore(const DeviceRestore &) = delete;
+    DeviceRestore &operator=(const DeviceRestore &) = delete;
+};
+
 // Make the device that owns `stream` current for this library's runtime before
 // any launch (the caller's framework may have selected it through another
 // runtime instance in the same process).  The legacy and per-thread default
@@ -107,23 +128,25 @@ int use_stream_device(cudaStream_t stream) {
 }
 
 // ------------------------------------------------------------ scan dispatch
-// Library-owned scratch for the dynamic scan: a unit counter, one flag per
-// chain and one published end state per chain.  One buffer per device,
-// allocated on first need and grown on demand (never while a stream is being
-// captured); kept until process exit.
+// Library-owned scratch, one buffer per (device, use), allocated on first need
+// and grown on demand (never while a stream is being captured); kept until
+// process exit.  Uses: the scan's segment carries (a unit counter, flags,
+// published states), and the backward's state checkpoints, its partial dB / dC
+// rows and its reverse carries.
+enum ScratchSlot { kScratchScan = 0, kScratchCkpt, kScratchPart, kScratchRev, kScratchBlock, kScratchSlots };
 struct DeviceScratch {
     void *ptr = nullptr;
     size_t bytes = 0;
 };
 std::mutex g_scratch_mu;
-DeviceScratch g_scratch[64];
+DeviceScratch g_scratch[64][kScratchSlots];
 
-int get_scratch(size_t bytes, cudaStream_t stream, void **out) {
+int get_scratch(size_t bytes, cudaStream_t stream, void **out, int slot = kScratchScan) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return S6_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    DeviceScratch &sc = g_scratch[dev];
+    DeviceScratch &sc = g_scratch[dev][slot];
     if (sc.bytes < bytes) {
         cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
         if (stream && cudaStreamIsCapturing(stream, &cap) != cudaSuccess)
@@ -166,7 +189,19 @@ int device_sm_count() {
 
 size_t round_up(size_t v, size_t m) { return (v + m - 1) / m * m; }
 
-template <typename IO, int NS, int TPC, bool CONV, bool ZOH, bool INIT>
+// Fault injection for tests (s6_debug_carry_fault): off unless a test sets it.
+constexpr unsigned int kCarryPolls = 1u << 22;  // ~0.3 s of polling at 64 ns sleeps
+std::atomic<int> g_dbg_skip_publish{-1};
+std::atomic<unsigned int> g_dbg_carry_polls{kCarryPolls};
+
+// Whether a scan should use the associative split: too few (sequence, channel
+// tile) chains to give a third of the CTA slots one each, and a sequence long
+// enough to cut into segments of at least two chunks.
+bool want_assoc(int64_t chains, int64_t L, int T, int64_t slots) {
+    return chains > 0 && 3 * chains <= slots && L >= 4 * static_cast<int64_t>(T);
+}
+
+template <typename IO, int NS, int TPC, bool CONV, int MODE, int EXT>
 int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, ScanArgs a,
                   cudaStream_t stream, const FixedScratch *fixed = nullptr) {
     // Tokens per chunk: 64 (bf16) / 32 (f32).  A
@@ -189,8 +224,9 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     const int io = dims->io_dtype;
     const size_t es = io_size(io);
     CUtensorMap tx, tdt, tz, ty, tB, tC;
+    // the constant-decay form reads no step size: its dt map (never used) is built on x
     if (!make_map_3d(&tx, x, io, dims->batch, dims->seqlen, dims->d_inner, CPB, Sh::XR) ||
-        !make_map_3d(&tdt, dt, io, dims->batch, dims->seqlen, dims->d_inner, CPB, T) ||
+        !make_map_3d(&tdt, MODE == s6::kModeConst ? x : dt, io, dims->batch, dims->seqlen, dims->d_inner, CPB, T) ||
         !make_map_3d(&ty, y, io, dims->batch, dims->seqlen, dims->d_inner, Sh::CPW, T))  // per-warp stores
         return S6_ERR_CUDA;
     if (z) {
@@ -208,18 +244,25 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     } else {
         tB = tC = tdt;  // never read
     }
-    auto kern = s6::s6_scan_kernel<IO, NS, TPC, T, STAGES, CONV, ZOH, INIT>;
+    constexpr bool INIT = EXT >= 1;
+    auto kern = s6::s6_scan_kernel<IO, NS, TPC, T, STAGES, CONV, MODE, EXT>;
     const size_t smem = sizeof(Smem);
-    static int occ = 0;  // resident CTAs per SM for this instantiation
-    if (!occ) {
+    // resident CTAs per SM for this instantiation, per device (the shared-memory
+    // opt-in is a per-device attribute)
+    static int occ_dev[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return S6_ERR_CUDA;
+    if (!occ_dev[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
             cudaSuccess)
             return S6_ERR_CUDA;
         int nb = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, s6::kScanBlock, smem) != cudaSuccess || nb < 1)
             return S6_ERR_CUDA;
-        occ = nb;
+        occ_dev[dev] = nb;
     }
+    const int occ = occ_dev[dev];
 
     // ---- work split: chains of segments, pulled dynamically when there are
     // too few chains to balance the SMs statically
@@ -229,12 +272,26 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     // Every SM gets the same number of persistent CTAs, and no more CTAs run
     // than there are chains (a CTA beyond that would only wait).
     const int64_t sms = device_sm_count();
+    const bool assoc = INIT && want_assoc(chains, L, T, sms * occ);
     int64_t per_sm = occ;
-    while (per_sm > 1 && per_sm * sms > chains)
+    while (!assoc && per_sm > 1 && per_sm * sms > chains)
         --per_sm;
     const int64_t workers = sms * per_sm;
     int64_t nseg = 1, seg_len = round_up(static_cast<size_t>(L), T);
-    if (chains < 4 * workers && L > 4 * T) {
+    if (assoc) {
+        // Associative split: every chain's segments scan at once (segment 0 in
+        // full, the others state-only from zero), then the later segments run
+        // again from their folded start states.  Enough segments to give every
+        // CTA slot a unit in the first phase, never shorter than 2 chunks.
+        int64_t want = (workers + chains - 1) / chains;
+        const int64_t max_seg = L / (2 * T);
+        if (want > max_seg)
+            want = max_seg;
+        if (want < 2)
+            want = 2;
+        seg_len = round_up(static_cast<size_t>((L + want - 1) / want), T);
+        nseg = (L + seg_len - 1) / seg_len;
+    } else if (chains < 4 * workers && L > 4 * T) {
         // about 16 units per worker: the last, partly filled wave of units is
         // short next to the whole run (a chain's segments run one after the
         // other, so at most `chains` units are ever in flight)
@@ -248,17 +305,25 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
             nseg = (L + seg_len - 1) / seg_len;
         }
     }
-    if (chains * nseg > 0x7fffffffLL)
+    a.assoc = assoc && nseg > 1;
+    const int64_t units = a.assoc ? chains * (2 * nseg - 1) : chains * nseg;
+    if (units > 0x7fffffffLL)
         return S6_ERR_UNSUPPORTED;
     a.nseg = static_cast<int>(nseg);
     a.seg_len = static_cast<int>(seg_len);
-    a.units = static_cast<int>(chains * nseg);
+    a.units = static_cast<int>(units);
     a.dynamic = nseg > 1;
+    a.carry_polls = g_dbg_carry_polls.load();
+    a.skip_publish = g_dbg_skip_publish.load();
     unsigned grid = static_cast<unsigned>(chains);
     if (a.dynamic) {
-        const size_t nflags = static_cast<size_t>(chains) * s6::kConsumerWarps;
+        // serial: one flag per (chain, consumer warp) and one end state per
+        // chain; associative: both per (chain, segment), plus the segments'
+        // sums of Delta
+        const size_t slots = static_cast<size_t>(chains) * (a.assoc ? nseg : 1);
+        const size_t nflags = slots * s6::kConsumerWarps;
         const size_t hdr = round_up(4 + 4 * nflags, 256);
-        const size_t carry = static_cast<size_t>(chains) * CPB * NS * sizeof(float);
+        const size_t carry = slots * CPB * NS * sizeof(float) + (a.assoc ? slots * CPB * sizeof(float) : 0);
         void *scr = nullptr;
         if (fixed) {
             if (hdr + carry > fixed->bytes)
@@ -272,51 +337,86 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
         a.counter = static_cast<unsigned int *>(scr);
         a.flags = a.counter + 1;
         a.carry = reinterpret_cast<float *>(static_cast<char *>(scr) + hdr);
+        a.carry_sum = a.carry + slots * CPB * NS;
         if (cudaMemsetAsync(scr, 0, 4 + 4 * nflags, stream) != cudaSuccess)
             return S6_ERR_CUDA;
-        grid = static_cast<unsigned>(chains < workers ? chains : workers);
+        const int64_t busy = a.assoc ? units : chains;  // units that can run at once
+        grid = static_cast<unsigned>(busy < workers ? busy : workers);
     }
     kern<<<grid, s6::kScanBlock, smem, stream>>>(tx, tdt, tz, ty, tB, tC, a);
     return launch_status(cudaGetLastError());
 }
 
-template <typename IO, bool CONV, bool ZOH, bool INIT>
+template <typename IO, bool CONV, int MODE, int EXT>
 int launch_scan_n(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, const ScanArgs &a,
                   cudaStream_t st, const FixedScratch *fixed = nullptr) {
-    if (dims->d_state <= 4)
-        return launch_scan_t<IO, 4, 1, CONV, ZOH, INIT>(dims, x, dt, z, y, a, st, fixed);
-    if (dims->d_state <= 8)
-        return launch_scan_t<IO, 8, 1, CONV, ZOH, INIT>(dims, x, dt, z, y, a, st, fixed);
-    return launch_scan_t<IO, 16, 2, CONV, ZOH, INIT>(dims, x, dt, z, y, a, st, fixed);
+    if constexpr (EXT == 2) {  // checkpoints: N = 16 only (checked by the caller)
+        return launch_scan_t<IO, 16, 2, CONV, MODE, 2>(dims, x, dt, z, y, a, st, fixed);
+    } else {
+        if (dims->d_state <= 4)
+            return launch_scan_t<IO, 4, 1, CONV, MODE, EXT>(dims, x, dt, z, y, a, st, fixed);
+        if (dims->d_state <= 8)
+            return launch_scan_t<IO, 8, 1, CONV, MODE, EXT>(dims, x, dt, z, y, a, st, fixed);
+        return launch_scan_t<IO, 16, 2, CONV, MODE, EXT>(dims, x, dt, z, y, a, st, fixed);
+    }
+}
+
+// Whether the problem has so few (sequence, channel tile) chains that the
+// associative split pays (decided again with the kernel's occupancy at launch).
+template <typename IO>
+bool few_chains(const s6_dims *dims) {
+    const int T = sizeof(IO) == 2 ? 64 : 32;
+    const int64_t cpb = dims->d_state <= 8 ? 128 : 64;  // channels per CTA tile
+    const int64_t chains = dims->batch * ((dims->d_inner + cpb - 1) / cpb);
+    return want_assoc(chains, dims->seqlen, T, 2 * static_cast<int64_t>(device_sm_count()));
 }
 
 template <typename IO>
-int launch_scan_io(const s6_dims *dims, bool conv, bool zoh, const void *x, const void *dt, const void *z, void *y,
+int launch_scan_io(const s6_dims *dims, bool conv, int mode, const void *x, const void *dt, const void *z, void *y,
                    const ScanArgs &a, cudaStream_t st, const FixedScratch *fixed = nullptr) {
-    if (a.h_init || a.conv_hist) {
+    using s6::kModeConst;
+    using s6::kModeSimplified;
+    using s6::kModeZOH;
+    if (mode == kModeConst)  // the constant-decay cell: no conv
+        return (a.h_init || few_chains<IO>(dims)) ? launch_scan_n<IO, false, kModeConst, 1>(dims, x, dt, z, y, a, st, fixed)
+                                                  : launch_scan_n<IO, false, kModeConst, 0>(dims, x, dt, z, y, a, st, fixed);
+    const bool zoh = mode == kModeZOH;
+    if (a.ckpt) {  // the backward's checkpointing forward
         if (conv)
-            return zoh ? launch_scan_n<IO, true, true, true>(dims, x, dt, z, y, a, st, fixed)
-                       : launch_scan_n<IO, true, false, true>(dims, x, dt, z, y, a, st, fixed);
-        return zoh ? launch_scan_n<IO, false, true, true>(dims, x, dt, z, y, a, st, fixed)
-                   : launch_scan_n<IO, false, false, true>(dims, x, dt, z, y, a, st, fixed);
+            return zoh ? launch_scan_n<IO, true, kModeZOH, 2>(dims, x, dt, z, y, a, st, fixed)
+                       : launch_scan_n<IO, true, kModeSimplified, 2>(dims, x, dt, z, y, a, st, fixed);
+        return zoh ? launch_scan_n<IO, false, kModeZOH, 2>(dims, x, dt, z, y, a, st, fixed)
+                   : launch_scan_n<IO, false, kModeSimplified, 2>(dims, x, dt, z, y, a, st, fixed);
+    }
+    // the extended instantiation: a given start state, or the associative split
+    if (a.h_init || a.conv_hist || few_chains<IO>(dims)) {
+        if (conv)
+            return zoh ? launch_scan_n<IO, true, kModeZOH, 1>(dims, x, dt, z, y, a, st, fixed)
+                       : launch_scan_n<IO, true, kModeSimplified, 1>(dims, x, dt, z, y, a, st, fixed);
+        return zoh ? launch_scan_n<IO, false, kModeZOH, 1>(dims, x, dt, z, y, a, st, fixed)
+                   : launch_scan_n<IO, false, kModeSimplified, 1>(dims, x, dt, z, y, a, st, fixed);
     }
     if (conv)
-        return zoh ? launch_scan_n<IO, true, true, false>(dims, x, dt, z, y, a, st, fixed)
-                   : launch_scan_n<IO, true, false, false>(dims, x, dt, z, y, a, st, fixed);
-    return zoh ? launch_scan_n<IO, false, true, false>(dims, x, dt, z, y, a, st, fixed)
-               : launch_scan_n<IO, false, false, false>(dims, x, dt, z, y, a, st, fixed);
+        return zoh ? launch_scan_n<IO, true, kModeZOH, 0>(dims, x, dt, z, y, a, st, fixed)
+                   : launch_scan_n<IO, true, kModeSimplified, 0>(dims, x, dt, z, y, a, st, fixed);
+    return zoh ? launch_scan_n<IO, false, kModeZOH, 0>(dims, x, dt, z, y, a, st, fixed)
+               : launch_scan_n<IO, false, kModeSimplified, 0>(dims, x, dt, z, y, a, st, fixed);
 }
 
+// mode: s6::kModeSimplified / kModeZOH (the zoh_mode argument of the scans) or
+// kModeConst (s6_diag_recurrence_fwd's constant decay: A_log carries the log2
+// of the decays, dt is not read).
 int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv_w, const float *conv_b,
                 const void *dt, const float *A_log, const void *B, const void *C, const float *D, const void *z,
-                const float *dt_bias, int zoh_mode, void *y, float *h_final, s6_stream_t stream,
+                const float *dt_bias, int mode, void *y, float *h_final, s6_stream_t stream,
                 const FixedScratch *fixed = nullptr, const float *h_init = nullptr,
-                const void *conv_hist = nullptr) {
+                const void *conv_hist = nullptr, float *ckpt = nullptr) {
     int st = check_dims(dims, true, conv);
     if (st != S6_OK)
         return st;
-    if (zoh_mode != 0 && zoh_mode != 1)
+    if (mode != s6::kModeSimplified && mode != s6::kModeZOH && mode != s6::kModeConst)
         return S6_ERR_INVALID_ARG;
+    const bool constd = mode == s6::kModeConst;
     if ((h_init && !aligned_to(h_init, 4)) || (conv_hist && !aligned_to(conv_hist, io_size(dims->io_dtype))))
         return S6_ERR_ALIGNMENT;
     if (dims->batch == 0 || dims->seqlen == 0) {
@@ -332,7 +432,7 @@ int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv
         }
         return S6_OK;
     }
-    if (!x || !dt || !A_log || !B || !C || !D || !y || (conv && !conv_w))
+    if (!x || (!dt && !constd) || !A_log || !B || !C || !D || !y || (conv && !conv_w) || (constd && conv))
         return S6_ERR_INVALID_ARG;
     const size_t es = io_size(dims->io_dtype);
     if ((dims->d_inner * es) % 16 != 0)
@@ -370,12 +470,13 @@ int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv
     a.h_final = h_final;
     a.h_init = h_init;
     a.conv_hist = conv ? conv_hist : nullptr;
+    a.ckpt = ckpt;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (use_stream_device(s) != S6_OK)
         return S6_ERR_CUDA;
     if (dims->io_dtype == S6_BF16)
-        return launch_scan_io<__nv_bfloat16>(dims, conv, zoh_mode == 1, x, dt, z, y, a, s, fixed);
-    return launch_scan_io<float>(dims, conv, zoh_mode == 1, x, dt, z, y, a, s, fixed);
+        return launch_scan_io<__nv_bfloat16>(dims, conv, mode, x, dt, z, y, a, s, fixed);
+    return launch_scan_io<float>(dims, conv, mode, x, dt, z, y, a, s, fixed);
 }
 
 // ------------------------------------------------------------ step dispatch
@@ -536,7 +637,7 @@ int launch_bwd_t(s6::BwdArgs a, cudaStream_t st) {
     const size_t ckf = static_cast<size_t>(a.nck) * NS * G;
     const size_t hbf = static_cast<size_t>(s6::kBwdChunk) * NS * G;
     void *scr = nullptr;
-    const int rc = get_scratch((ckf + hbf) * sizeof(float), st, &scr);
+    const int rc = get_scratch((ckf + hbf) * sizeof(float), st, &scr, kScratchCkpt);
     if (rc != S6_OK)
         return rc;
     a.ck = static_cast<float *>(scr);
@@ -562,6 +663,186 @@ int launch_bwd_io(const s6::BwdArgs &a, bool zoh, bool conv, cudaStream_t st) {
     if (conv)
         return zoh ? launch_bwd_n<IO, true, true>(a, st) : launch_bwd_n<IO, false, true>(a, st);
     return zoh ? launch_bwd_n<IO, true, false>(a, st) : launch_bwd_n<IO, false, false>(a, st);
+}
+
+// ------------------------------------------------- backward at N = 16 (pipelined)
+// The reverse kernel over persistent CTAs: (segment, chain) units pulled
+// last-segment-first when the chains alone would not balance the SMs.
+template <typename IO, bool ZOH, bool CONV>
+int launch_bwd_rev(const s6_dims *dims, s6::RevArgs r, const void *x, const void *dt, const void *z, const void *dy,
+                   const void *B, const void *C, cudaStream_t st) {
+    using Smem = s6::RevSmem<IO, CONV>;
+    static_assert(offsetof(Smem, x) % 128 == 0 && offsetof(Smem, dt) % 128 == 0 && offsetof(Smem, z) % 128 == 0 &&
+                      offsetof(Smem, dy) % 128 == 0 && offsetof(Smem, braw) % 128 == 0 &&
+                      offsetof(Smem, craw) % 128 == 0,
+                  "TMA buffers must be 128-byte aligned");
+    static_assert(offsetof(Smem, hbuf) % 16 == 0 && offsetof(Smem, bc) % 16 == 0 && offsetof(Smem, full) % 8 == 0,
+                  "vector and barrier fields must be aligned");
+    auto kern = s6::s6_scan_bwd_rev_kernel<IO, ZOH, CONV>;
+    const size_t smem = sizeof(Smem);
+    static int occ_dev[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return S6_ERR_CUDA;
+    if (!occ_dev[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+            return S6_ERR_CUDA;
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, s6::kScanBlock, smem) != cudaSuccess || nb < 1)
+            return S6_ERR_CUDA;
+        occ_dev[dev] = nb;
+    }
+    const int occ = occ_dev[dev];
+    constexpr int KC = s6::kRevChunk;
+    const int io = dims->io_dtype;
+    CUtensorMap tx, tdt, tz, tdy, tB, tC;
+    if (!make_map_3d(&tx, x, io, dims->batch, dims->seqlen, dims->d_inner, 64, Smem::XR) ||
+        !make_map_3d(&tdt, dt, io, dims->batch, dims->seqlen, dims->d_inner, 64, KC) ||
+        !make_map_3d(&tdy, dy, io, dims->batch, dims->seqlen, dims->d_inner, 64, KC) ||
+        !make_map_3d(&tB, B, io, dims->batch, dims->seqlen, 16, 16, KC) ||
+        !make_map_3d(&tC, C, io, dims->batch, dims->seqlen, 16, 16, KC))
+        return S6_ERR_CUDA;
+    if (z) {
+        if (!make_map_3d(&tz, z, io, dims->batch, dims->seqlen, dims->d_inner, 64, KC))
+            return S6_ERR_CUDA;
+    } else {
+        tz = tdt;  // never read
+    }
+    const int64_t L = dims->seqlen;
+    const int64_t chains = dims->batch * r.tiles;
+    const int64_t sms = device_sm_count();
+    int64_t per_sm = occ;
+    while (per_sm > 1 && per_sm * sms > chains)
+        --per_sm;
+    const int64_t workers = sms * per_sm;
+    int64_t nseg = 1, seg_len = round_up(static_cast<size_t>(L), KC);
+    if (chains < 4 * workers && L > 8 * KC) {
+        // about 8 units per worker, segments of at least 8 sub-chunks
+        const int64_t grid = chains < workers ? chains : workers;
+        int64_t want = (8 * grid + chains - 1) / chains;
+        const int64_t max_seg = L / (8 * KC);
+        if (want > max_seg)
+            want = max_seg;
+        if (want > 1) {
+            seg_len = round_up(static_cast<size_t>((L + want - 1) / want), KC);
+            nseg = (L + seg_len - 1) / seg_len;
+        }
+    }
+    if (chains * nseg > 0x7fffffffLL)
+        return S6_ERR_UNSUPPORTED;
+    r.nseg = static_cast<int>(nseg);
+    r.seg_len = static_cast<int>(seg_len);
+    r.units = static_cast<int>(chains * nseg);
+    r.dynamic = nseg > 1;
+    r.carry_polls = g_dbg_carry_polls.load();
+    unsigned grid = static_cast<unsigned>(chains);
+    if (r.dynamic) {
+        const size_t nflags = static_cast<size_t>(chains) * s6::kConsumerWarps;
+        const size_t hdr = round_up(4 + 4 * nflags, 256);
+        const size_t carry = static_cast<size_t>(chains) * 64 * s6::kRevCarry * sizeof(float);
+        void *scr = nullptr;
+        const int rc = get_scratch(hdr + carry, st, &scr, kScratchRev);
+        if (rc != S6_OK)
+            return rc;
+        r.counter = static_cast<unsigned int *>(scr);
+        r.flags = r.counter + 1;
+        r.carry = reinterpret_cast<float *>(static_cast<char *>(scr) + hdr);
+        if (cudaMemsetAsync(scr, 0, 4 + 4 * nflags, st) != cudaSuccess)
+            return S6_ERR_CUDA;
+        grid = static_cast<unsigned>(chains < workers ? chains : workers);
+    }
+    kern<<<grid, s6::kScanBlock, smem, st>>>(tx, tdt, tz, tdy, tB, tC, r);
+    return launch_status(cudaGetLastError());
+}
+
+// Whether the pipelined backward applies: N = 16 and rows that the tensor unit
+// can move (16-byte aligned bases, d * sizeof(io) a multiple of 16).
+bool bwd_rev_ok(const s6_dims *dims, const void *x, const void *dt, const void *z, const void *dy, const void *B,
+                const void *C) {
+    if (dims->d_state != 16 || (dims->d_inner * io_size(dims->io_dtype)) % 16 != 0)
+        return false;
+    const void *p[] = {x, dt, z, dy, B, C};
+    for (const void *q : p)
+        if (q && !aligned16(q))
+            return false;
+    return true;
+}
+
+// The pipelined backward: the forward kernel stores the state every
+// kRevChunk tokens, the reverse kernel walks the chains back and writes
+// per-tile dB / dC rows, and a reduction sums them over the tiles.
+int bwd_rev(const s6_dims *dims, bool conv, const void *x, const float *conv_w, const float *conv_b, const void *dt,
+            const float *A_log, const void *B, const void *C, const float *D, const void *z, const float *dt_bias,
+            int zoh_mode, const float *h_init, const void *dy, float *dx, float *dconv_w, float *dconv_b, float *ddt,
+            float *dz, float *dB, float *dC, float *dA_log, float *dD, float *ddt_bias, float *dh_init,
+            cudaStream_t s) {
+    const int64_t Bt = dims->batch, L = dims->seqlen, d = dims->d_inner;
+    const int64_t nck = (L + s6::kRevChunk - 1) / s6::kRevChunk;
+    const int64_t tiles = (d + 63) / 64;
+    void *ck = nullptr, *pt = nullptr;
+    int rc = get_scratch(sizeof(float) * Bt * nck * d * 16, s, &ck, kScratchCkpt);
+    if (rc == S6_OK)
+        rc = get_scratch(sizeof(float) * tiles * Bt * L * 32, s, &pt, kScratchPart);
+    if (rc != S6_OK)
+        return rc;
+    // 1. the forward with checkpoints (no outputs)
+    const s6_dims fd = *dims;
+    rc = scan_common(&fd, conv, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode,
+                     const_cast<void *>(x), nullptr, reinterpret_cast<s6_stream_t>(s), nullptr, h_init, nullptr,
+                     static_cast<float *>(ck));
+    if (rc != S6_OK)
+        return rc;
+    // 2. the reverse walk
+    s6::RevArgs r;
+    std::memset(&r, 0, sizeof(r));
+    r.Bt = static_cast<int>(Bt);
+    r.L = static_cast<int>(L);
+    r.d = static_cast<int>(d);
+    r.K = conv ? static_cast<int>(dims->conv_width) : 0;
+    r.has_z = z != nullptr;
+    r.tiles = static_cast<int>(tiles);
+    r.nck = static_cast<int>(nck);
+    r.A_log = A_log;
+    r.D = D;
+    r.dt_bias = dt_bias;
+    r.conv_w = conv_w;
+    r.conv_b = conv_b;
+    r.ckpt = static_cast<const float *>(ck);
+    r.du = dx;
+    r.ddt = ddt;
+    r.dz = dz;
+    r.part = static_cast<float *>(pt);
+    r.dA_log = dA_log;
+    r.dD = dD;
+    r.ddt_bias = ddt_bias;
+    r.dconv_w = dconv_w;
+    r.dconv_b = dconv_b;
+    r.dh_init = dh_init;
+    const bool zoh = zoh_mode == 1;
+    if (dims->io_dtype == S6_BF16) {
+        using T = __nv_bfloat16;
+        rc = conv ? (zoh ? launch_bwd_rev<T, true, true>(dims, r, x, dt, z, dy, B, C, s)
+                         : launch_bwd_rev<T, false, true>(dims, r, x, dt, z, dy, B, C, s))
+                  : (zoh ? launch_bwd_rev<T, true, false>(dims, r, x, dt, z, dy, B, C, s)
+                         : launch_bwd_rev<T, false, false>(dims, r, x, dt, z, dy, B, C, s));
+    } else {
+        rc = conv ? (zoh ? launch_bwd_rev<float, true, true>(dims, r, x, dt, z, dy, B, C, s)
+                         : launch_bwd_rev<float, false, true>(dims, r, x, dt, z, dy, B, C, s))
+                  : (zoh ? launch_bwd_rev<float, true, false>(dims, r, x, dt, z, dy, B, C, s)
+                         : launch_bwd_rev<float, false, false>(dims, r, x, dt, z, dy, B, C, s));
+    }
+    if (rc != S6_OK)
+        return rc;
+    // 3. dB, dC over the tiles
+    const long long rows = Bt * L;
+    long long blocks = (rows * 32 + 255) / 256;
+    const long long cap = static_cast<long long>(device_sm_count()) * 8;
+    if (blocks > cap)
+        blocks = cap;
+    s6::s6_bwd_bc_reduce_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(static_cast<const float *>(pt),
+                                                                             static_cast<int>(tiles), rows, dB, dC);
+    return launch_status(cudaGetLastError());
 }
 
 // The backward entry points share their checks and set-up; `conv` selects the
@@ -611,6 +892,9 @@ int bwd_common(const s6_dims *dims, bool conv, const void *x, const float *conv_
             return S6_ERR_CUDA;
         return S6_OK;
     }
+    if (bwd_rev_ok(dims, x, dt, z, dy, B, C))
+        return bwd_rev(dims, conv, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, h_init, dy, dx,
+                       dconv_w, dconv_b, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, s);
     s6::BwdArgs a;
     std::memset(&a, 0, sizeof(a));
     a.Bt = static_cast<int>(Bt);
@@ -669,6 +953,9 @@ const char *s6_status_string(int status) {
 int s6_scan_fwd(const s6_dims *dims, const void *u, const void *dt, const float *A_log, const void *B, const void *C,
                 const float *D, const void *z, const float *dt_bias, int zoh_mode, void *y, float *h_final,
                 s6_stream_t stream) {
+    DeviceRestore restore_device;
+    if (zoh_mode != 0 && zoh_mode != 1)
+        return S6_ERR_INVALID_ARG;
     return scan_common(dims, false, u, nullptr, nullptr, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final,
                        stream);
 }
@@ -676,6 +963,9 @@ int s6_scan_fwd(const s6_dims *dims, const void *u, const void *dt, const float 
 int s6_conv_scan_fwd(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b, const void *dt,
                      const float *A_log, const void *B, const void *C, const float *D, const void *z,
                      const float *dt_bias, int zoh_mode, void *y, float *h_final, s6_stream_t stream) {
+    DeviceRestore restore_device;
+    if (zoh_mode != 0 && zoh_mode != 1)
+        return S6_ERR_INVALID_ARG;
     return scan_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final,
                        stream);
 }
@@ -684,6 +974,9 @@ int s6_conv_scan_fwd_noalloc(const s6_dims *dims, const void *x, const float *co
                              const void *dt, const float *A_log, const void *B, const void *C, const float *D,
                              const void *z, const float *dt_bias, int zoh_mode, void *y, float *h_final,
                              s6_stream_t stream) {
+    DeviceRestore restore_device;
+    if (zoh_mode != 0 && zoh_mode != 1)
+        return S6_ERR_INVALID_ARG;
     FixedScratch fx;
     const int st = noalloc_scratch(reinterpret_cast<cudaStream_t>(stream), &fx);
     if (st != S6_OK)
@@ -695,6 +988,9 @@ int s6_conv_scan_fwd_noalloc(const s6_dims *dims, const void *x, const float *co
 int s6_scan_fwd_from_state(const s6_dims *dims, const void *u, const void *dt, const float *A_log, const void *B,
                            const void *C, const float *D, const void *z, const float *dt_bias, int zoh_mode,
                            const float *h_init, void *y, float *h_final, s6_stream_t stream) {
+    DeviceRestore restore_device;
+    if (zoh_mode != 0 && zoh_mode != 1)
+        return S6_ERR_INVALID_ARG;
     return scan_common(dims, false, u, nullptr, nullptr, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final,
                        stream, nullptr, h_init, nullptr);
 }
@@ -703,14 +999,32 @@ int s6_conv_scan_fwd_from_state(const s6_dims *dims, const void *x, const float 
                                 const void *dt, const float *A_log, const void *B, const void *C, const float *D,
                                 const void *z, const float *dt_bias, int zoh_mode, const float *h_init,
                                 const void *conv_hist, void *y, float *h_final, s6_stream_t stream) {
+    DeviceRestore restore_device;
+    if (zoh_mode != 0 && zoh_mode != 1)
+        return S6_ERR_INVALID_ARG;
     return scan_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, stream,
                        nullptr, h_init, conv_hist);
+}
+
+int s6_diag_recurrence_fwd(const s6_dims *dims, int decay_source, const void *u, const void *dt, const float *A_log,
+                           const float *dt_bias, const float *log2_decay, const void *B, const void *C,
+                           const float *D, const void *z, const float *h_init, void *y, float *h_final,
+                           s6_stream_t stream) {
+    DeviceRestore restore_device;
+    if (decay_source == S6_DECAY_LIVE)
+        return scan_common(dims, false, u, nullptr, nullptr, dt, A_log, B, C, D, z, dt_bias, s6::kModeSimplified, y,
+                           h_final, stream, nullptr, h_init, nullptr);
+    if (decay_source == S6_DECAY_CONST)
+        return scan_common(dims, false, u, nullptr, nullptr, nullptr, log2_decay, B, C, D, z, nullptr,
+                           s6::kModeConst, y, h_final, stream, nullptr, h_init, nullptr);
+    return S6_ERR_INVALID_ARG;
 }
 
 int s6_scan_bwd(const s6_dims *dims, const void *u, const void *dt, const float *A_log, const void *B, const void *C,
                 const float *D, const void *z, const float *dt_bias, int zoh_mode, const float *h_init, const void *dy,
                 float *du, float *ddt, float *dz, float *dB, float *dC, float *dA_log, float *dD, float *ddt_bias,
                 float *dh_init, s6_stream_t stream) {
+    DeviceRestore restore_device;
     return bwd_common(dims, false, u, nullptr, nullptr, dt, A_log, B, C, D, z, dt_bias, zoh_mode, h_init, dy, du,
                       nullptr, nullptr, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, stream);
 }
@@ -720,12 +1034,14 @@ int s6_conv_scan_bwd(const s6_dims *dims, const void *x, const float *conv_w, co
                      const float *dt_bias, int zoh_mode, const float *h_init, const void *dy, float *dx,
                      float *dconv_w, float *dconv_b, float *ddt, float *dz, float *dB, float *dC, float *dA_log,
                      float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream) {
+    DeviceRestore restore_device;
     return bwd_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, h_init, dy, dx,
                       dconv_w, dconv_b, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, stream);
 }
 
 int causal_conv1d_silu_fwd(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b, void *out,
                            s6_stream_t stream) {
+    DeviceRestore restore_device;
     int st = check_dims(dims, true, true);
     if (st != S6_OK)
         return st;
@@ -755,6 +1071,7 @@ int causal_conv1d_silu_fwd(const s6_dims *dims, const void *x, const float *conv
 int s6_step(const s6_dims *dims, const float *A_log, const float *D, const float *dt_bias, const float *conv_w,
             const float *conv_b, int zoh_mode, const void *u_t, const void *dt_t, const void *B_t, const void *C_t,
             const void *z_t, float *h_ssm, void *conv_state, void *y_t, s6_stream_t stream) {
+    DeviceRestore restore_device;
     int st = check_dims(dims, false, true);
     if (st != S6_OK)
         return st;
@@ -806,9 +1123,166 @@ int s6_step(const s6_dims *dims, const float *A_log, const float *D, const float
     return zoh_mode ? launch_step_n<float, true>(a, s) : launch_step_n<float, false>(a, s);
 }
 
+// Fault injection for tests: makes one unit of the next segmented scans skip
+// publishing its carry, with a short poll limit, so that the successor's bounded
+// wait runs out (S6_ERR_TIMEOUT through s6_device_status).  Host-side state only.
+int s6_debug_carry_fault(int skip_publish_unit, unsigned int carry_polls) {
+    g_dbg_skip_publish.store(skip_publish_unit < 0 ? -1 : skip_publish_unit);
+    g_dbg_carry_polls.store(carry_polls == 0 ? kCarryPolls : carry_polls);
+    return S6_OK;
+}
+
+int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x, float *conv_state, float *h_ssm,
+                  s6_stream_t stream) {
+    DeviceRestore restore_device;
+    if (!dims || !w)
+        return S6_ERR_INVALID_ARG;
+    const int64_t Bt = dims->batch, dm = dims->d_model, di = dims->d_inner, N = dims->d_state, R = dims->dt_rank,
+                  K = dims->conv_width;
+    if (Bt < 0 || dm < 1 || di < 1 || N < 1 || R < 1 || !(dims->eps >= 0.0f))
+        return S6_ERR_INVALID_ARG;
+    if (N > kMaxState || K < 2 || K > 4)
+        return S6_ERR_UNSUPPORTED;
+    if (Bt > (1 << 20) || dm > (1 << 20) || di > (1 << 24) || R > 1024)
+        return S6_ERR_UNSUPPORTED;
+    if (Bt == 0)
+        return S6_OK;
+    const void *req[] = {w->ln_w, w->ln_b, w->in_q, w->in_s, w->conv_w, w->xp_q, w->xp_s, w->dt_q, w->dt_s,
+                         w->dt_bias, w->A_log, w->D, w->out_q, w->out_s, x, conv_state, h_ssm};
+    for (const void *p : req)
+        if (!p)
+            return S6_ERR_INVALID_ARG;
+    const void *f32p[] = {w->ln_w, w->ln_b, w->in_s, w->conv_w, w->conv_b, w->xp_s, w->dt_s, w->dt_bias, w->A_log,
+                          w->D, w->out_s, x, conv_state, h_ssm};
+    for (const void *p : f32p)
+        if (p && !aligned_to(p, 4))
+            return S6_ERR_ALIGNMENT;
+    if (N == 16 && (!aligned16(w->A_log) || !aligned16(h_ssm)))
+        return S6_ERR_ALIGNMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (use_stream_device(s) != S6_OK)
+        return S6_ERR_CUDA;
+    // intermediate rows: xin | z, the x_proj rows (dt | B | C), the gated readout
+    const int64_t row = R + 2 * N;
+    void *scr = nullptr;
+    const size_t fl = static_cast<size_t>(Bt) * (2 * di + round_up(static_cast<size_t>(row), 4) + di);
+    int rc = get_scratch(fl * sizeof(float), s, &scr, kScratchBlock);
+    if (rc != S6_OK)
+        return rc;
+    float *xz = static_cast<float *>(scr);
+    float *dbc = xz + static_cast<size_t>(Bt) * 2 * di;
+    float *g = dbc + static_cast<size_t>(Bt) * round_up(static_cast<size_t>(row), 4);
+    const int64_t sms = device_sm_count();
+    const unsigned mt = static_cast<unsigned>((Bt + s6::kGemmBM - 1) / s6::kGemmBM);
+    auto splits_for = [&](int64_t n_out, int64_t k) {
+        // enough reduction slices to put about two blocks on every SM
+        const int64_t tiles = ((n_out + s6::kGemmBN - 1) / s6::kGemmBN) * mt;
+        int64_t sp = (2 * sms + tiles - 1) / tiles;
+        const int64_t max_sp = (k + s6::kGemmBK - 1) / s6::kGemmBK;
+        if (sp > max_sp)
+            sp = max_sp;
+        if (sp < 1)
+            sp = 1;
+        const int64_t ks = round_up(static_cast<size_t>((k + sp - 1) / sp), s6::kGemmBK);
+        return std::make_pair(static_cast<int>((k + ks - 1) / ks), static_cast<int>(ks));
+    };
+    // 1. LayerNorm + in_proj -> xin | z
+    s6::Q8GemmArgs g1;
+    std::memset(&g1, 0, sizeof(g1));
+    g1.M = static_cast<int>(Bt);
+    g1.N = static_cast<int>(2 * di);
+    g1.K = static_cast<int>(dm);
+    g1.x = x;
+    g1.ldx = static_cast<int>(dm);
+    g1.wq = w->in_q;
+    g1.ws = w->in_s;
+    g1.y = xz;
+    g1.ldy = static_cast<int>(2 * di);
+    g1.k_split = static_cast<int>(dm);
+    g1.ln_w = w->ln_w;
+    g1.ln_b = w->ln_b;
+    g1.eps = dims->eps;
+    s6::q8_gemm_kernel<s6::kProLN><<<dim3(static_cast<unsigned>((2 * di + s6::kGemmBN - 1) / s6::kGemmBN), mt, 1),
+                                     s6::kGemmThreads, 0, s>>>(g1);
+    if (cudaGetLastError() != cudaSuccess)
+        return S6_ERR_CUDA;
+    // 2. conv + SiLU + x_proj -> dt | B | C (split over the channels, summed atomically)
+    if (cudaMemsetAsync(dbc, 0, sizeof(float) * Bt * round_up(static_cast<size_t>(row), 4), s) != cudaSuccess)
+        return S6_ERR_CUDA;
+    const auto sp2 = splits_for(row, di);
+    s6::Q8GemmArgs g2;
+    std::memset(&g2, 0, sizeof(g2));
+    g2.M = static_cast<int>(Bt);
+    g2.N = static_cast<int>(row);
+    g2.K = static_cast<int>(di);
+    g2.x = xz;
+    g2.ldx = static_cast<int>(2 * di);
+    g2.wq = w->xp_q;
+    g2.ws = w->xp_s;
+    g2.y = dbc;
+    g2.ldy = static_cast<int>(round_up(static_cast<size_t>(row), 4));
+    g2.accumulate = 1;
+    g2.k_split = sp2.second;
+    g2.hist = conv_state;
+    g2.conv_w = w->conv_w;
+    g2.conv_b = w->conv_b;
+    g2.Kc = static_cast<int>(K);
+    s6::q8_gemm_kernel<s6::kProConv><<<dim3(static_cast<unsigned>((row + s6::kGemmBN - 1) / s6::kGemmBN), mt,
+                                            static_cast<unsigned>(sp2.first)),
+                                       s6::kGemmThreads, 0, s>>>(g2);
+    if (cudaGetLastError() != cudaSuccess)
+        return S6_ERR_CUDA;
+    // 3. dt_proj + the recurrence + readout + gate
+    s6::BlockSsmArgs a3;
+    a3.Bt = static_cast<int>(Bt);
+    a3.di = static_cast<int>(di);
+    a3.N = static_cast<int>(N);
+    a3.R = static_cast<int>(R);
+    a3.Kc = static_cast<int>(K);
+    a3.xz = xz;
+    a3.dbc = dbc;
+    a3.dt_q = w->dt_q;
+    a3.dt_s = w->dt_s;
+    a3.dt_bias = w->dt_bias;
+    a3.A_log = w->A_log;
+    a3.D = w->D;
+    a3.conv_w = w->conv_w;
+    a3.conv_b = w->conv_b;
+    a3.hist = conv_state;
+    a3.h = h_ssm;
+    a3.g = g;
+    // the x_proj rows were written with a padded stride
+    a3.dbc_ld = static_cast<int>(round_up(static_cast<size_t>(row), 4));
+    s6::block_ssm_kernel<16><<<dim3(static_cast<unsigned>((di + s6::kSsmThreads - 1) / s6::kSsmThreads),
+                                    static_cast<unsigned>(Bt)),
+                               s6::kSsmThreads, sizeof(float) * row, s>>>(a3);
+    if (cudaGetLastError() != cudaSuccess)
+        return S6_ERR_CUDA;
+    // 4. out_proj, added into the residual stream
+    const auto sp4 = splits_for(dm, di);
+    s6::Q8GemmArgs g4;
+    std::memset(&g4, 0, sizeof(g4));
+    g4.M = static_cast<int>(Bt);
+    g4.N = static_cast<int>(dm);
+    g4.K = static_cast<int>(di);
+    g4.x = g;
+    g4.ldx = static_cast<int>(di);
+    g4.wq = w->out_q;
+    g4.ws = w->out_s;
+    g4.y = x;
+    g4.ldy = static_cast<int>(dm);
+    g4.accumulate = 1;
+    g4.k_split = sp4.second;
+    s6::q8_gemm_kernel<s6::kProPlain><<<dim3(static_cast<unsigned>((dm + s6::kGemmBN - 1) / s6::kGemmBN), mt,
+                                             static_cast<unsigned>(sp4.first)),
+                                        s6::kGemmThreads, 0, s>>>(g4);
+    return launch_status(cudaGetLastError());
+}
+
 // Read and clear the device-side error word after the stream's work so far
 // (synchronises `stream`).  S6_ERR_TIMEOUT if a bounded wait gave up.
 int s6_device_status(s6_stream_t stream) {
+    DeviceRestore restore_device;
     unsigned int v = 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (use_stream_device(s) != S6_OK)

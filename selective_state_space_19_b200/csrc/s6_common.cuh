@@ -202,33 +202,6 @@ __device__ __forceinline__ f2_t f2_softplus_fast(f2_t v) {
     return f2_fma(e, q, f2_pack(fmaxf(v0, 0.0f), fmaxf(v1, 0.0f)));
 }
 
-// 2^x for a pair x <= 0 on the FMA pipe: x = n + f with n = round(x) taken
-// from the low mantissa bits of x + 1.5*2^23, f in [-1/2, 1/2], 2^f by a
-// degree-6 polynomial (float32 relative error 7.9e-8), scaled by adding n to
-// the exponent field.  x is clamped at -125 (results stay normal; the decay
-// is below 1e-37 there).
-__device__ __forceinline__ f2_t f2_exp2_poly(f2_t x) {
-    float x0, x1;
-    f2_unpack(x, x0, x1);
-    x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-    const f2_t magic = f2_pack(12582912.0f, 12582912.0f);
-    const f2_t t = f2_add(x, magic);
-    const f2_t f = f2_sub(x, f2_sub(t, magic));
-    f2_t p = f2_pack(0.0001534580806037411f, 0.0001534580806037411f);
-    p = f2_fma(p, f, f2_pack(0.0013399930903688073f, 0.0013399930903688073f));
-    p = f2_fma(p, f, f2_pack(0.009618489071726799f, 0.009618489071726799f));
-    p = f2_fma(p, f, f2_pack(0.05550328642129898f, 0.05550328642129898f));
-    p = f2_fma(p, f, f2_pack(0.24022646248340607f, 0.24022646248340607f));
-    p = f2_fma(p, f, f2_pack(0.6931471824645996f, 0.6931471824645996f));
-    p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
-    float t0, t1, p0, p1;
-    f2_unpack(t, t0, t1);
-    f2_unpack(p, p0, p1);
-    p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-    return f2_pack(p0, p1);
-}
-
 // softplus(v) = log(1 + e^v) = max(v, 0) + log1p(e^-|v|).
 // log1p(e) is formed as log2(1 + e) * ln2, corrected for the rounding of
 // 1 + e by the factor e / ((1 + e) - 1) (the subtraction is exact); when

@@ -77,6 +77,16 @@ constexpr int kMetaFirst = 1;  // first chunk of its unit
 constexpr int kMetaLast = 2;   // last chunk of its unit
 constexpr int kMetaEnd = 4;    // no more work
 constexpr int kMetaCarry = 8;  // the unit starts from a published carry or the given start state
+constexpr int kMetaNoY = 16;   // associative split: a state-only unit (no outputs)
+
+constexpr int kCkptEvery = 16;  // tokens between the backward's state checkpoints
+
+// Write and decay forms (the MODE template argument).
+constexpr int kModeSimplified = 0;  // decay 2^(Delta A log2 e), write Delta B u
+constexpr int kModeZOH = 1;         // decay as above, write (A_bar - 1)/A B u
+constexpr int kModeConst = 2;       // constant decay 2^w per (channel, state), write B u:
+                                    // the constant-decay cell of "the s6 cell",
+                                    // "one cell, two architectures"; A_log carries w
 
 struct ScanArgs {
     int Bt, L, d, N, K;
@@ -84,8 +94,9 @@ struct ScanArgs {
     int tiles;    // channel tiles per sequence
     int nseg;     // segments per sequence
     int seg_len;  // tokens per segment (a multiple of the chunk length)
-    int units;    // Bt * tiles * nseg
+    int units;    // Bt * tiles * nseg (serial), Bt * tiles * (2 nseg - 1) (associative)
     int dynamic;  // 1: persistent CTAs pull units from *counter
+    int assoc;    // 1: associative split (extended instantiation only)
     int bc_tma;   // 1: B/C rows arrive by TMA with the stage
     const void *B;  // [Bt, L, N] io (read directly when bc_tma == 0)
     const void *C;
@@ -97,9 +108,17 @@ struct ScanArgs {
     float *h_final;        // [Bt, d, N] or null
     unsigned int *counter;  // dynamic: next unit to hand out (zeroed before launch)
     unsigned int *flags;    // dynamic: [Bt*tiles][consumer warps] last published segment + 1
-    float *carry;           // dynamic: [Bt*tiles][CPB][NS] published end states
+    float *carry;           // serial: [Bt*tiles][CPB][NS] published end states;
+                            // associative: [Bt*tiles][nseg][CPB][NS] end state of segment 0 (slot 0)
+                            // and the state-only units' states from zero (slots 1..nseg-1)
+    float *carry_sum;       // associative: [Bt*tiles][nseg][CPB] sum of Delta over each state-only unit
     const float *h_init;    // [Bt, d, N] start state, or null (zeros)
     const void *conv_hist;  // [Bt, d, K-1] io conv history before token 0 (oldest first), or null (zeros)
+    float *ckpt;               // extended instantiation, N = 16: the state before every
+                               // kCkptEvery-th token, [Bt][ceil(L / kCkptEvery)][d][16]
+                               // (the backward's checkpoints); y is then not written.  Or null.
+    unsigned int carry_polls;  // polls of a predecessor's flag before the wait gives up
+    int skip_publish;          // fault injection for tests: this unit publishes no carry (-1: none)
 };
 
 template <int NS, int TPC, int T, bool CONV>
@@ -140,13 +159,32 @@ struct ScanSmem {
 
 struct UnitPos {
     int b, tile, seg, chain;
+    bool state_only;  // associative split: scan from zero, outputs not written
 };
 
+// Unit order.  Serial split: segment-major, unit u = seg * chains + chain.
+// Associative split: first every chain's segment 0 (a full unit), then the
+// state-only units of segments 1..nseg-1, then the full units of segments
+// 1..nseg-1 -- each in segment-major order.  A unit only ever waits for units
+// handed out before it.
 __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
     const int per = a.Bt * a.tiles;
     UnitPos p;
-    p.seg = u / per;
-    p.chain = u - p.seg * per;
+    p.state_only = false;
+    if (a.assoc) {
+        const int ns = a.nseg;
+        if (u >= per * ns) {
+            u -= per * ns;
+            p.seg = u / per + 1;
+        } else {
+            p.seg = u / per;
+            p.state_only = p.seg > 0;
+        }
+        p.chain = u - (u / per) * per;
+    } else {
+        p.seg = u / per;
+        p.chain = u - p.seg * per;
+    }
     p.b = p.chain / a.tiles;
     p.tile = p.chain - p.b * a.tiles;
     return p;
@@ -154,9 +192,11 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
 
 constexpr uint32_t kWaitPolls = 1u << 24;
 
-// INIT: the scan may start from a given state (h_init, conv_hist); a separate
-// instantiation, so that the plain scan's code is not touched by it.
-template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, bool ZOH, bool INIT>
+// EXT: 0 the plain scan; 1 the extended scan, which may start from a given
+// state (h_init, conv_hist) and may take the associative split; 2 the
+// extended scan in checkpoint mode for the backward (N = 16 only).  Separate
+// instantiations, so that each one carries only its own code.
+template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, int MODE, int EXT>
 __global__ void __launch_bounds__(kScanBlock, 2)
     s6_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
@@ -165,6 +205,11 @@ __global__ void __launch_bounds__(kScanBlock, 2)
     using Sh = ScanShape<NS, TPC, T, CONV>;
     using Smem = ScanSmem<IO, NS, TPC, T, STAGES, CONV>;
     using tr = io_traits<IO>;
+    constexpr bool ZOH = MODE == kModeZOH;
+    constexpr bool CONSTD = MODE == kModeConst;  // decay from a constant, no step size
+    constexpr bool INIT = EXT >= 1;  // given start state, associative split
+    constexpr bool CKPT = EXT == 2;  // checkpoints for the backward, no outputs
+    static_assert(!CKPT || (NS == 16 && TPC == 2), "checkpoints are kept at N = 16 only");
     constexpr int NH = Sh::NH;
     constexpr int NP = NH / 2;  // state pairs per thread
     constexpr int CPB = Sh::CPB;
@@ -192,7 +237,8 @@ __global__ void __launch_bounds__(kScanBlock, 2)
         // =========================================================== producer
         if (lane == 0) {
             prefetch_tensormap(&tm_x);
-            prefetch_tensormap(&tm_dt);
+            if (!CONSTD)
+                prefetch_tensormap(&tm_dt);
             if (a.has_z)
                 prefetch_tensormap(&tm_z);
             if (a.bc_tma) {
@@ -329,19 +375,20 @@ __global__ void __launch_bounds__(kScanBlock, 2)
             }
             const UnitPos up = unit_pos(unit, a);
             const int t0 = tlo + k * T;
-            const bool carry_in = a.dynamic && k == 0 && up.seg > 0;
+            const bool carry_in = a.dynamic && k == 0 && up.seg > 0 && !up.state_only;
             const bool given_in = INIT && a.h_init && k == 0 && up.seg == 0;  // a chain's start state is given
             const int fl = (k == 0 ? kMetaFirst : 0) | (k == nk - 1 ? kMetaLast : 0) |
-                           (carry_in || given_in ? kMetaCarry : 0);
+                           (carry_in || given_in ? kMetaCarry : 0) | (up.state_only ? kMetaNoY : 0);
             if (lane == 0) {
                 sm.meta[s] = make_int4(unit, t0, min(T, thi - t0), fl);
                 const int c0 = up.tile * CPB;
                 constexpr uint32_t kX = XR * CPB * sizeof(IO);
                 constexpr uint32_t kR = T * CPB * sizeof(IO);
                 const uint32_t kBC = a.bc_tma ? 2u * T * a.N * static_cast<uint32_t>(sizeof(IO)) : 0u;
-                mbar_arrive_expect_tx(&sm.full[s], kX + kR + (a.has_z ? kR : 0u) + kBC);
+                mbar_arrive_expect_tx(&sm.full[s], kX + (CONSTD ? 0u : kR) + (a.has_z ? kR : 0u) + kBC);
                 tma_load_3d(&sm.x[s].v[0][0], &tm_x, &sm.full[s], c0, t0 - (CONV ? kHalo : 0), up.b);
-                tma_load_3d(&sm.dt[s].v[0][0], &tm_dt, &sm.full[s], c0, t0, up.b);
+                if (!CONSTD)
+                    tma_load_3d(&sm.dt[s].v[0][0], &tm_dt, &sm.full[s], c0, t0, up.b);
                 if (a.has_z)
                     tma_load_3d(&sm.z[s].v[0][0], &tm_z, &sm.full[s], c0, t0, up.b);
                 if (a.bc_tma) {
@@ -361,28 +408,77 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                 }
             }
             if (carry_in) {
-                // the predecessor segment publishes one flag per consumer warp
-                bool got = true;
-                if (lane < kConsumerWarps) {
-                    got = false;
-                    const unsigned int *f = &a.flags[static_cast<size_t>(up.chain) * kConsumerWarps + lane];
-                    for (uint32_t i = 0; i < (1u << 22); ++i) {
-                        if (ld_acquire_gpu(f) >= static_cast<unsigned int>(up.seg)) {
-                            got = true;
-                            break;
+                if (INIT && a.assoc) {
+                    // Associative split.  The start state of segment `seg` is
+                    // E_{seg-1}, folded from segment 0's end state E_0 and the
+                    // state-only units' (P_j, s_j) for j = 1 .. seg-1:
+                    //     E_j = P_j * E_{j-1} + s_j,   P_j = prod of the segment's
+                    //     decays = 2^(A log2 e * sum of its Delta)
+                    // -- the pair combine (a1, b1) o (a2, b2) = (a1 a2, a2 b1 + b2)
+                    // applied left to right.  Every unit folded here was handed
+                    // out before this one, so the (bounded) waits end.
+                    const size_t base = static_cast<size_t>(up.chain) * a.nseg;
+                    bool got = true;
+                    if (lane < kConsumerWarps) {
+                        for (int j = 0; j < up.seg && got; ++j) {
+                            got = false;
+                            const unsigned int *f = &a.flags[(base + j) * kConsumerWarps + lane];
+                            for (uint32_t i = 0; i < a.carry_polls; ++i) {
+                                if (ld_acquire_gpu(f) >= 1u) {
+                                    got = true;
+                                    break;
+                                }
+                                __nanosleep(64);
+                            }
                         }
-                        __nanosleep(64);
                     }
+                    if (!__all_sync(0xffffffffu, got)) {
+                        if (lane == 0)
+                            raise_device_error(2u);
+                    }
+                    const int c0 = up.tile * CPB;
+                    for (int i = lane; i < CPB * NS; i += 32) {
+                        const int ch = i / NS;
+                        const int n = i - ch * NS;
+                        const int cc = c0 + ch;
+                        // A log2 e with A = -exp(A_log) (the constant cell: w, the log2
+                        // of its decay, with a unit step per token); zero for padding
+                        float A2 = 0.0f;
+                        if (cc < a.d && n < a.N) {
+                            const float al = a.A_log[static_cast<size_t>(cc) * a.N + n];
+                            A2 = CONSTD ? al : -expf(al) * kLog2e;
+                        }
+                        float h = __ldcg(a.carry + base * CPB * NS + i);
+                        for (int j = 1; j < up.seg; ++j) {
+                            const float sj = __ldcg(a.carry_sum + (base + j) * CPB + ch);
+                            h = fmaf(ex2_approx(A2 * sj), h, __ldcg(a.carry + (base + j) * CPB * NS + i));
+                        }
+                        sm.hinit[s][ch][n] = h;
+                    }
+                } else {
+                    // the predecessor segment publishes one flag per consumer warp
+                    bool got = true;
+                    if (lane < kConsumerWarps) {
+                        got = false;
+                        const unsigned int *f = &a.flags[static_cast<size_t>(up.chain) * kConsumerWarps + lane];
+                        for (uint32_t i = 0; i < a.carry_polls; ++i) {
+                            if (ld_acquire_gpu(f) >= static_cast<unsigned int>(up.seg)) {
+                                got = true;
+                                break;
+                            }
+                            __nanosleep(64);
+                        }
+                    }
+                    if (!__all_sync(0xffffffffu, got)) {
+                        if (lane == 0)
+                            raise_device_error(2u);
+                    }
+                    const float4 *src =
+                        reinterpret_cast<const float4 *>(a.carry + static_cast<size_t>(up.chain) * CPB * NS);
+                    float4 *dst = reinterpret_cast<float4 *>(&sm.hinit[s][0][0]);
+                    for (int i = lane; i < CPB * NS / 4; i += 32)
+                        dst[i] = __ldcg(src + i);
                 }
-                if (!__all_sync(0xffffffffu, got)) {
-                    if (lane == 0)
-                        raise_device_error(2u);
-                }
-                const float4 *src =
-                    reinterpret_cast<const float4 *>(a.carry + static_cast<size_t>(up.chain) * CPB * NS);
-                float4 *dst = reinterpret_cast<float4 *>(&sm.hinit[s][0][0]);
-                for (int i = lane; i < CPB * NS / 4; i += 32)
-                    dst[i] = __ldcg(src + i);
             }
             ++k;
         }
@@ -398,6 +494,7 @@ __global__ void __launch_bounds__(kScanBlock, 2)
 
     f2_t hp[NP], A2p[NP], nrAp[NP];
     float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, cb = 0.f, Dd = 0.f, bias = 0.f;
+    float sdel = 0.f;  // extended instantiation: sum of the unit's Delta (associative split)
     bool live = false;
     int chain = 0, seg = 0, bseq = 0, c0 = 0;
 #pragma unroll
@@ -409,6 +506,8 @@ __global__ void __launch_bounds__(kScanBlock, 2)
     // MUFU pipe is fed while the state arithmetic proceeds.
     f2_t ab[NP];
     auto decays = [&](float delta) {
+        if constexpr (CONSTD)
+            return;  // the decays are the constants in A2p
         const f2_t dd = f2_pack(delta, delta);
 #pragma unroll
         for (int q = 0; q < NP; ++q) {
@@ -434,13 +533,15 @@ __global__ void __launch_bounds__(kScanBlock, 2)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int q = 2 * q2 + e;
-                const f2_t abq = ab[q];
-                if (NEXT) {
+                const f2_t abq = CONSTD ? A2p[q] : ab[q];
+                if (NEXT && !CONSTD) {
                     float d0, d1;
                     f2_unpack(f2_mul(ddn, A2p[q]), d0, d1);
                     ab[q] = f2_pack(ex2_approx(d0), ex2_approx(d1));
                 }
-                if (ZOH) {
+                if (CONSTD) {
+                    hp[q] = f2_fma(abq, hp[q], f2_mul(uu, Bp[e]));
+                } else if (ZOH) {
                     const f2_t nk = f2_mul(nrAp[q], f2_mul(uu, Bp[e]));
                     hp[q] = f2_fma(abq, f2_sub(hp[q], nk), nk);
                 } else {
@@ -496,6 +597,7 @@ __global__ void __launch_bounds__(kScanBlock, 2)
             Dd = live ? a.D[ch] : 0.0f;
             bias = (live && a.dt_bias) ? a.dt_bias[ch] : 0.0f;
             const bool carry_in = (m.w & kMetaCarry) != 0;
+            sdel = 0.f;
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
                 float al[2] = {0.f, 0.f}, nr[2] = {0.f, 0.f};
@@ -503,9 +605,17 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                 for (int e = 0; e < 2; ++e) {
                     const int n = n0 + 2 * q + e;
                     if (live && n < a.N) {
-                        const float A = -expf(a.A_log[static_cast<size_t>(ch) * a.N + n]);  // A = -exp(A_log)
-                        al[e] = A * kLog2e;
-                        nr[e] = -1.0f / A;
+                        if (CONSTD) {
+                            // the constant cell: its decay 2^w, computed once per unit in
+                            // double precision and rounded once -- a decay near 1 keeps
+                            // about 1/(1 - a) tokens, and its rounding error is
+                            // multiplied by that memory length
+                            al[e] = static_cast<float>(exp2(static_cast<double>(a.A_log[static_cast<size_t>(ch) * a.N + n])));
+                        } else {
+                            const float A = -expf(a.A_log[static_cast<size_t>(ch) * a.N + n]);  // A = -exp(A_log)
+                            al[e] = A * kLog2e;
+                            nr[e] = -1.0f / A;
+                        }
                     }
                 }
                 A2p[q] = f2_pack(al[0], al[1]);
@@ -547,12 +657,22 @@ __global__ void __launch_bounds__(kScanBlock, 2)
             }
             const f2_t BIAS = f2_pack(bias, bias);
             auto silu2 = [&](f2_t v) {
-                if constexpr (sizeof(IO) == 2)
-                    return f2_silu_tanh(v);
-                else
+                // bfloat16 outputs take the tanh form; float32 outputs, and the
+                // backward's checkpoints, the exponential one
+                if constexpr (sizeof(IO) == 2) {
+                    if constexpr (CKPT)
+                        return f2_silu_fast(v);
+                    else
+                        return f2_silu_tanh(v);
+                } else {
                     return f2_silu_fast(v);
+                }
             };
-            float za = ld(zq, 0), zb = ld(zq, 2), da = ld(dq, 0), db = ld(dq, 2);
+            float za = ld(zq, 0), zb = ld(zq, 2), da = 0.f, db = 0.f;
+            if (!CONSTD) {
+                da = ld(dq, 0);
+                db = ld(dq, 2);
+            }
             float xa = CONV ? 0.f : ld(xq, 0), xb = CONV ? 0.f : ld(xq, 2);
             auto quad_scalars = [&](int p, f2_t &u2, f2_t &d2, f2_t &g2) {
                 if (CONV) {
@@ -575,14 +695,19 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                 }
                 const f2_t gz = silu2(f2_pack(za, zb));
                 g2 = a.has_z ? gz : f2_pack(1.0f, 1.0f);
-                d2 = f2_softplus_fast(f2_add(f2_pack(da, db), BIAS));
+                if constexpr (CONSTD)
+                    d2 = f2_pack(1.0f, 1.0f);  // a unit step: the segment sums count tokens
+                else
+                    d2 = f2_softplus_fast(f2_add(f2_pack(da, db), BIAS));
                 // this thread's z and dt rows of the next quad, read one quad
                 // ahead like the conv window (rows past the chunk lie in the
                 // tiles' padding)
                 za = ld(zq, p + 4);
                 zb = ld(zq, p + 6);
-                da = ld(dq, p + 4);
-                db = ld(dq, p + 6);
+                if (!CONSTD) {
+                    da = ld(dq, p + 4);
+                    db = ld(dq, p + 6);
+                }
             };
             const int base = lane & ~1;
             // publish this thread's (u, Delta) of its two tokens; read the quad's
@@ -621,6 +746,24 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                         f2_unpack(d2n, dlo, dhi);
                         dnext = __shfl_sync(0xffffffffu, dlo, base);
                     }
+                    if constexpr (CKPT) {
+                        // checkpoint mode: the state before every kCkptEvery-th token
+                        // (chunks start on multiples of it); state-only units hold
+                        // no true state
+                        if ((p % kCkptEvery) == 0 && !(m.w & kMetaNoY) && live) {
+                            const int tk = m.y + p;
+                            const int nck = (a.L + kCkptEvery - 1) / kCkptEvery;
+                            float *cp = a.ckpt + ((static_cast<size_t>(bseq) * nck + tk / kCkptEvery) * a.d +
+                                                  (c0 + cl)) * 16 + n0;
+#pragma unroll
+                            for (int qq = 0; qq < NP; qq += 2) {
+                                float v0, v1, v2, v3;
+                                f2_unpack(hp[qq], v0, v1);
+                                f2_unpack(hp[qq + 1], v2, v3);
+                                *reinterpret_cast<float4 *>(cp + 2 * qq) = make_float4(v0, v1, v2, v3);
+                            }
+                        }
+                    }
                     const float acc0 = update_pipe(bc[p], c0s.x, c0s.y, c1s.y, std::true_type{});
                     float acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
                     if (FULL || p + 1 < tc)
@@ -629,6 +772,15 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                         acc2 = update_pipe(bc[p + 2], c0s.z, c0s.w, c1s.w, std::true_type{});
                     if (FULL || p + 3 < tc)
                         acc3 = update_pipe(bc[p + 3], c1s.z, c1s.w, dnext, std::integral_constant<bool, !LAST>{});
+                    if constexpr (INIT) {
+                        sdel += c0s.y;
+                        if (FULL || p + 1 < tc)
+                            sdel += c1s.y;
+                        if (FULL || p + 2 < tc)
+                            sdel += c0s.w;
+                        if (FULL || p + 3 < tc)
+                            sdel += c1s.w;
+                    }
                     // each thread finishes its own tokens: own partial + the partner's
                     const float ra = __shfl_xor_sync(0xffffffffu, half ? acc0 : acc1, 1);
                     const float rb = __shfl_xor_sync(0xffffffffu, half ? acc2 : acc3, 1);
@@ -704,7 +856,10 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                 }
                 const f2_t gz = f2_silu_fast(f2_pack(ld(zp, pr), ld(zp, pr + 1)));
                 g2 = a.has_z ? gz : f2_pack(1.0f, 1.0f);
-                d2 = f2_softplus_fast(f2_add(f2_pack(ld(dp, pr), ld(dp, pr + 1)), BIAS));
+                if constexpr (CONSTD)
+                    d2 = f2_pack(1.0f, 1.0f);
+                else
+                    d2 = f2_softplus_fast(f2_add(f2_pack(ld(dp, pr), ld(dp, pr + 1)), BIAS));
             };
             auto run = [&](auto full_tag) {
                 constexpr bool FULL = decltype(full_tag)::value;
@@ -733,9 +888,13 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                     f2_unpack(d2n, dn0, dn1);
                     const float acc0 = update_pipe(bc[p], u0, d0, d1, std::true_type{});
                     yw[p][cw] = tr::from_f(fmaf(Dd, u0, acc0) * g0);
+                    if constexpr (INIT)
+                        sdel += d0;
                     if (FULL || p + 1 < tc) {
                         const float acc1 = update_pipe(bc[p + 1], u1, d1, dn0, std::integral_constant<bool, !LAST>{});
                         yw[p + 1][cw] = tr::from_f(fmaf(Dd, u1, acc1) * g1);
+                        if constexpr (INIT)
+                            sdel += d1;
                     }
                     u2c = u2n;
                     d2c = d2n;
@@ -764,20 +923,56 @@ __global__ void __launch_bounds__(kScanBlock, 2)
 
         if (m.w & kMetaLast) {
             const int ch = c0 + cl;
-            if (a.dynamic && seg + 1 < a.nseg) {
-                float *cp = a.carry + (static_cast<size_t>(chain) * CPB + cl) * NS + n0;
+            if (INIT && a.assoc) {
+                // associative split: a state-only unit publishes (h from zero,
+                // sum of Delta); the first segment publishes its end state
+                if ((m.w & kMetaNoY) || (seg == 0 && a.nseg > 1)) {
+                    if (m.x != a.skip_publish) {
+                        const size_t slot = static_cast<size_t>(chain) * a.nseg + seg;
+                        float *cp = a.carry + (slot * CPB + cl) * NS + n0;
 #pragma unroll
-                for (int q = 0; q < NP; q += 2) {
-                    float v0, v1, v2, v3;
-                    f2_unpack(hp[q], v0, v1);
-                    f2_unpack(hp[q + 1], v2, v3);
-                    __stcg(reinterpret_cast<float4 *>(cp + 2 * q), make_float4(v0, v1, v2, v3));
+                        for (int q = 0; q < NP; q += 2) {
+                            float v0, v1, v2, v3;
+                            f2_unpack(hp[q], v0, v1);
+                            f2_unpack(hp[q + 1], v2, v3);
+                            __stcg(reinterpret_cast<float4 *>(cp + 2 * q), make_float4(v0, v1, v2, v3));
+                        }
+                        if (sub == 0)
+                            __stcg(a.carry_sum + slot * CPB + cl, sdel);
+                        __syncwarp();
+                        if (lane == 0) {
+                            __threadfence();
+                            st_release_gpu(&a.flags[slot * kConsumerWarps + warp], 1u);
+                        }
+                    }
+                } else if (seg == a.nseg - 1 && live && a.h_final) {
+                    float *hf = a.h_final + (static_cast<size_t>(bseq) * a.d + ch) * a.N;
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        float v0, v1;
+                        f2_unpack(hp[q], v0, v1);
+                        if (n0 + 2 * q < a.N)
+                            hf[n0 + 2 * q] = v0;
+                        if (n0 + 2 * q + 1 < a.N)
+                            hf[n0 + 2 * q + 1] = v1;
+                    }
                 }
-                __syncwarp();
-                if (lane == 0) {
-                    __threadfence();
-                    st_release_gpu(&a.flags[static_cast<size_t>(chain) * kConsumerWarps + warp],
-                                   static_cast<unsigned int>(seg + 1));
+            } else if (a.dynamic && seg + 1 < a.nseg) {
+                if (m.x != a.skip_publish) {
+                    float *cp = a.carry + (static_cast<size_t>(chain) * CPB + cl) * NS + n0;
+#pragma unroll
+                    for (int q = 0; q < NP; q += 2) {
+                        float v0, v1, v2, v3;
+                        f2_unpack(hp[q], v0, v1);
+                        f2_unpack(hp[q + 1], v2, v3);
+                        __stcg(reinterpret_cast<float4 *>(cp + 2 * q), make_float4(v0, v1, v2, v3));
+                    }
+                    __syncwarp();
+                    if (lane == 0) {
+                        __threadfence();
+                        st_release_gpu(&a.flags[static_cast<size_t>(chain) * kConsumerWarps + warp],
+                                       static_cast<unsigned int>(seg + 1));
+                    }
                 }
             } else if (live && a.h_final) {
                 float *hf = a.h_final + (static_cast<size_t>(bseq) * a.d + ch) * a.N;
@@ -798,13 +993,19 @@ __global__ void __launch_bounds__(kScanBlock, 2)
         __syncwarp();
         if (lane == 0) {
             mbar_arrive(&sm.empty[s]);
-            if (c0 + warp * CPW < a.d) {  // a tile's last warps may lie past d
-                tma_store_3d(&tm_y, &sm.y[warp][c % kYBuf].v[0][0], c0 + warp * CPW, m.y, bseq);
-                bulk_commit_group();
+            if (!CKPT && !(INIT && (m.w & kMetaNoY))) {
+                if (c0 + warp * CPW < a.d) {  // a tile's last warps may lie past d
+                    tma_store_3d(&tm_y, &sm.y[warp][c % kYBuf].v[0][0], c0 + warp * CPW, m.y, bseq);
+                    bulk_commit_group();
+                }
+                // the buffer this warp writes next chunk (stored kYBuf-1 chunks
+                // ago) must have been read by its store
+                bulk_wait_group_read<kYBuf - 1>();
+            } else {
+                // no store from this chunk: drain all, so that the rotation's
+                // next buffer is free whatever the earlier chunks stored
+                bulk_wait_group_read<0>();
             }
-            // the buffer this warp writes next chunk (stored kYBuf-1 chunks
-            // ago) must have been read by its store
-            bulk_wait_group_read<kYBuf - 1>();
         }
         __syncwarp();
     }

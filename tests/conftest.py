@@ -24,3 +24,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Largest parity errors observed in the session, per quantity."""
+    try:
+        from s6_testutil import OBSERVED
+    except ImportError:  # pragma: no cover
+        return
+    if not OBSERVED:
+        return
+    terminalreporter.write_sep("-", "largest observed max|got-ref|/(1+|ref|)")
+    for k in sorted(OBSERVED):
+        terminalreporter.write_line(f"{k:40s} {OBSERVED[k]:.3e}")

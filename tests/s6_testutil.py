@@ -43,8 +43,17 @@ def rel_err(got, ref) -> float:
     return float(np.max(np.abs(got - ref) / (1.0 + np.abs(ref))))
 
 
+# largest error seen per quantity in this session (printed in the terminal summary)
+OBSERVED = {}
+
+
+def note(key, err):
+    OBSERVED[key] = max(OBSERVED.get(key, 0.0), float(err))
+
+
 def assert_close(got, ref, io, what=""):
     err = rel_err(got, ref)
+    note(f"{what} ({io})", err)
     assert np.all(np.isfinite(np.asarray(got, dtype=np.float64))), f"{what}: non-finite values"
     assert err <= TOL[io], f"{what}: max|got-ref|/(1+|ref|) = {err:.3e} > {TOL[io]:.0e}"
     return err

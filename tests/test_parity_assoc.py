@@ -1,0 +1,106 @@
+"""GPU parity of the associative split of the sequence against the float64 oracle.
+
+When a problem has too few (sequence, channel-tile) pairs to occupy the GPU --
+a single long prompt, say -- the scan cuts each sequence into segments that run
+at once: segment 0 in full, the others first from a zero state (publishing
+their end state and the sum of their step sizes), then again from the start
+state folded from those pieces with the pair combine
+(a1, b1) o (a2, b2) = (a1 a2, a2 b1 + b2).  The result must equal the plain
+recurrence.  These shapes select that schedule (at most a third as many
+(sequence, 64- or 128-channel tile) pairs as CTA slots, sequences of at least
+four chunks); y and h_final are compared element by element with the oracle.
+"""
+import numpy as np
+import pytest
+
+from oracle import s6_oracle as O
+import s6_inputs as SI
+from s6_testutil import as_f64, assert_close, dev_inputs, from_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    dict(Bt=1, L=3000, d=128, N=16, K=4),   # 2 chains, ragged last chunk
+    dict(Bt=2, L=1100, d=200, N=16, K=4),   # d not a multiple of the tile
+    dict(Bt=1, L=777, d=256, N=8, K=3),     # one thread per channel, 2 chains
+    dict(Bt=3, L=520, d=64, N=3, K=2),
+]
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+@pytest.mark.parametrize("zoh", [False, True])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_assoc_split_fused(io, zoh, shape):
+    import selective_state_space_19_b200 as S
+    import torch
+    inp = SI.scan_inputs("mamba_mini", io=io, seed=shape["L"] + shape["d"], **shape)
+    t = dev_inputs(inp)
+    y, h = S.s6_conv_scan_fwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"],
+                              z=t["z"], dt_bias=t["dt_bias"], zoh_mode=int(zoh))
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    ry, rh = O.scan(inp["x"], inp["dt"], inp["A_log"], inp["B"], inp["C"], inp["D"], z=inp["z"],
+                    dt_bias=inp["dt_bias"], zoh=zoh, conv_w=inp["conv_w"], conv_b=inp["conv_b"])
+    assert_close(as_f64(from_dev(y)), ry, io, "assoc y")
+    assert_close(h.cpu().numpy(), rh, io, "assoc h_final")
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_assoc_split_unfused_random_A(io):
+    """The unfused scan, random A_log (so nothing depends on A_log = log(n+1)),
+    no dt_bias and no gate."""
+    import selective_state_space_19_b200 as S
+    import torch
+    inp = SI.scan_inputs("mamba_mini", Bt=1, L=2500, d=192, N=16, K=4, io=io, seed=5, random_A=True)
+    t = dev_inputs(inp)
+    y, h = S.s6_scan_fwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], t["D"])
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    ry, rh = O.scan(inp["x"], inp["dt"], inp["A_log"], inp["B"], inp["C"], inp["D"])
+    assert_close(as_f64(from_dev(y)), ry, io, "assoc y")
+    assert_close(h.cpu().numpy(), rh, io, "assoc h_final")
+
+
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_assoc_split_from_state(io):
+    """Segment 0 starts from a given state and conv history; the folded start
+    states of the later segments carry it."""
+    import selective_state_space_19_b200 as S
+    import torch
+    Bt, L, d, N, K = 2, 1500, 128, 16, 4
+    inp = SI.scan_inputs("mamba_mini", Bt=Bt, L=L, d=d, N=N, K=K, io=io, seed=21)
+    rng = np.random.default_rng(22)
+    h0 = rng.standard_normal((Bt, d, N)).astype(np.float32)
+    hist = SI.to_storage(rng.standard_normal((Bt, d, K - 1)).astype(np.float32), io)
+    t = dev_inputs(inp)
+    y, h = S.s6_conv_scan_fwd_from_state(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"],
+                                         t["D"], z=t["z"], dt_bias=t["dt_bias"], zoh_mode=1, h_init=to_dev(h0),
+                                         conv_hist=to_dev(hist))
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    ry, rh = O.scan(inp["x"], inp["dt"], inp["A_log"], inp["B"], inp["C"], inp["D"], z=inp["z"],
+                    dt_bias=inp["dt_bias"], zoh=True, conv_w=inp["conv_w"], conv_b=inp["conv_b"], h_init=h0,
+                    conv_hist=hist)
+    assert_close(as_f64(from_dev(y)), ry, io, "assoc y")
+    assert_close(h.cpu().numpy(), rh, io, "assoc h_final")
+
+
+def test_assoc_split_long_single_sequence_sampled():
+    """One long prompt at the long-sequence workload's width: Bt1 L16384 d1536
+    bf16 (24 chains), sampled channels over the whole sequence."""
+    import selective_state_space_19_b200 as S
+    import torch
+    inp = SI.scan_inputs("long_seq", Bt=1, L=16384, seed=44)
+    t = dev_inputs(inp)
+    y, h = S.s6_conv_scan_fwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"],
+                              z=t["z"], dt_bias=t["dt_bias"])
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    rng = np.random.default_rng(3)
+    ch = np.stack([np.zeros(40, np.int64), np.concatenate([[0, 63, 64, 1535], rng.integers(0, 1536, 36)])], axis=1)
+    ry, rh = O.scan(inp["x"], inp["dt"], inp["A_log"], inp["B"], inp["C"], inp["D"], z=inp["z"],
+                    dt_bias=inp["dt_bias"], conv_w=inp["conv_w"], conv_b=inp["conv_b"], channels=ch)
+    yg = as_f64(from_dev(y))
+    hg = h.cpu().numpy()
+    assert_close(np.stack([yg[b, :, c] for b, c in ch]), ry, "bf16", "assoc y")
+    assert_close(np.stack([hg[b, c] for b, c in ch]), rh, "bf16", "assoc h_final")

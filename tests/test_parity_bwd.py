@@ -16,7 +16,7 @@ import pytest
 
 from oracle import s6_oracle as O
 import s6_inputs as SI
-from s6_testutil import as_f64, dev_inputs, from_dev, rel_err, to_dev
+from s6_testutil import as_f64, dev_inputs, from_dev, note, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +42,7 @@ def _case(io, zoh, gate, with_h, Bt, L, d, N, seed):
     for k in keys:
         g = got[k].cpu().numpy().astype(np.float64)
         err = rel_err(g, ref[k])
+        note(f"grad {k} ({io})", err)
         assert np.all(np.isfinite(g)), k
         assert err <= GTOL, f"{k}: max|g-ref|/(1+|ref|) = {err:.3e} (io={io}, zoh={zoh}, gate={gate})"
     if not gate:
@@ -92,4 +93,66 @@ def test_fused_bwd_matches_oracle(io, zoh, shape):
         g = got[k].cpu().numpy().astype(np.float64)
         assert np.all(np.isfinite(g)), k
         err = rel_err(g, ref[k])
+        note(f"grad fused {k} ({io})", err)
         assert err <= GTOL, f"{k}: max|g-ref|/(1+|ref|) = {err:.3e} (io={io}, zoh={zoh}, {shape})"
+
+
+# ------------------------------------------------ the pipelined path (N = 16)
+# At N = 16 with rows the tensor unit can move, the backward runs the forward
+# kernel with state checkpoints, the reverse kernel over (segment, chain)
+# units, and a reduction of the per-tile dB / dC rows.  These shapes cut the
+# chains into segments (dLoss/dh and the conv's dpre window handed from one
+# segment to the one before it) and take the associative split in the
+# checkpointing forward.
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("zoh", [False, True])
+def test_bwd_segmented_chains(io, zoh):
+    _case(io, zoh, True, with_h=True, Bt=1, L=2000, d=128, N=16, seed=91)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("zoh", [False, True])
+def test_fused_bwd_segmented_chains(io, zoh):
+    import torch
+    import selective_state_space_19_b200 as S
+    Bt, L, d, N, K = 2, 1500, 64, 16, 4
+    inp = SI.scan_inputs("mamba_mini", Bt=Bt, L=L, d=d, N=N, K=K, io=io, seed=92)
+    rng = np.random.default_rng(93)
+    dy = SI.to_storage(rng.standard_normal((Bt, L, d)).astype(np.float32), io)
+    ref = O.conv_scan_bwd(inp["x"], inp["conv_w"], inp["conv_b"], inp["dt"], inp["A_log"], inp["B"], inp["C"],
+                          inp["D"], dy, z=inp["z"], dt_bias=inp["dt_bias"], zoh=zoh)
+    t = dev_inputs(inp)
+    got = S.s6_conv_scan_bwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"],
+                             to_dev(dy), z=t["z"], dt_bias=t["dt_bias"], zoh_mode=int(zoh), want_dh_init=True)
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    for k in ("dx", "dconv_w", "dconv_b", "ddt", "dz", "dB", "dC", "dA_log", "dD", "ddt_bias", "dh_init"):
+        g = got[k].cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(g)), k
+        err = rel_err(g, ref[k])
+        note(f"grad fused {k} ({io})", err)
+        assert err <= GTOL, f"{k}: max|g-ref|/(1+|ref|) = {err:.3e} (io={io}, zoh={zoh})"
+
+
+def test_bwd_unaligned_rows_take_the_simple_kernel():
+    """Rows that are not 16-byte aligned (an offset view) take the plain
+    backward kernel; the gradients still match the oracle."""
+    import torch
+    import selective_state_space_19_b200 as S
+    Bt, L, d, N = 2, 90, 64, 16
+    inp = SI.scan_inputs("mamba_mini", Bt=Bt, L=L, d=d, N=N, io="f32", seed=94)
+    rng = np.random.default_rng(95)
+    dy = rng.standard_normal((Bt, L, d)).astype(np.float32)
+    ref = O.scan_bwd(inp["x"], inp["dt"], inp["A_log"], inp["B"], inp["C"], inp["D"], dy, z=inp["z"],
+                     dt_bias=inp["dt_bias"])
+    t = dev_inputs(inp)
+    buf = torch.empty(Bt * L * d + 1, device="cuda")
+    u_off = buf[1:].view(Bt, L, d)  # 4 bytes past a 16-byte boundary
+    u_off.copy_(t["x"])
+    got = S.s6_scan_bwd(u_off, t["dt"], t["A_log"], t["B"], t["C"], t["D"], to_dev(dy), z=t["z"],
+                        dt_bias=t["dt_bias"])
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    for k in ("du", "ddt", "dz", "dB", "dC", "dA_log", "dD", "ddt_bias"):
+        err = rel_err(got[k].cpu().numpy().astype(np.float64), ref[k])
+        assert err <= GTOL, f"{k}: {err:.3e}"

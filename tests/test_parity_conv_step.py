@@ -7,7 +7,7 @@ import pytest
 
 from oracle import s6_oracle as O
 import s6_inputs as SI
-from s6_testutil import as_f64, assert_close, dev_inputs, from_dev, to_dev
+from s6_testutil import as_f64, assert_close, dev_inputs, from_dev, sample_channels, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -50,8 +50,9 @@ def _step_gpu(S, t, tok, h, cs, zoh):
 @pytest.mark.parametrize("cfg", [dict(Bt=1, L=6, d=8, N=3, K=3), dict(Bt=4, L=40, d=200, N=16, K=4),
                                  dict(Bt=3, L=25, d=72, N=5, K=2), dict(Bt=2, L=30, d=64, N=8, K=4)])
 def test_streaming_equals_full_forward(io, zoh, cfg):
-    """'Token streaming ... matches the full forward': L single-token steps on the
-    GPU reproduce the oracle's full-sequence outputs and final state."""
+    """The streaming check of "Carry context through a selective state" (Verified
+    by the local recipe): L single-token steps on the GPU reproduce the oracle's
+    full-sequence outputs and final state."""
     import selective_state_space_19_b200 as S
     import torch
     inp = SI.scan_inputs("mamba_mini", io=io, seed=31 + cfg["L"], **cfg)
@@ -182,6 +183,42 @@ def test_decode_workload_sampled():
         assert_close(np.stack([y[b, :, dd] for b, dd in ch]), ry, "f32", "y")
         hg = h.cpu().numpy()
         assert_close(np.stack([hg[b, dd] for b, dd in ch]), rh, "f32", "h_ssm")
+
+
+def test_decode_workload_full_length():
+    """The streaming-decode workload at its stated length: 1024 single-token steps
+    through each of the 6 blocks (d1536, N16, K4, float32 state), on a stated
+    subset of 16 sequences (the workload's per-(step, block) seeding with a
+    16-sequence batch), against the oracle's scan of the same token sequence:
+    y at every step on 96 sampled channels per block, the final h_ssm on those
+    channels, and the final conv history of every channel (exact)."""
+    import selective_state_space_19_b200 as S
+    import torch
+    Bt, d, N, K, steps, blocks = 16, 1536, 16, 4, 1024, 6
+    ch = sample_channels(Bt, d, 92, seed=9)
+    for block in range(blocks):
+        p = SI.decode_params(block)
+        pt = {k: to_dev(v) for k, v in p.items()}
+        toks = [SI.decode_tokens(s, block, Bt=Bt) for s in range(steps)]
+        seq = {k: np.stack([tok[k] for tok in toks], axis=0) for k in ("x", "dt", "z", "B", "C")}  # [steps, Bt, .]
+        td = {k: to_dev(v) for k, v in seq.items()}
+        h = torch.zeros(Bt, d, N, device="cuda")
+        cs = torch.zeros(Bt, d, K - 1, device="cuda")
+        ys = torch.empty(steps, Bt, d, device="cuda")
+        for s in range(steps):
+            S.s6_step(td["x"][s], td["dt"][s], td["B"][s], td["C"][s], pt["A_log"], pt["D"], pt["conv_w"], h, cs,
+                      z_t=td["z"][s], dt_bias=pt["dt_bias"], conv_b=pt["conv_b"], y_t=ys[s])
+        torch.cuda.synchronize()
+        assert S.s6_device_status() == 0
+        ref_in = {k: np.ascontiguousarray(np.transpose(v, (1, 0, 2))) for k, v in seq.items()}  # [Bt, steps, .]
+        ry, rh = O.scan(ref_in["x"], ref_in["dt"], p["A_log"], ref_in["B"], ref_in["C"], p["D"], z=ref_in["z"],
+                        dt_bias=p["dt_bias"], conv_w=p["conv_w"], conv_b=p["conv_b"], channels=ch)
+        y = ys.cpu().numpy()  # [steps, Bt, d]
+        assert_close(np.stack([y[:, b, dd] for b, dd in ch]), ry, "f32", "decode 1024-step y")
+        hg = h.cpu().numpy()
+        assert_close(np.stack([hg[b, dd] for b, dd in ch]), rh, "f32", "decode 1024-step h_ssm")
+        # the history holds the last K-1 inputs exactly, oldest first
+        np.testing.assert_array_equal(cs.cpu().numpy(), np.transpose(seq["x"][-(K - 1):], (1, 2, 0)))
 
 
 def test_step_rejects_bad_arguments():

@@ -6,14 +6,16 @@ plan, so a library call must not cudaMalloc on their behalf.  The no-allocation
 entry point keeps its segment carries in a fixed array inside the library.
 These tests call it through the C ABI on shapes that do need the carries, twice
 in a row on the same device (the array keeps the previous call's contents), and
-compare with s6_conv_scan_fwd within the parity tolerance.  The file is
+compare with s6_conv_scan_fwd within the parity tolerance, and with the float64
+oracle on sampled channels.  The file is
 collected last and also passes when run alone in a fresh process.
 """
 import numpy as np
 import pytest
 
+from oracle import s6_oracle as O
 import s6_inputs as SI
-from s6_testutil import TOL, as_f64, assert_close, dev_inputs, from_dev
+from s6_testutil import TOL, as_f64, assert_close, dev_inputs, from_dev, sample_channels
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +44,13 @@ def test_noalloc_matches_allocating_entry_point_twice(io, zoh):
         assert S.s6_device_status() == 0
         assert_close(as_f64(from_dev(y)), as_f64(from_dev(y_ref)), io, "y")
         assert_close(h.cpu().numpy(), h_ref.cpu().numpy(), io, "h_final")
+    # and, standing on its own, against the float64 oracle on sampled channels
+    ch = sample_channels(2, 256, 30, seed=76)
+    ry, rh = O.scan(inp["x"], inp["dt"], inp["A_log"], inp["B"], inp["C"], inp["D"], z=inp["z"],
+                    dt_bias=inp["dt_bias"], zoh=zoh, conv_w=inp["conv_w"], conv_b=inp["conv_b"], channels=ch)
+    yg, hg = as_f64(from_dev(y)), h.cpu().numpy()
+    assert_close(np.stack([yg[b, :, c] for b, c in ch]), ry, io, "noalloc y vs oracle")
+    assert_close(np.stack([hg[b, c] for b, c in ch]), rh, io, "noalloc h_final vs oracle")
 
 
 def test_noalloc_other_shape_after_a_larger_one():
