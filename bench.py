@@ -784,14 +784,46 @@ def run_ours(args):
     return 0
 
 
+def run_profile_case(case):
+    """Small fixed cases for ncu captures of kernels outside the timed step:
+    'bwd' -- three s6_scan_bwd calls on the long_seq recipe at Bt16 L1024 (the
+    full workload's 384 chains, ~0.65 GB on the device); 'block' -- three decode
+    token steps of 256 sequences through the 6 Mamba-mini blocks."""
+    import torch
+    import selective_state_space_19_b200 as S
+    dev = torch.device("cuda", 0)
+    if case == "bwd":
+        inp = SI.scan_inputs("long_seq", Bt=16, L=1024, seed=3)
+        t = {k: to_dev(inp[k], dev) for k in ("x", "z", "B", "C", "dt", "A_log", "D", "dt_bias")}
+        gen = torch.Generator(device=dev).manual_seed(7)
+        dy = torch.randn(16, 1024, 1536, device=dev, generator=gen).to(torch.bfloat16)
+        for _ in range(3):
+            S.s6_scan_bwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], t["D"], dy, z=t["z"], dt_bias=t["dt_bias"])
+    else:
+        cfgb = SI.MAMBA_MINI_BLOCK
+        ws = [{k: to_dev(np.ascontiguousarray(v), dev) for k, v in SI.block_weights(b).items()}
+              for b in range(cfgb["blocks"])]
+        cs = [torch.zeros(256, cfgb["di"], cfgb["K"] - 1, device=dev) for _ in ws]
+        hs = [torch.zeros(256, cfgb["di"], cfgb["N"], device=dev) for _ in ws]
+        x = to_dev(SI.block_tokens(0), dev)
+        for _ in range(3):
+            for b, w in enumerate(ws):
+                S.s6_block_step(x, cs[b], hs[b], w, eps=cfgb["eps"])
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    print(f"profile case {case}: ok", flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["full", "small"], default="full",
-                    help="small: the workload at L=2048 (for ncu captures)")
+    ap.add_argument("--case", choices=["full", "small", "bwd", "block"], default="full",
+                    help="small: the workload at L=2048 (for ncu captures); bwd, block: small cases of the "
+                         "backward and the decode block for captures (no JSON line)")
     ap.add_argument("--no-rows", action="store_true", help="skip the decode-step and standalone-conv rows")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -799,6 +831,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.case in ("bwd", "block"):
+        return run_profile_case(args.case)
     return run_ours(args)
 
 

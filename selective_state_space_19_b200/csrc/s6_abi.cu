@@ -1162,121 +1162,127 @@ int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (use_stream_device(s) != S6_OK)
         return S6_ERR_CUDA;
-    // intermediate rows: xin | z, the x_proj rows (dt | B | C), the gated readout
+    // intermediate rows: LayerNorm(x), xin | z, SiLU(conv(xin)), the x_proj rows
+    // (dt | B | C), the gated readout -- each region a multiple of 4 floats
     const int64_t row = R + 2 * N;
+    const size_t l_hn = round_up(static_cast<size_t>(dm), 4), l_xz = round_up(static_cast<size_t>(2 * di), 4),
+                 l_xc = round_up(static_cast<size_t>(di), 4), l_dbc = round_up(static_cast<size_t>(row), 4);
     void *scr = nullptr;
-    const size_t fl = static_cast<size_t>(Bt) * (2 * di + round_up(static_cast<size_t>(row), 4) + di);
+    const size_t fl = static_cast<size_t>(Bt) * (l_hn + l_xz + l_xc + l_dbc + l_xc);
     int rc = get_scratch(fl * sizeof(float), s, &scr, kScratchBlock);
     if (rc != S6_OK)
         return rc;
-    float *xz = static_cast<float *>(scr);
-    float *dbc = xz + static_cast<size_t>(Bt) * 2 * di;
-    float *g = dbc + static_cast<size_t>(Bt) * round_up(static_cast<size_t>(row), 4);
+    float *hn = static_cast<float *>(scr);
+    float *xz = hn + static_cast<size_t>(Bt) * l_hn;
+    float *xc = xz + static_cast<size_t>(Bt) * l_xz;
+    float *dbc = xc + static_cast<size_t>(Bt) * l_xc;
+    float *g = dbc + static_cast<size_t>(Bt) * l_dbc;
     const int64_t sms = device_sm_count();
     const unsigned mt = static_cast<unsigned>((Bt + s6::kGemmBM - 1) / s6::kGemmBM);
-    auto splits_for = [&](int64_t n_out, int64_t k) {
-        // enough reduction slices to put about two blocks on every SM
+    // a product Y = X W^T over the whole batch; the reduction is split across
+    // blocks (atomic adds into Y) until there are about two blocks per SM
+    auto gemm = [&](const float *X, int ldx, int64_t n_out, int64_t k, const int8_t *wq, const float *ws, float *Y,
+                    int ldy, bool add) -> int {
         const int64_t tiles = ((n_out + s6::kGemmBN - 1) / s6::kGemmBN) * mt;
-        int64_t sp = (2 * sms + tiles - 1) / tiles;
+        int64_t sp = add ? (2 * sms + tiles - 1) / tiles : 1;
         const int64_t max_sp = (k + s6::kGemmBK - 1) / s6::kGemmBK;
         if (sp > max_sp)
             sp = max_sp;
         if (sp < 1)
             sp = 1;
         const int64_t ks = round_up(static_cast<size_t>((k + sp - 1) / sp), s6::kGemmBK);
-        return std::make_pair(static_cast<int>((k + ks - 1) / ks), static_cast<int>(ks));
+        s6::Q8GemmArgs ga;
+        ga.M = static_cast<int>(Bt);
+        ga.N = static_cast<int>(n_out);
+        ga.K = static_cast<int>(k);
+        ga.x = X;
+        ga.ldx = ldx;
+        ga.wq = wq;
+        ga.ws = ws;
+        ga.y = Y;
+        ga.ldy = ldy;
+        ga.accumulate = add ? 1 : 0;
+        ga.k_split = static_cast<int>(ks);
+        const dim3 grid(static_cast<unsigned>((n_out + s6::kGemmBN - 1) / s6::kGemmBN), mt,
+                        static_cast<unsigned>((k + ks - 1) / ks));
+        const bool vec = ldx % 4 == 0 && k % 8 == 0 && aligned16(X) && aligned_to(wq, 8);
+        static int opted[64][2] = {};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            return S6_ERR_CUDA;
+        if (!opted[dev][vec]) {
+            const cudaError_t e =
+                vec ? cudaFuncSetAttribute(s6::q8_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(s6::kGemmSmem))
+                    : cudaFuncSetAttribute(s6::q8_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(s6::kGemmSmem));
+            if (e != cudaSuccess)
+                return S6_ERR_CUDA;
+            opted[dev][vec] = 1;
+        }
+        if (vec)
+            s6::q8_gemm_kernel<true><<<grid, s6::kGemmThreads, s6::kGemmSmem, s>>>(ga);
+        else
+            s6::q8_gemm_kernel<false><<<grid, s6::kGemmThreads, s6::kGemmSmem, s>>>(ga);
+        return cudaGetLastError() == cudaSuccess ? S6_OK : S6_ERR_CUDA;
     };
-    // 1. LayerNorm + in_proj -> xin | z
-    s6::Q8GemmArgs g1;
-    std::memset(&g1, 0, sizeof(g1));
-    g1.M = static_cast<int>(Bt);
-    g1.N = static_cast<int>(2 * di);
-    g1.K = static_cast<int>(dm);
-    g1.x = x;
-    g1.ldx = static_cast<int>(dm);
-    g1.wq = w->in_q;
-    g1.ws = w->in_s;
-    g1.y = xz;
-    g1.ldy = static_cast<int>(2 * di);
-    g1.k_split = static_cast<int>(dm);
-    g1.ln_w = w->ln_w;
-    g1.ln_b = w->ln_b;
-    g1.eps = dims->eps;
-    s6::q8_gemm_kernel<s6::kProLN><<<dim3(static_cast<unsigned>((2 * di + s6::kGemmBN - 1) / s6::kGemmBN), mt, 1),
-                                     s6::kGemmThreads, 0, s>>>(g1);
+    // 1. LayerNorm, then in_proj -> xin | z
+    s6::block_layernorm_kernel<<<static_cast<unsigned>((Bt + 7) / 8), s6::kLnThreads, 0, s>>>(
+        x, w->ln_w, w->ln_b, hn, static_cast<int>(Bt), static_cast<int>(dm), dims->eps);
     if (cudaGetLastError() != cudaSuccess)
         return S6_ERR_CUDA;
-    // 2. conv + SiLU + x_proj -> dt | B | C (split over the channels, summed atomically)
-    if (cudaMemsetAsync(dbc, 0, sizeof(float) * Bt * round_up(static_cast<size_t>(row), 4), s) != cudaSuccess)
-        return S6_ERR_CUDA;
-    const auto sp2 = splits_for(row, di);
-    s6::Q8GemmArgs g2;
-    std::memset(&g2, 0, sizeof(g2));
-    g2.M = static_cast<int>(Bt);
-    g2.N = static_cast<int>(row);
-    g2.K = static_cast<int>(di);
-    g2.x = xz;
-    g2.ldx = static_cast<int>(2 * di);
-    g2.wq = w->xp_q;
-    g2.ws = w->xp_s;
-    g2.y = dbc;
-    g2.ldy = static_cast<int>(round_up(static_cast<size_t>(row), 4));
-    g2.accumulate = 1;
-    g2.k_split = sp2.second;
-    g2.hist = conv_state;
-    g2.conv_w = w->conv_w;
-    g2.conv_b = w->conv_b;
-    g2.Kc = static_cast<int>(K);
-    s6::q8_gemm_kernel<s6::kProConv><<<dim3(static_cast<unsigned>((row + s6::kGemmBN - 1) / s6::kGemmBN), mt,
-                                            static_cast<unsigned>(sp2.first)),
-                                       s6::kGemmThreads, 0, s>>>(g2);
-    if (cudaGetLastError() != cudaSuccess)
-        return S6_ERR_CUDA;
+    rc = gemm(hn, static_cast<int>(dm), 2 * di, dm, w->in_q, w->in_s, xz, static_cast<int>(l_xz), false);
+    if (rc != S6_OK)
+        return rc;
+    // 2. conv + SiLU (history shifted) and x_proj -> dt | B | C, a block per sequence
+    {
+        const size_t smem = sizeof(float) * di;
+        if (smem > 48 * 1024) {
+            static int opted[64] = {};
+            int dev = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+                return S6_ERR_CUDA;
+            if (opted[dev] < static_cast<int>(smem)) {
+                if (smem > 227 * 1024 || cudaFuncSetAttribute(s6::block_conv_xproj_kernel,
+                                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                              static_cast<int>(smem)) != cudaSuccess)
+                    return S6_ERR_UNSUPPORTED;
+                opted[dev] = static_cast<int>(smem);
+            }
+        }
+        s6::block_conv_xproj_kernel<<<static_cast<unsigned>(Bt), s6::kConvXThreads, smem, s>>>(
+            xz, static_cast<int>(l_xz), w->conv_w, w->conv_b, conv_state, xc, static_cast<int>(l_xc), w->xp_q,
+            w->xp_s, dbc, static_cast<int>(l_dbc), static_cast<int>(di), static_cast<int>(K), static_cast<int>(row));
+        if (cudaGetLastError() != cudaSuccess)
+            return S6_ERR_CUDA;
+    }
     // 3. dt_proj + the recurrence + readout + gate
     s6::BlockSsmArgs a3;
     a3.Bt = static_cast<int>(Bt);
     a3.di = static_cast<int>(di);
     a3.N = static_cast<int>(N);
     a3.R = static_cast<int>(R);
-    a3.Kc = static_cast<int>(K);
     a3.xz = xz;
+    a3.xc = xc;
+    a3.xz_ld = static_cast<int>(l_xz);
+    a3.xc_ld = static_cast<int>(l_xc);
+    a3.g_ld = static_cast<int>(l_xc);
     a3.dbc = dbc;
+    a3.dbc_ld = static_cast<int>(l_dbc);
     a3.dt_q = w->dt_q;
     a3.dt_s = w->dt_s;
     a3.dt_bias = w->dt_bias;
     a3.A_log = w->A_log;
     a3.D = w->D;
-    a3.conv_w = w->conv_w;
-    a3.conv_b = w->conv_b;
-    a3.hist = conv_state;
     a3.h = h_ssm;
     a3.g = g;
-    // the x_proj rows were written with a padded stride
-    a3.dbc_ld = static_cast<int>(round_up(static_cast<size_t>(row), 4));
     s6::block_ssm_kernel<16><<<dim3(static_cast<unsigned>((di + s6::kSsmThreads - 1) / s6::kSsmThreads),
                                     static_cast<unsigned>(Bt)),
                                s6::kSsmThreads, sizeof(float) * row, s>>>(a3);
     if (cudaGetLastError() != cudaSuccess)
         return S6_ERR_CUDA;
     // 4. out_proj, added into the residual stream
-    const auto sp4 = splits_for(dm, di);
-    s6::Q8GemmArgs g4;
-    std::memset(&g4, 0, sizeof(g4));
-    g4.M = static_cast<int>(Bt);
-    g4.N = static_cast<int>(dm);
-    g4.K = static_cast<int>(di);
-    g4.x = g;
-    g4.ldx = static_cast<int>(di);
-    g4.wq = w->out_q;
-    g4.ws = w->out_s;
-    g4.y = x;
-    g4.ldy = static_cast<int>(dm);
-    g4.accumulate = 1;
-    g4.k_split = sp4.second;
-    s6::q8_gemm_kernel<s6::kProPlain><<<dim3(static_cast<unsigned>((dm + s6::kGemmBN - 1) / s6::kGemmBN), mt,
-                                             static_cast<unsigned>(sp4.first)),
-                                        s6::kGemmThreads, 0, s>>>(g4);
-    return launch_status(cudaGetLastError());
+    return gemm(g, static_cast<int>(l_xc), dm, di, w->out_q, w->out_s, x, static_cast<int>(dm), true);
 }
 
 // Read and clear the device-side error word after the stream's work so far

@@ -11,148 +11,268 @@
 //     h       = 2^(Delta A log2 e) h + (Delta B) xc,   y = <h, C> + D xc
 //     x      += out_proj(y SiLU(z))              di -> dm
 //
-// Four kernels: (1) LayerNorm fused into the in_proj product, (2) the conv +
-// SiLU fused into the x_proj product (K split across blocks, partial sums
-// added atomically), (3) dt_proj fused with the recurrence, one thread per
-// (sequence, channel) with its N states, and (4) out_proj with the residual
-// add (K split, atomic adds into x).  The products are float32 on the CUDA
-// cores: the int8 weights are converted exactly when a tile is staged in
-// shared memory and the row scale is applied to the finished sum.
+// Kernels: LayerNorm (a warp per row); the in_proj product; the conv + SiLU
+// with the history shifted in place; the x_proj product; dt_proj fused with the
+// recurrence and the gate (a thread per (sequence, channel)); the out_proj
+// product added into x.  The products (q8_gemm_kernel) are float32 on the CUDA
+// cores: int8 weight rows converted exactly when staged in shared memory, the
+// row scale applied to the finished sum, the reduction split across blocks
+// with atomic adds where the output tile count alone would not fill the GPU.
 #pragma once
 
 #include "s6_common.cuh"
 
 namespace s6 {
 
+__device__ __forceinline__ float silu_exact(float v) { return v / (1.0f + __expf(-v)); }
+
+// ------------------------------------------------------------ LayerNorm
+constexpr int kLnThreads = 256;  // 8 rows per block, a warp per row
+
+// out[m] = (x[m] - mean) / sqrt(var + eps) * w + b (biased variance)
+__global__ void __launch_bounds__(kLnThreads) block_layernorm_kernel(const float *x, const float *w, const float *b,
+                                                                     float *out, int M, int K, float eps) {
+    const int m = blockIdx.x * (kLnThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (m >= M)
+        return;
+    const float *xr = x + static_cast<size_t>(m) * K;
+    float s = 0.f;
+    for (int k = lane; k < K; k += 32)
+        s += xr[k];
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / K;
+    float v = 0.f;
+    for (int k = lane; k < K; k += 32) {
+        const float d = xr[k] - mean;
+        v = fmaf(d, d, v);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    const float r = rsqrtf(v / K + eps);
+    float *orow = out + static_cast<size_t>(m) * K;
+    for (int k = lane; k < K; k += 32)
+        orow[k] = fmaf((xr[k] - mean) * r, w[k], b[k]);
+}
+
+// ------------------------------------------------------------ conv + x_proj
+constexpr int kConvXThreads = 256;
+
+// One block per sequence m: xc[c] = SiLU(conv_b + sum_{j<K-1} w[j] hist[j] +
+// w[K-1] xin[c]) for every channel (the history drops its oldest input and
+// appends xin), kept in shared memory and written out; then the x_proj rows
+// dbc[m][o] = xp_s[o] * sum_c xp_q[o][c] xc[c], a warp per output row.
+__global__ void __launch_bounds__(kConvXThreads) block_conv_xproj_kernel(
+    const float *xz, int ldxz, const float *conv_w, const float *conv_b, float *hist, float *xc, int ldxc,
+    const int8_t *xp_q, const float *xp_s, float *dbc, int ld_dbc, int di, int Kc, int n_out) {
+    extern __shared__ __align__(16) float xcs[];  // di floats
+    const int m = blockIdx.x;
+    for (int c = threadIdx.x; c < di; c += kConvXThreads) {
+        const float xin = xz[static_cast<size_t>(m) * ldxz + c];
+        float *hs = hist + (static_cast<size_t>(m) * di + c) * (Kc - 1);
+        const float *w = conv_w + static_cast<size_t>(c) * Kc;
+        float pre = conv_b ? conv_b[c] : 0.f;
+        float hv[3] = {0.f, 0.f, 0.f};
+        for (int j = 0; j < Kc - 1; ++j) {
+            hv[j] = hs[j];
+            pre = fmaf(w[j], hv[j], pre);
+        }
+        pre = fmaf(w[Kc - 1], xin, pre);
+        for (int j = 0; j + 1 < Kc - 1; ++j)
+            hs[j] = hv[j + 1];
+        hs[Kc - 2] = xin;
+        const float v = silu_exact(pre);
+        xcs[c] = v;
+        xc[static_cast<size_t>(m) * ldxc + c] = v;
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool vec = (di % 4) == 0 && (reinterpret_cast<uintptr_t>(xp_q) & 3) == 0;
+    for (int o = warp; o < n_out; o += kConvXThreads / 32) {
+        const int8_t *q = xp_q + static_cast<size_t>(o) * di;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (vec) {
+            // four channels per lane step: one 4-byte weight load, one float4 of xc
+            const int *qw = reinterpret_cast<const int *>(q);
+            const float4 *x4 = reinterpret_cast<const float4 *>(xcs);
+#pragma unroll 4
+            for (int c4 = lane; c4 < di / 4; c4 += 32) {
+                const int wv = qw[c4];
+                const float4 xv = x4[c4];
+                acc[0] = fmaf(static_cast<float>(static_cast<int8_t>(wv & 0xff)), xv.x, acc[0]);
+                acc[1] = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 8) & 0xff)), xv.y, acc[1]);
+                acc[2] = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 16) & 0xff)), xv.z, acc[2]);
+                acc[3] = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 24) & 0xff)), xv.w, acc[3]);
+            }
+        } else {
+#pragma unroll 4
+            for (int c = lane; c < di; c += 32)
+                acc[c & 3] = fmaf(static_cast<float>(q[c]), xcs[c], acc[c & 3]);
+        }
+        float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane == 0)
+            dbc[static_cast<size_t>(m) * ld_dbc + o] = sum * xp_s[o];
+    }
+}
+
+// ------------------------------------------------------------ int8 products
 constexpr int kGemmBM = 64;  // rows (sequences) per block tile
 constexpr int kGemmBN = 64;  // outputs per block tile
 constexpr int kGemmBK = 32;  // reduction slice staged per step
 constexpr int kGemmThreads = 256;
-constexpr int kProPlain = 0;  // X read as is
-constexpr int kProLN = 1;     // X = LayerNorm of the rows
-constexpr int kProConv = 2;   // X = SiLU(conv(history, xin)) per (row, channel)
 
 struct Q8GemmArgs {
     int M, N, K;
-    const float *x;  // [M][ldx]: the rows (the pre-conv xin rows for kProConv)
+    const float *x;  // [M][ldx]
     int ldx;
     const int8_t *wq;  // [N][K] int8 rows
     const float *ws;   // [N] row scales
     float *y;          // [M][ldy]
     int ldy;
-    int accumulate;  // 1: y += (atomic adds, for split K), 0: y =
-    int k_split;     // reduction length per blockIdx.z
-    const float *ln_w, *ln_b;  // kProLN: [K]
-    float eps;
-    const float *hist;    // kProConv: [M][K][Kc-1] conv history, oldest first
-    const float *conv_w;  // kProConv: [K][Kc]
-    const float *conv_b;  // kProConv: [K] or null
-    int Kc;
+    int accumulate;  // 1: y += (atomic adds, for a split reduction), 0: y =
+    int k_split;     // reduction length per blockIdx.z (a multiple of kGemmBK)
 };
 
-__device__ __forceinline__ float silu_exact(float v) { return v / (1.0f + __expf(-v)); }
+// dynamic shared memory of q8_gemm_kernel: two slices of X and of W
+constexpr size_t kGemmSmem = 2 * (kGemmBM + kGemmBN) * (kGemmBK + 4) * sizeof(float);
 
 // Y[m][n] (+)= ws[n] * sum_k wq[n][k] X[m][k].  A 64 x 64 output tile per
-// block, 4 x 4 outputs per thread, 32-wide slices of K staged in shared memory
-// (X transposed to [k][m], the int8 weights converted to float [k][n]).
-template <int PRO>
+// block; thread (tm, tn) owns rows tm + 16 i and outputs tn + 16 j (i, j < 4),
+// so that the 128-bit shared-memory reads of a quarter warp hit distinct banks.
+// 32-wide K slices are staged row-major with a 4-float pad, the next slice
+// read into registers while the current one is multiplied.  VEC: every X row
+// start is 16-byte aligned and every W row 8-byte aligned (ldx % 4 == 0,
+// K % 8 == 0, aligned bases), so slices move as float4 / 8-byte vectors.
+template <bool VEC>
 __global__ void __launch_bounds__(kGemmThreads) q8_gemm_kernel(const Q8GemmArgs a) {
-    constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;
-    __shared__ __align__(16) float Xs[BK][BM + 4];
-    __shared__ __align__(16) float Ws[BK][BN + 4];
-    __shared__ float2 stats[BM];  // kProLN: (mean, 1/sqrt(var + eps)) of each row
+    constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK, LD = BK + 4;
+    extern __shared__ __align__(16) float gemm_smem[];
+    float(*Xs)[BM][LD] = reinterpret_cast<float(*)[BM][LD]>(gemm_smem);             // [2][BM][LD]
+    float(*Ws)[BN][LD] = reinterpret_cast<float(*)[BN][LD]>(gemm_smem + 2 * BM * LD);  // [2][BN][LD]
     const int tid = threadIdx.x;
     const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
     const int kb = blockIdx.z * a.k_split;
     const int ke = min(a.K, kb + a.k_split);
     const int tm = tid >> 4, tn = tid & 15;
-
-    if (PRO == kProLN) {
-        // row statistics over the whole row (this kernel is launched unsplit)
-        const int warp = tid >> 5, lane = tid & 31;
-        for (int r = warp; r < BM; r += kGemmThreads / 32) {
-            const int m = m0 + r;
-            float s = 0.f;
-            if (m < a.M)
-                for (int k = lane; k < a.K; k += 32)
-                    s += a.x[static_cast<size_t>(m) * a.ldx + k];
+    // staging: each thread moves 8 consecutive k of one X row and of one W row
+    constexpr int G = BK / 32;                   // groups of 8 per thread
+    const int lr = tid >> 2;                     // row within the tile (0..63)
+    const int lk = (tid & 3) * (8 * G);          // first k of its 8 G
+    float xr[8 * G], wr[8 * G];
+    auto fetch = [&](int k0) {
+        const int m = m0 + lr, n = n0 + lr;
 #pragma unroll
-            for (int o = 16; o; o >>= 1)
-                s += __shfl_xor_sync(0xffffffffu, s, o);
-            const float mean = s / a.K;
-            float v = 0.f;
-            if (m < a.M)
-                for (int k = lane; k < a.K; k += 32) {
-                    const float dlt = a.x[static_cast<size_t>(m) * a.ldx + k] - mean;
-                    v = fmaf(dlt, dlt, v);
+        for (int g = 0; g < G; ++g) {
+            const int k = k0 + lk + 8 * g;
+            float *xo = xr + 8 * g, *wo = wr + 8 * g;
+            if (VEC && k + 8 <= ke) {
+                if (m < a.M) {
+                    const float4 *src = reinterpret_cast<const float4 *>(a.x + static_cast<size_t>(m) * a.ldx + k);
+                    const float4 v0 = src[0], v1 = src[1];
+                    xo[0] = v0.x;
+                    xo[1] = v0.y;
+                    xo[2] = v0.z;
+                    xo[3] = v0.w;
+                    xo[4] = v1.x;
+                    xo[5] = v1.y;
+                    xo[6] = v1.z;
+                    xo[7] = v1.w;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        xo[e] = 0.f;
                 }
+                if (n < a.N) {
+                    const uint2 q = *reinterpret_cast<const uint2 *>(a.wq + static_cast<size_t>(n) * a.K + k);
 #pragma unroll
-            for (int o = 16; o; o >>= 1)
-                v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0)
-                stats[r] = make_float2(mean, rsqrtf(v / a.K + a.eps));
+                    for (int e = 0; e < 4; ++e) {
+                        wo[e] = static_cast<float>(static_cast<int8_t>((q.x >> (8 * e)) & 0xffu));
+                        wo[4 + e] = static_cast<float>(static_cast<int8_t>((q.y >> (8 * e)) & 0xffu));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        wo[e] = 0.f;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int kk = k + e;
+                    xo[e] = (m < a.M && kk < ke) ? a.x[static_cast<size_t>(m) * a.ldx + kk] : 0.f;
+                    wo[e] = (n < a.N && kk < ke) ? static_cast<float>(a.wq[static_cast<size_t>(n) * a.K + kk]) : 0.f;
+                }
+            }
         }
-        __syncthreads();
-    }
+    };
+    auto stage = [&](int buf) {
+#pragma unroll
+        for (int q = 0; q < 2 * G; ++q) {
+            *reinterpret_cast<float4 *>(&Xs[buf][lr][lk + 4 * q]) =
+                make_float4(xr[4 * q], xr[4 * q + 1], xr[4 * q + 2], xr[4 * q + 3]);
+            *reinterpret_cast<float4 *>(&Ws[buf][lr][lk + 4 * q]) =
+                make_float4(wr[4 * q], wr[4 * q + 1], wr[4 * q + 2], wr[4 * q + 3]);
+        }
+    };
 
     f2_t acc[4][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         acc[i][0] = acc[i][1] = f2_pack(0.f, 0.f);
 
+    int buf = 0;
+    if (kb < ke) {
+        fetch(kb);
+        stage(0);
+    }
+    __syncthreads();
     for (int k0 = kb; k0 < ke; k0 += BK) {
+        const bool more = k0 + BK < ke;
+        if (more)
+            fetch(k0 + BK);  // in flight while this slice is multiplied
 #pragma unroll
-        for (int i = 0; i < (BM * BK) / kGemmThreads; ++i) {
-            const int e = tid + i * kGemmThreads;
-            const int r = e / BK, kk = e % BK;
-            const int m = m0 + r, k = k0 + kk;
-            float v = 0.f;
-            if (m < a.M && k < ke) {
-                if (PRO == kProConv) {
-                    const float *hs = a.hist + (static_cast<size_t>(m) * a.K + k) * (a.Kc - 1);
-                    const float *w = a.conv_w + static_cast<size_t>(k) * a.Kc;
-                    float pre = a.conv_b ? a.conv_b[k] : 0.f;
-                    for (int j = 0; j < a.Kc - 1; ++j)
-                        pre = fmaf(w[j], hs[j], pre);
-                    pre = fmaf(w[a.Kc - 1], a.x[static_cast<size_t>(m) * a.ldx + k], pre);
-                    v = silu_exact(pre);
-                } else {
-                    v = a.x[static_cast<size_t>(m) * a.ldx + k];
-                    if (PRO == kProLN) {
-                        const float2 st = stats[r];
-                        v = fmaf((v - st.x) * st.y, a.ln_w[k], a.ln_b[k]);
-                    }
-                }
-            }
-            Xs[kk][r] = v;
-        }
-#pragma unroll
-        for (int i = 0; i < (BN * BK) / kGemmThreads; ++i) {
-            const int e = tid + i * kGemmThreads;
-            const int r = e / BK, kk = e % BK;
-            const int n = n0 + r, k = k0 + kk;
-            Ws[kk][r] = (n < a.N && k < ke) ? static_cast<float>(a.wq[static_cast<size_t>(n) * a.K + k]) : 0.f;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < BK; ++kk) {
-            const float4 xv = *reinterpret_cast<const float4 *>(&Xs[kk][tm * 4]);
-            const float4 wv = *reinterpret_cast<const float4 *>(&Ws[kk][tn * 4]);
-            const f2_t w01 = f2_pack(wv.x, wv.y), w23 = f2_pack(wv.z, wv.w);
-            const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+        for (int kq = 0; kq < BK; kq += 4) {
+            float xk[4][4], wk[4][4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const f2_t xx = f2_pack(xs[i], xs[i]);
-                acc[i][0] = f2_fma(xx, w01, acc[i][0]);
-                acc[i][1] = f2_fma(xx, w23, acc[i][1]);
+                const float4 xv = *reinterpret_cast<const float4 *>(&Xs[buf][tm + 16 * i][kq]);
+                const float4 wv = *reinterpret_cast<const float4 *>(&Ws[buf][tn + 16 * i][kq]);
+                xk[i][0] = xv.x;
+                xk[i][1] = xv.y;
+                xk[i][2] = xv.z;
+                xk[i][3] = xv.w;
+                wk[i][0] = wv.x;
+                wk[i][1] = wv.y;
+                wk[i][2] = wv.z;
+                wk[i][3] = wv.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const f2_t w01 = f2_pack(wk[0][e], wk[1][e]);
+                const f2_t w23 = f2_pack(wk[2][e], wk[3][e]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const f2_t xx = f2_pack(xk[i][e], xk[i][e]);
+                    acc[i][0] = f2_fma(xx, w01, acc[i][0]);
+                    acc[i][1] = f2_fma(xx, w23, acc[i][1]);
+                }
             }
         }
-        __syncthreads();
+        if (more) {
+            stage(buf ^ 1);
+            __syncthreads();
+            buf ^= 1;
+        }
     }
 
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int m = m0 + tm * 4 + i;
+        const int m = m0 + tm + 16 * i;
         if (m >= a.M)
             continue;
         float v[4];
@@ -160,7 +280,7 @@ __global__ void __launch_bounds__(kGemmThreads) q8_gemm_kernel(const Q8GemmArgs 
         f2_unpack(acc[i][1], v[2], v[3]);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int n = n0 + tn * 4 + j;
+            const int n = n0 + tn + 16 * j;
             if (n >= a.N)
                 continue;
             const float out = v[j] * a.ws[n];
@@ -173,76 +293,62 @@ __global__ void __launch_bounds__(kGemmThreads) q8_gemm_kernel(const Q8GemmArgs 
     }
 }
 
+// ------------------------------------------------------------ the recurrence
 struct BlockSsmArgs {
-    int Bt, di, N, R, Kc;
-    const float *xz;   // [Bt][2 di]: xin | z
+    int Bt, di, N, R;
+    const float *xz;   // [Bt][xz_ld]: xin | z
+    const float *xc;   // [Bt][xc_ld]: SiLU(conv(xin))
+    int xz_ld, xc_ld, g_ld;
     const float *dbc;  // [Bt][dbc_ld]: dt | B | C (the x_proj rows, R + 2N used)
     int dbc_ld;
     const int8_t *dt_q;
     const float *dt_s, *dt_bias;  // [di][R], [di], [di]
     const float *A_log, *D;       // [di][N], [di]
-    const float *conv_w, *conv_b;  // [di][Kc], [di] or null
-    float *hist;  // [Bt][di][Kc-1] conv history, updated in place
-    float *h;     // [Bt][di][N] state, updated in place
-    float *g;     // [Bt][di] gated readout y * SiLU(z)
+    float *h;  // [Bt][di][N] state, updated in place
+    float *g;  // [Bt][g_ld] gated readout y * SiLU(z)
 };
 
 constexpr int kSsmThreads = 256;
 
-// One thread per (sequence, channel): the conv + SiLU (history shifted in
-// place), dt_proj from the sequence's R dt values, softplus, the N state
-// updates and the readout, gated.  HBM-bound on h (read and written once).
+// One thread per (sequence, channel): dt_proj from the sequence's R dt values,
+// softplus, the N state updates and the readout, gated.  HBM-bound on h (read
+// and written once).  Block (x, y): channels 256 x .. of sequence y.
 template <int NS>
 __global__ void __launch_bounds__(kSsmThreads) block_ssm_kernel(const BlockSsmArgs a) {
     extern __shared__ float srow[];  // this sequence's x_proj row (R + 2N floats)
     const int rowlen = a.R + 2 * a.N;
-    const int m = blockIdx.y;  // the sequence
+    const int m = blockIdx.y;
     const int c = blockIdx.x * kSsmThreads + threadIdx.x;
     for (int i = threadIdx.x; i < rowlen; i += kSsmThreads)
         srow[i] = a.dbc[static_cast<size_t>(m) * a.dbc_ld + i];
     __syncthreads();
     if (c >= a.di)
         return;
-    const float xin = a.xz[static_cast<size_t>(m) * 2 * a.di + c];
-    const float zv = a.xz[static_cast<size_t>(m) * 2 * a.di + a.di + c];
-    // conv + SiLU, history shifted
-    float *hs = a.hist + (static_cast<size_t>(m) * a.di + c) * (a.Kc - 1);
-    const float *w = a.conv_w + static_cast<size_t>(c) * a.Kc;
-    float pre = a.conv_b ? a.conv_b[c] : 0.f;
-    float hv[3] = {0.f, 0.f, 0.f};
-    for (int j = 0; j < a.Kc - 1; ++j) {
-        hv[j] = hs[j];
-        pre = fmaf(w[j], hv[j], pre);
-    }
-    pre = fmaf(w[a.Kc - 1], xin, pre);
-    for (int j = 0; j + 1 < a.Kc - 1; ++j)
-        hs[j] = hv[j + 1];
-    hs[a.Kc - 2] = xin;
-    const float xc = silu_exact(pre);
-    // dt_proj + softplus
+    const float xc = a.xc[static_cast<size_t>(m) * a.xc_ld + c];
+    const float zv = a.xz[static_cast<size_t>(m) * a.xz_ld + a.di + c];
     float dtv = 0.f;
     const int8_t *q = a.dt_q + static_cast<size_t>(c) * a.R;
     for (int r = 0; r < a.R; ++r)
         dtv = fmaf(static_cast<float>(q[r]), srow[r], dtv);
     const float v = fmaf(dtv, a.dt_s[c], a.dt_bias[c]);
-    const float delta = fmaxf(v, 0.f) + log1pf(__expf(-fabsf(v)));
-    // the recurrence and the readout
+    const float delta = fmaxf(v, 0.f) + log1pf(__expf(-fabsf(v)));  // softplus
     const float *Bm = srow + a.R, *Cm = srow + a.R + a.N;
     const float *al = a.A_log + static_cast<size_t>(c) * a.N;
     float *hp = a.h + (static_cast<size_t>(m) * a.di + c) * a.N;
     float acc = 0.f;
     const float du = delta * xc;
+    const float dl2 = -delta * kLog2e;
     if (NS == 16 && a.N == 16) {
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-            float4 h4 = reinterpret_cast<const float4 *>(hp)[q4];
+            const float4 h4 = reinterpret_cast<const float4 *>(hp)[q4];
             const float4 a4 = reinterpret_cast<const float4 *>(al)[q4];
             float hh[4] = {h4.x, h4.y, h4.z, h4.w};
             const float aa[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int n = 4 * q4 + e;
-                const float ab = ex2_approx(delta * (-__expf(aa[e])) * kLog2e);  // exp(Delta A), A = -exp(A_log)
+                const float ab = ex2_approx(dl2 * __expf(aa[e]));  // exp(Delta A), A = -exp(A_log)
                 hh[e] = fmaf(ab, hh[e], du * Bm[n]);
                 acc = fmaf(hh[e], Cm[n], acc);
             }
@@ -250,14 +356,14 @@ __global__ void __launch_bounds__(kSsmThreads) block_ssm_kernel(const BlockSsmAr
         }
     } else {
         for (int n = 0; n < a.N; ++n) {
-            const float ab = ex2_approx(delta * (-__expf(al[n])) * kLog2e);
+            const float ab = ex2_approx(dl2 * __expf(al[n]));
             const float hn = fmaf(ab, hp[n], du * Bm[n]);
             hp[n] = hn;
             acc = fmaf(hn, Cm[n], acc);
         }
     }
     const float y = fmaf(a.D[c], xc, acc);
-    a.g[static_cast<size_t>(m) * a.di + c] = y * silu_exact(zv);
+    a.g[static_cast<size_t>(m) * a.g_ld + c] = y * silu_exact(zv);
 }
 
 }  // namespace s6

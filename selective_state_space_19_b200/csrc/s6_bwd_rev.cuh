@@ -33,6 +33,8 @@
 // the segment after it, which was pulled earlier, so every (bounded) wait ends.
 #pragma once
 
+#include <type_traits>
+
 #include "s6_common.cuh"
 #include "s6_scan.cuh"
 
@@ -438,151 +440,164 @@ __global__ void __launch_bounds__(kScanBlock, 1)
         }
         __syncwarp();
 
-        // ---- 2. recompute the sub-chunk forward from the checkpoint; keep every state
-        {
-            f2_t h[4] = {f2_pack(ck0.x, ck0.y), f2_pack(ck0.z, ck0.w), f2_pack(ck1.x, ck1.y), f2_pack(ck1.z, ck1.w)};
+        float *accp = &sm.acc[c & 1][0][0];  // this sub-chunk's dB / dC sums
+        // phases 2 and 3 over the sub-chunk's tokens; a full sub-chunk takes a
+        // compile-time trip count
+        auto phases = [&](auto full_tag) {
+            constexpr bool FULL = decltype(full_tag)::value;
+            const int tc = FULL ? KC : tcount;
+            // ---- 2. recompute the sub-chunk forward from the checkpoint; keep every state
+            {
+                f2_t h[4] = {f2_pack(ck0.x, ck0.y), f2_pack(ck0.z, ck0.w), f2_pack(ck1.x, ck1.y), f2_pack(ck1.z, ck1.w)};
 #pragma unroll 2
-            for (int j = 0; j < tcount; ++j) {
+                for (int j = 0; j < tc; ++j) {
+                    const float4 du = tb[j][cw];
+                    const f2_t dd = f2_pack(du.x, du.x);
+                    const f2_t uu = f2_pack(du.y, du.y);
+                    const f2_t wdu = f2_mul(dd, uu);
+                    const ulonglong2 B01 = *reinterpret_cast<const ulonglong2 *>(&bc[j][0][n0]);
+                    const ulonglong2 B23 = *reinterpret_cast<const ulonglong2 *>(&bc[j][0][n0 + 4]);
+                    const f2_t Bq[4] = {B01.x, B01.y, B23.x, B23.y};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float x0, x1;
+                        f2_unpack(f2_mul(dd, A2p[q]), x0, x1);
+                        const f2_t ab = f2_pack(ex2_approx(x0), ex2_approx(x1));
+                        if (ZOH) {
+                            const f2_t nk = f2_mul(nrAp[q], f2_mul(uu, Bq[q]));
+                            h[q] = f2_fma(ab, f2_sub(h[q], nk), nk);
+                        } else {
+                            h[q] = f2_fma(ab, h[q], f2_mul(wdu, Bq[q]));
+                        }
+                    }
+                    float a0, a1, a2, a3, a4, a5, a6, a7;
+                    f2_unpack(h[0], a0, a1);
+                    f2_unpack(h[1], a2, a3);
+                    f2_unpack(h[2], a4, a5);
+                    f2_unpack(h[3], a6, a7);
+                    hb[j][0][lane] = make_float4(a0, a1, a2, a3);
+                    hb[j][1][lane] = make_float4(a4, a5, a6, a7);
+                }
+            }
+            __syncwarp();
+
+            // ---- 3. walk the sub-chunk back
+            // h_t of the token being walked back; h_{t-1} becomes the next token's h_t
+            float4 h0 = hb[tc - 1][0][lane], h1 = hb[tc - 1][1][lane];
+#pragma unroll 2
+            for (int j = tc - 1; j >= 0; --j) {
                 const float4 du = tb[j][cw];
-                const f2_t dd = f2_pack(du.x, du.x);
-                const f2_t uu = f2_pack(du.y, du.y);
-                const f2_t wdu = f2_mul(dd, uu);
+                const float delta = du.x, u = du.y, ds = du.z, dygp = du.w;
+                // softplus'(v) = sigmoid(v) = 1 - e^-Delta (Delta = softplus(v))
+                const float sig_v = 1.0f - ex2_approx(-delta * kLog2e);
+                float4 p0 = ck0, p1 = ck1;  // h_{t-1}
+                if (j > 0) {
+                    p0 = hb[j - 1][0][lane];
+                    p1 = hb[j - 1][1][lane];
+                }
+                const f2_t ht[4] = {f2_pack(h0.x, h0.y), f2_pack(h0.z, h0.w), f2_pack(h1.x, h1.y), f2_pack(h1.z, h1.w)};
+                const f2_t hp[4] = {f2_pack(p0.x, p0.y), f2_pack(p0.z, p0.w), f2_pack(p1.x, p1.y), f2_pack(p1.z, p1.w)};
                 const ulonglong2 B01 = *reinterpret_cast<const ulonglong2 *>(&bc[j][0][n0]);
                 const ulonglong2 B23 = *reinterpret_cast<const ulonglong2 *>(&bc[j][0][n0 + 4]);
+                const ulonglong2 C01 = *reinterpret_cast<const ulonglong2 *>(&bc[j][1][n0]);
+                const ulonglong2 C23 = *reinterpret_cast<const ulonglong2 *>(&bc[j][1][n0 + 4]);
                 const f2_t Bq[4] = {B01.x, B01.y, B23.x, B23.y};
+                const f2_t Cq[4] = {C01.x, C01.y, C23.x, C23.y};
+                const f2_t dsv = f2_pack(ds, ds);
+                const f2_t dd = f2_pack(delta, delta);
+                const f2_t uu = f2_pack(u, u);
+                const f2_t wdu = f2_mul(dd, uu);
+                f2_t acc_s = zero2, acc_b = zero2, acc_q = zero2, acc_z = zero2;
+                float vB[8], vC[8];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     float x0, x1;
                     f2_unpack(f2_mul(dd, A2p[q]), x0, x1);
                     const f2_t ab = f2_pack(ex2_approx(x0), ex2_approx(x1));
+                    const f2_t dh = f2_fma(dsv, Cq[q], gcar[q]);
+                    acc_s = f2_fma(ht[q], Cq[q], acc_s);
+                    const f2_t dC2 = f2_mul(dsv, ht[q]);
+                    f2_t dB2;
                     if (ZOH) {
-                        const f2_t nk = f2_mul(nrAp[q], f2_mul(uu, Bq[q]));
-                        h[q] = f2_fma(ab, f2_sub(h[q], nk), nk);
+                        const f2_t gain = f2_mul(f2_sub(f2_pack(1.f, 1.f), ab), nrAp[q]);  // (a - 1)/A
+                        const f2_t dhB = f2_mul(dh, Bq[q]);
+                        dB2 = f2_mul(f2_mul(dh, gain), uu);
+                        acc_b = f2_fma(dhB, gain, acc_b);
+                        acc_z = f2_fma(dhB, ab, acc_z);  // dgain/dDelta = a
                     } else {
-                        h[q] = f2_fma(ab, h[q], f2_mul(wdu, Bq[q]));
+                        dB2 = f2_mul(dh, wdu);
+                        acc_b = f2_fma(dh, Bq[q], acc_b);
                     }
+                    const f2_t qv = f2_mul(f2_mul(dh, hp[q]), ab);  // dh h_{t-1} a
+                    acc_q = f2_fma(qv, Ap[q], acc_q);
+                    dAacc[q] = f2_fma(qv, dd, dAacc[q]);
+                    if (ZOH) {
+                        float g0, g1, A0, A1, ab0, ab1, dhb0, dhb1;
+                        f2_unpack(Ap[q], A0, A1);
+                        f2_unpack(ab, ab0, ab1);
+                        f2_unpack(f2_mul(f2_mul(dh, Bq[q]), uu), dhb0, dhb1);
+                        g0 = dhb0 * zoh_dgain_dA_rev(delta * A0, ab0, delta, A0);
+                        g1 = dhb1 * zoh_dgain_dA_rev(delta * A1, ab1, delta, A1);
+                        dAacc[q] = f2_add(dAacc[q], f2_pack(g0, g1));
+                    }
+                    gcar[q] = f2_mul(dh, ab);
+                    f2_unpack(dB2, vB[2 * q], vB[2 * q + 1]);
+                    f2_unpack(dC2, vC[2 * q], vC[2 * q + 1]);
                 }
-                float a0, a1, a2, a3, a4, a5, a6, a7;
-                f2_unpack(h[0], a0, a1);
-                f2_unpack(h[1], a2, a3);
-                f2_unpack(h[2], a4, a5);
-                f2_unpack(h[3], a6, a7);
-                hb[j][0][lane] = make_float4(a0, a1, a2, a3);
-                hb[j][1][lane] = make_float4(a4, a5, a6, a7);
-            }
-        }
-        __syncwarp();
-
-        // ---- 3. walk the sub-chunk back
-        float *accp = &sm.acc[c & 1][0][0];
-#pragma unroll 2
-        for (int j = tcount - 1; j >= 0; --j) {
-            const float4 du = tb[j][cw];
-            const float delta = du.x, u = du.y, ds = du.z, dygp = du.w;
-            // softplus'(v) = sigmoid(v) = 1 - e^-Delta (Delta = softplus(v))
-            const float sig_v = 1.0f - ex2_approx(-delta * kLog2e);
-            float4 h0 = hb[j][0][lane], h1 = hb[j][1][lane];
-            float4 p0 = ck0, p1 = ck1;  // h_{t-1}
-            if (j > 0) {
-                p0 = hb[j - 1][0][lane];
-                p1 = hb[j - 1][1][lane];
-            }
-            const f2_t ht[4] = {f2_pack(h0.x, h0.y), f2_pack(h0.z, h0.w), f2_pack(h1.x, h1.y), f2_pack(h1.z, h1.w)};
-            const f2_t hp[4] = {f2_pack(p0.x, p0.y), f2_pack(p0.z, p0.w), f2_pack(p1.x, p1.y), f2_pack(p1.z, p1.w)};
-            const ulonglong2 B01 = *reinterpret_cast<const ulonglong2 *>(&bc[j][0][n0]);
-            const ulonglong2 B23 = *reinterpret_cast<const ulonglong2 *>(&bc[j][0][n0 + 4]);
-            const ulonglong2 C01 = *reinterpret_cast<const ulonglong2 *>(&bc[j][1][n0]);
-            const ulonglong2 C23 = *reinterpret_cast<const ulonglong2 *>(&bc[j][1][n0 + 4]);
-            const f2_t Bq[4] = {B01.x, B01.y, B23.x, B23.y};
-            const f2_t Cq[4] = {C01.x, C01.y, C23.x, C23.y};
-            const f2_t dsv = f2_pack(ds, ds);
-            const f2_t dd = f2_pack(delta, delta);
-            const f2_t uu = f2_pack(u, u);
-            const f2_t wdu = f2_mul(dd, uu);
-            f2_t acc_s = zero2, acc_b = zero2, acc_q = zero2, acc_z = zero2;
-            float vB[8], vC[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float x0, x1;
-                f2_unpack(f2_mul(dd, A2p[q]), x0, x1);
-                const f2_t ab = f2_pack(ex2_approx(x0), ex2_approx(x1));
-                const f2_t dh = f2_fma(dsv, Cq[q], gcar[q]);
-                acc_s = f2_fma(ht[q], Cq[q], acc_s);
-                const f2_t dC2 = f2_mul(dsv, ht[q]);
-                f2_t dB2;
+                // sums over the channel's 16 states: this thread's 8, then the partner's
+                float s0, s1, b0, b1, q0, q1, z0, z1;
+                f2_unpack(acc_s, s0, s1);
+                f2_unpack(acc_b, b0, b1);
+                f2_unpack(acc_q, q0, q1);
+                f2_unpack(acc_z, z0, z1);
+                float sp = s0 + s1, bp = b0 + b1, qp = q0 + q1;
+                sp += __shfl_xor_sync(full, sp, 1);
+                bp += __shfl_xor_sync(full, bp, 1);
+                qp += __shfl_xor_sync(full, qp, 1);
+                float zp = 0.f;
                 if (ZOH) {
-                    const f2_t gain = f2_mul(f2_sub(f2_pack(1.f, 1.f), ab), nrAp[q]);  // (a - 1)/A
-                    const f2_t dhB = f2_mul(dh, Bq[q]);
-                    dB2 = f2_mul(f2_mul(dh, gain), uu);
-                    acc_b = f2_fma(dhB, gain, acc_b);
-                    acc_z = f2_fma(dhB, ab, acc_z);  // dgain/dDelta = a
-                } else {
-                    dB2 = f2_mul(dh, wdu);
-                    acc_b = f2_fma(dh, Bq[q], acc_b);
+                    zp = z0 + z1;
+                    zp += __shfl_xor_sync(full, zp, 1);
                 }
-                const f2_t qv = f2_mul(f2_mul(dh, hp[q]), ab);  // dh h_{t-1} a
-                acc_q = f2_fma(qv, Ap[q], acc_q);
-                dAacc[q] = f2_fma(qv, dd, dAacc[q]);
-                if (ZOH) {
-                    float g0, g1, A0, A1, ab0, ab1, dhb0, dhb1;
-                    f2_unpack(Ap[q], A0, A1);
-                    f2_unpack(ab, ab0, ab1);
-                    f2_unpack(f2_mul(f2_mul(dh, Bq[q]), uu), dhb0, dhb1);
-                    g0 = dhb0 * zoh_dgain_dA_rev(delta * A0, ab0, delta, A0);
-                    g1 = dhb1 * zoh_dgain_dA_rev(delta * A1, ab1, delta, A1);
-                    dAacc[q] = f2_add(dAacc[q], f2_pack(g0, g1));
+                const float s_tot = fmaf(Dd, u, sp);
+                const float dut = ZOH ? fmaf(ds, Dd, bp) : fmaf(ds, Dd, delta * bp);
+                const float ddel = ZOH ? fmaf(u, zp, qp) : fmaf(u, bp, qp);
+                const float dv = ddel * sig_v;
+                float dxo = dut;
+                if (CONV) {
+                    const float pre = pre_at(j);
+                    const float sp_ = rcp_approx(1.0f + ex2_approx(fminf(-pre * kLog2e, 120.0f)));
+                    const float dpre = dut * sp_ * fmaf(pre, 1.0f - sp_, 1.0f);  // SiLU'(pre)
+                    dxo = fmaf(w3, dpre, fmaf(w2, dp1, fmaf(w1, dp2, w0 * dp3)));
+                    dW0 = fmaf(dpre, ld(xs, j), dW0);
+                    dW1 = fmaf(dpre, ld(xs, j + 1), dW1);
+                    dW2 = fmaf(dpre, ld(xs, j + 2), dW2);
+                    dW3 = fmaf(dpre, ld(xs, j + 3), dW3);
+                    dcb += dpre;
+                    dp3 = dp2;
+                    dp2 = dp1;
+                    dp1 = dpre;
                 }
-                gcar[q] = f2_mul(dh, ab);
-                f2_unpack(dB2, vB[2 * q], vB[2 * q + 1]);
-                f2_unpack(dC2, vC[2 * q], vC[2 * q + 1]);
+                dDa = fmaf(ds, u, dDa);
+                dba += dv;
+                if (live && sub == (j & 1)) {
+                    const size_t o = (static_cast<size_t>(b) * a.L + t0 + j) * a.d + ch;
+                    a.du[o] = dxo;
+                    a.ddt[o] = dv;
+                    if (a.has_z)
+                        a.dz[o] = dygp * s_tot;
+                }
+                // dB, dC of token t0 + j summed over the warp's channels, then the CTA's
+                const float r = reduce_scatter16(vB, vC, lane);
+                atomicAdd(accp + j * 32 + o_lane, r);
+                h0 = p0;
+                h1 = p1;
             }
-            // sums over the channel's 16 states: this thread's 8, then the partner's
-            float s0, s1, b0, b1, q0, q1, z0, z1;
-            f2_unpack(acc_s, s0, s1);
-            f2_unpack(acc_b, b0, b1);
-            f2_unpack(acc_q, q0, q1);
-            f2_unpack(acc_z, z0, z1);
-            float sp = s0 + s1, bp = b0 + b1, qp = q0 + q1;
-            sp += __shfl_xor_sync(full, sp, 1);
-            bp += __shfl_xor_sync(full, bp, 1);
-            qp += __shfl_xor_sync(full, qp, 1);
-            float zp = 0.f;
-            if (ZOH) {
-                zp = z0 + z1;
-                zp += __shfl_xor_sync(full, zp, 1);
-            }
-            const float s_tot = fmaf(Dd, u, sp);
-            const float dut = ZOH ? fmaf(ds, Dd, bp) : fmaf(ds, Dd, delta * bp);
-            const float ddel = ZOH ? fmaf(u, zp, qp) : fmaf(u, bp, qp);
-            const float dv = ddel * sig_v;
-            float dxo = dut;
-            if (CONV) {
-                const float pre = pre_at(j);
-                const float sp_ = rcp_approx(1.0f + ex2_approx(fminf(-pre * kLog2e, 120.0f)));
-                const float dpre = dut * sp_ * fmaf(pre, 1.0f - sp_, 1.0f);  // SiLU'(pre)
-                dxo = fmaf(w3, dpre, fmaf(w2, dp1, fmaf(w1, dp2, w0 * dp3)));
-                dW0 = fmaf(dpre, ld(xs, j), dW0);
-                dW1 = fmaf(dpre, ld(xs, j + 1), dW1);
-                dW2 = fmaf(dpre, ld(xs, j + 2), dW2);
-                dW3 = fmaf(dpre, ld(xs, j + 3), dW3);
-                dcb += dpre;
-                dp3 = dp2;
-                dp2 = dp1;
-                dp1 = dpre;
-            }
-            dDa = fmaf(ds, u, dDa);
-            dba += dv;
-            if (live && sub == (j & 1)) {
-                const size_t o = (static_cast<size_t>(b) * a.L + t0 + j) * a.d + ch;
-                a.du[o] = dxo;
-                a.ddt[o] = dv;
-                if (a.has_z)
-                    a.dz[o] = dygp * s_tot;
-            }
-            // dB, dC of token t0 + j summed over the warp's channels, then the CTA's
-            const float r = reduce_scatter16(vB, vC, lane);
-            atomicAdd(accp + j * 32 + o_lane, r);
-        }
+        };
+        if (tcount == KC)
+            phases(std::true_type{});
+        else
+            phases(std::false_type{});
 
         // release the stage (its tiles are no longer read)
         __syncwarp();

@@ -799,7 +799,7 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                     g2c = g2n;
                 };
                 if (FULL) {
-#pragma unroll 3
+#pragma unroll 2
                     for (int p = 0; p < T - 4; p += 4)
                         quad(p, p >> 2, std::false_type{});
                     quad(T - 4, (T - 4) >> 2, std::true_type{});
