@@ -1181,10 +1181,11 @@ int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x
     const unsigned mt = static_cast<unsigned>((Bt + s6::kGemmBM - 1) / s6::kGemmBM);
     // a product Y = X W^T over the whole batch; the reduction is split across
     // blocks (atomic adds into Y) until there are about two blocks per SM
+    // (accumulate: Y += the product, Y already holding what it should be added to)
     auto gemm = [&](const float *X, int ldx, int64_t n_out, int64_t k, const int8_t *wq, const float *ws, float *Y,
                     int ldy, bool add) -> int {
         const int64_t tiles = ((n_out + s6::kGemmBN - 1) / s6::kGemmBN) * mt;
-        int64_t sp = add ? (2 * sms + tiles - 1) / tiles : 1;
+        int64_t sp = add ? (4 * sms + tiles - 1) / tiles : 1;
         const int64_t max_sp = (k + s6::kGemmBK - 1) / s6::kGemmBK;
         if (sp > max_sp)
             sp = max_sp;
@@ -1231,7 +1232,11 @@ int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x
         x, w->ln_w, w->ln_b, hn, static_cast<int>(Bt), static_cast<int>(dm), dims->eps);
     if (cudaGetLastError() != cudaSuccess)
         return S6_ERR_CUDA;
-    rc = gemm(hn, static_cast<int>(dm), 2 * di, dm, w->in_q, w->in_s, xz, static_cast<int>(l_xz), false);
+    // in_proj also splits its reduction (atomic adds into a zeroed xz): its 2 di x Bt
+    // outputs alone give too few blocks to hide the load latency
+    if (cudaMemsetAsync(xz, 0, sizeof(float) * Bt * l_xz, s) != cudaSuccess)
+        return S6_ERR_CUDA;
+    rc = gemm(hn, static_cast<int>(dm), 2 * di, dm, w->in_q, w->in_s, xz, static_cast<int>(l_xz), true);
     if (rc != S6_OK)
         return rc;
     // 2. conv + SiLU (history shifted) and x_proj -> dt | B | C, a block per sequence

@@ -29,7 +29,11 @@ __device__ __forceinline__ float silu_exact(float v) { return v / (1.0f + __expf
 // ------------------------------------------------------------ LayerNorm
 constexpr int kLnThreads = 256;  // 8 rows per block, a warp per row
 
-// out[m] = (x[m] - mean) / sqrt(var + eps) * w + b (biased variance)
+constexpr int kLnPerLane = 32;   // rows up to 1024 values are held in registers
+
+// out[m] = (x[m] - mean) / sqrt(var + eps) * w + b (biased variance).  The
+// row is read once into registers (two-pass statistics from them); longer
+// rows are read again for each pass.
 __global__ void __launch_bounds__(kLnThreads) block_layernorm_kernel(const float *x, const float *w, const float *b,
                                                                      float *out, int M, int K, float eps) {
     const int m = blockIdx.x * (kLnThreads / 32) + (threadIdx.x >> 5);
@@ -37,6 +41,41 @@ __global__ void __launch_bounds__(kLnThreads) block_layernorm_kernel(const float
     if (m >= M)
         return;
     const float *xr = x + static_cast<size_t>(m) * K;
+    float *orow = out + static_cast<size_t>(m) * K;
+    if (K <= 32 * kLnPerLane) {
+        float v[kLnPerLane];
+#pragma unroll
+        for (int i = 0; i < kLnPerLane; ++i) {
+            const int k = lane + 32 * i;
+            v[i] = k < K ? xr[k] : 0.f;
+        }
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < kLnPerLane; ++i)
+            s += v[i];
+#pragma unroll
+        for (int o = 16; o; o >>= 1)
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+        const float mean = s / K;
+        float q = 0.f;
+#pragma unroll
+        for (int i = 0; i < kLnPerLane; ++i) {
+            const int k = lane + 32 * i;
+            const float d = k < K ? v[i] - mean : 0.f;
+            q = fmaf(d, d, q);
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1)
+            q += __shfl_xor_sync(0xffffffffu, q, o);
+        const float r = rsqrtf(q / K + eps);
+#pragma unroll
+        for (int i = 0; i < kLnPerLane; ++i) {
+            const int k = lane + 32 * i;
+            if (k < K)
+                orow[k] = fmaf((v[i] - mean) * r, w[k], b[k]);
+        }
+        return;
+    }
     float s = 0.f;
     for (int k = lane; k < K; k += 32)
         s += xr[k];
@@ -44,16 +83,15 @@ __global__ void __launch_bounds__(kLnThreads) block_layernorm_kernel(const float
     for (int o = 16; o; o >>= 1)
         s += __shfl_xor_sync(0xffffffffu, s, o);
     const float mean = s / K;
-    float v = 0.f;
+    float q = 0.f;
     for (int k = lane; k < K; k += 32) {
         const float d = xr[k] - mean;
-        v = fmaf(d, d, v);
+        q = fmaf(d, d, q);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    const float r = rsqrtf(v / K + eps);
-    float *orow = out + static_cast<size_t>(m) * K;
+        q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float r = rsqrtf(q / K + eps);
     for (int k = lane; k < K; k += 32)
         orow[k] = fmaf((xr[k] - mean) * r, w[k], b[k]);
 }
@@ -64,44 +102,89 @@ constexpr int kConvXThreads = 256;
 // One block per sequence m: xc[c] = SiLU(conv_b + sum_{j<K-1} w[j] hist[j] +
 // w[K-1] xin[c]) for every channel (the history drops its oldest input and
 // appends xin), kept in shared memory and written out; then the x_proj rows
-// dbc[m][o] = xp_s[o] * sum_c xp_q[o][c] xc[c], a warp per output row.
+// dbc[m][o] = xp_s[o] * sum_c xp_q[o][c] xc[c], each row split over four
+// consecutive threads (a quarter of the channels each) and summed by shuffles.
 __global__ void __launch_bounds__(kConvXThreads) block_conv_xproj_kernel(
-    const float *xz, int ldxz, const float *conv_w, const float *conv_b, float *hist, float *xc, int ldxc,
-    const int8_t *xp_q, const float *xp_s, float *dbc, int ld_dbc, int di, int Kc, int n_out) {
+    const float *__restrict__ xz, int ldxz, const float *__restrict__ conv_w, const float *__restrict__ conv_b,
+    float *__restrict__ hist, float *__restrict__ xc, int ldxc, const int8_t *__restrict__ xp_q,
+    const float *__restrict__ xp_s, float *__restrict__ dbc, int ld_dbc, int di, int Kc, int n_out) {
     extern __shared__ __align__(16) float xcs[];  // di floats
     const int m = blockIdx.x;
-    for (int c = threadIdx.x; c < di; c += kConvXThreads) {
-        const float xin = xz[static_cast<size_t>(m) * ldxz + c];
-        float *hs = hist + (static_cast<size_t>(m) * di + c) * (Kc - 1);
-        const float *w = conv_w + static_cast<size_t>(c) * Kc;
-        float pre = conv_b ? conv_b[c] : 0.f;
-        float hv[3] = {0.f, 0.f, 0.f};
-        for (int j = 0; j < Kc - 1; ++j) {
-            hv[j] = hs[j];
-            pre = fmaf(w[j], hv[j], pre);
+    // conv: a thread's channels in groups of 4, every load of a group issued first
+    for (int c0 = threadIdx.x; c0 < di; c0 += 4 * kConvXThreads) {
+        float xin[4], hv[4][3], wv[4][4], bv[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int c = c0 + g * kConvXThreads;
+            xin[g] = 0.f;
+            bv[g] = 0.f;
+#pragma unroll
+            for (int j = 0; j < 3; ++j)
+                hv[g][j] = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                wv[g][j] = 0.f;
+            if (c < di) {
+                xin[g] = xz[static_cast<size_t>(m) * ldxz + c];
+                const float *hs = hist + (static_cast<size_t>(m) * di + c) * (Kc - 1);
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+                    if (j < Kc - 1)
+                        hv[g][j] = hs[j];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (j < Kc)
+                        wv[g][j] = conv_w[static_cast<size_t>(c) * Kc + j];
+                bv[g] = conv_b ? conv_b[c] : 0.f;
+            }
         }
-        pre = fmaf(w[Kc - 1], xin, pre);
-        for (int j = 0; j + 1 < Kc - 1; ++j)
-            hs[j] = hv[j + 1];
-        hs[Kc - 2] = xin;
-        const float v = silu_exact(pre);
-        xcs[c] = v;
-        xc[static_cast<size_t>(m) * ldxc + c] = v;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int c = c0 + g * kConvXThreads;
+            if (c >= di)
+                continue;
+            // taps: w[j] on the history (oldest first), w[Kc-1] on xin
+            float pre = bv[g];
+#pragma unroll
+            for (int j = 0; j < 3; ++j)
+                if (j < Kc - 1)
+                    pre = fmaf(wv[g][j], hv[g][j], pre);
+            float wlast = wv[g][3];
+            if (Kc == 3)
+                wlast = wv[g][2];
+            else if (Kc == 2)
+                wlast = wv[g][1];
+            pre = fmaf(wlast, xin[g], pre);
+            float *hs = hist + (static_cast<size_t>(m) * di + c) * (Kc - 1);
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+                if (j + 1 < Kc - 1)
+                    hs[j] = hv[g][j + 1];
+            hs[Kc - 2] = xin[g];
+            const float v = silu_exact(pre);
+            xcs[c] = v;
+            xc[static_cast<size_t>(m) * ldxc + c] = v;
+        }
     }
     __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const bool vec = (di % 4) == 0 && (reinterpret_cast<uintptr_t>(xp_q) & 3) == 0;
-    for (int o = warp; o < n_out; o += kConvXThreads / 32) {
-        const int8_t *q = xp_q + static_cast<size_t>(o) * di;
+    const bool vec = (di % 16) == 0 && (reinterpret_cast<uintptr_t>(xp_q) & 3) == 0;
+    const int part = threadIdx.x & 3;  // which quarter of the channels
+    // every thread runs the same number of rounds, so the shuffles below see
+    // full warps
+    for (int ob = 0; ob < n_out; ob += kConvXThreads / 4) {
+        const int o = ob + (threadIdx.x >> 2);
+        const bool on = o < n_out;
+        const int8_t *q = xp_q + static_cast<size_t>(on ? o : 0) * di;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (vec) {
-            // four channels per lane step: one 4-byte weight load, one float4 of xc
-            const int *qw = reinterpret_cast<const int *>(q);
-            const float4 *x4 = reinterpret_cast<const float4 *>(xcs);
-#pragma unroll 4
-            for (int c4 = lane; c4 < di / 4; c4 += 32) {
-                const int wv = qw[c4];
-                const float4 xv = x4[c4];
+        if (!on) {
+        } else if (vec) {
+            const int quarter = di / 16;  // 4-channel groups per quarter
+            const int *qw = reinterpret_cast<const int *>(q) + part * quarter;
+            const float4 *x4 = reinterpret_cast<const float4 *>(xcs) + part * quarter;
+#pragma unroll 8
+            for (int i = 0; i < quarter; ++i) {
+                const int wv = qw[i];
+                const float4 xv = x4[i];
                 acc[0] = fmaf(static_cast<float>(static_cast<int8_t>(wv & 0xff)), xv.x, acc[0]);
                 acc[1] = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 8) & 0xff)), xv.y, acc[1]);
                 acc[2] = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 16) & 0xff)), xv.z, acc[2]);
@@ -109,14 +192,13 @@ __global__ void __launch_bounds__(kConvXThreads) block_conv_xproj_kernel(
             }
         } else {
 #pragma unroll 4
-            for (int c = lane; c < di; c += 32)
-                acc[c & 3] = fmaf(static_cast<float>(q[c]), xcs[c], acc[c & 3]);
+            for (int c = part; c < di; c += 4)
+                acc[(c >> 2) & 3] = fmaf(static_cast<float>(q[c]), xcs[c], acc[(c >> 2) & 3]);
         }
         float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-#pragma unroll
-        for (int off = 16; off; off >>= 1)
-            sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane == 0)
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        if (on && part == 0)
             dbc[static_cast<size_t>(m) * ld_dbc + o] = sum * xp_s[o];
     }
 }
@@ -326,25 +408,43 @@ __global__ void __launch_bounds__(kSsmThreads) block_ssm_kernel(const BlockSsmAr
         return;
     const float xc = a.xc[static_cast<size_t>(m) * a.xc_ld + c];
     const float zv = a.xz[static_cast<size_t>(m) * a.xz_ld + a.di + c];
+    float *hp = a.h + (static_cast<size_t>(m) * a.di + c) * a.N;
+    const float *al = a.A_log + static_cast<size_t>(c) * a.N;
+    float4 h4[4], a4[4];
+    if (NS == 16 && a.N == 16) {  // the state and its rates in flight first
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            h4[q4] = reinterpret_cast<const float4 *>(hp)[q4];
+            a4[q4] = reinterpret_cast<const float4 *>(al)[q4];
+        }
+    }
     float dtv = 0.f;
     const int8_t *q = a.dt_q + static_cast<size_t>(c) * a.R;
-    for (int r = 0; r < a.R; ++r)
-        dtv = fmaf(static_cast<float>(q[r]), srow[r], dtv);
+    if ((a.R % 4) == 0 && (reinterpret_cast<uintptr_t>(a.dt_q) & 3) == 0) {
+        const int *qw = reinterpret_cast<const int *>(q);
+#pragma unroll 6
+        for (int r4 = 0; r4 < a.R / 4; ++r4) {
+            const int wv = qw[r4];
+            dtv = fmaf(static_cast<float>(static_cast<int8_t>(wv & 0xff)), srow[4 * r4], dtv);
+            dtv = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 8) & 0xff)), srow[4 * r4 + 1], dtv);
+            dtv = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 16) & 0xff)), srow[4 * r4 + 2], dtv);
+            dtv = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 24) & 0xff)), srow[4 * r4 + 3], dtv);
+        }
+    } else {
+        for (int r = 0; r < a.R; ++r)
+            dtv = fmaf(static_cast<float>(q[r]), srow[r], dtv);
+    }
     const float v = fmaf(dtv, a.dt_s[c], a.dt_bias[c]);
     const float delta = fmaxf(v, 0.f) + log1pf(__expf(-fabsf(v)));  // softplus
     const float *Bm = srow + a.R, *Cm = srow + a.R + a.N;
-    const float *al = a.A_log + static_cast<size_t>(c) * a.N;
-    float *hp = a.h + (static_cast<size_t>(m) * a.di + c) * a.N;
     float acc = 0.f;
     const float du = delta * xc;
     const float dl2 = -delta * kLog2e;
     if (NS == 16 && a.N == 16) {
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-            const float4 h4 = reinterpret_cast<const float4 *>(hp)[q4];
-            const float4 a4 = reinterpret_cast<const float4 *>(al)[q4];
-            float hh[4] = {h4.x, h4.y, h4.z, h4.w};
-            const float aa[4] = {a4.x, a4.y, a4.z, a4.w};
+            float hh[4] = {h4[q4].x, h4[q4].y, h4[q4].z, h4[q4].w};
+            const float aa[4] = {a4[q4].x, a4[q4].y, a4[q4].z, a4[q4].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int n = 4 * q4 + e;
