@@ -26,6 +26,19 @@ namespace s6 {
 
 __device__ __forceinline__ float silu_exact(float v) { return v / (1.0f + __expf(-v)); }
 
+// Four int8 values (bytes of w, lowest first) as floats without the
+// conversion unit: each byte, biased to unsigned (b + 128), is placed under the
+// exponent of 2^23 -- the float 2^23 + b + 128, exact -- and 2^23 + 128 is
+// subtracted.
+__device__ __forceinline__ float4 i8x4_to_f32x4(int w) {
+    const unsigned u = static_cast<unsigned>(w) ^ 0x80808080u;
+    constexpr float kBias = 8388608.0f + 128.0f;
+    return make_float4(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440)) - kBias,
+                       __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7441)) - kBias,
+                       __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7442)) - kBias,
+                       __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7443)) - kBias);
+}
+
 // ------------------------------------------------------------ LayerNorm
 constexpr int kLnThreads = 256;  // 8 rows per block, a warp per row
 
@@ -167,38 +180,35 @@ __global__ void __launch_bounds__(kConvXThreads) block_conv_xproj_kernel(
         }
     }
     __syncthreads();
-    const bool vec = (di % 16) == 0 && (reinterpret_cast<uintptr_t>(xp_q) & 3) == 0;
-    const int part = threadIdx.x & 3;  // which quarter of the channels
-    // every thread runs the same number of rounds, so the shuffles below see
-    // full warps
-    for (int ob = 0; ob < n_out; ob += kConvXThreads / 4) {
-        const int o = ob + (threadIdx.x >> 2);
-        const bool on = o < n_out;
-        const int8_t *q = xp_q + static_cast<size_t>(on ? o : 0) * di;
+    // x_proj: a warp per output row, lanes over 4-channel groups (coalesced
+    // weight rows, consecutive float4 of xc)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool vec = (di % 4) == 0 && (reinterpret_cast<uintptr_t>(xp_q) & 3) == 0;
+    for (int o = warp; o < n_out; o += kConvXThreads / 32) {
+        const int8_t *q = xp_q + static_cast<size_t>(o) * di;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (!on) {
-        } else if (vec) {
-            const int quarter = di / 16;  // 4-channel groups per quarter
-            const int *qw = reinterpret_cast<const int *>(q) + part * quarter;
-            const float4 *x4 = reinterpret_cast<const float4 *>(xcs) + part * quarter;
-#pragma unroll 8
-            for (int i = 0; i < quarter; ++i) {
-                const int wv = qw[i];
-                const float4 xv = x4[i];
-                acc[0] = fmaf(static_cast<float>(static_cast<int8_t>(wv & 0xff)), xv.x, acc[0]);
-                acc[1] = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 8) & 0xff)), xv.y, acc[1]);
-                acc[2] = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 16) & 0xff)), xv.z, acc[2]);
-                acc[3] = fmaf(static_cast<float>(static_cast<int8_t>((wv >> 24) & 0xff)), xv.w, acc[3]);
+        if (vec) {
+            const int *qw = reinterpret_cast<const int *>(q);
+            const float4 *x4 = reinterpret_cast<const float4 *>(xcs);
+#pragma unroll 4
+            for (int c4 = lane; c4 < di / 4; c4 += 32) {
+                const float4 wv = i8x4_to_f32x4(qw[c4]);
+                const float4 xv = x4[c4];
+                acc[0] = fmaf(wv.x, xv.x, acc[0]);
+                acc[1] = fmaf(wv.y, xv.y, acc[1]);
+                acc[2] = fmaf(wv.z, xv.z, acc[2]);
+                acc[3] = fmaf(wv.w, xv.w, acc[3]);
             }
         } else {
 #pragma unroll 4
-            for (int c = part; c < di; c += 4)
-                acc[(c >> 2) & 3] = fmaf(static_cast<float>(q[c]), xcs[c], acc[(c >> 2) & 3]);
+            for (int c = lane; c < di; c += 32)
+                acc[c & 3] = fmaf(static_cast<float>(q[c]), xcs[c], acc[c & 3]);
         }
         float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-        if (on && part == 0)
+#pragma unroll
+        for (int off = 16; off; off >>= 1)
+            sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane == 0)
             dbc[static_cast<size_t>(m) * ld_dbc + o] = sum * xp_s[o];
     }
 }
@@ -272,11 +282,15 @@ __global__ void __launch_bounds__(kGemmThreads) q8_gemm_kernel(const Q8GemmArgs 
                 }
                 if (n < a.N) {
                     const uint2 q = *reinterpret_cast<const uint2 *>(a.wq + static_cast<size_t>(n) * a.K + k);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        wo[e] = static_cast<float>(static_cast<int8_t>((q.x >> (8 * e)) & 0xffu));
-                        wo[4 + e] = static_cast<float>(static_cast<int8_t>((q.y >> (8 * e)) & 0xffu));
-                    }
+                    const float4 w0 = i8x4_to_f32x4(static_cast<int>(q.x)), w1 = i8x4_to_f32x4(static_cast<int>(q.y));
+                    wo[0] = w0.x;
+                    wo[1] = w0.y;
+                    wo[2] = w0.z;
+                    wo[3] = w0.w;
+                    wo[4] = w1.x;
+                    wo[5] = w1.y;
+                    wo[6] = w1.z;
+                    wo[7] = w1.w;
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e)

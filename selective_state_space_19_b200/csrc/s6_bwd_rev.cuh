@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(kScanBlock, 1)
 
     if (warp == kConsumerWarps) {
         // =========================================================== producer
+        // (its waits sleep between polls, leaving the issue slots to the consumers)
         if (lane == 0) {
             prefetch_tensormap(&tm_x);
             prefetch_tensormap(&tm_dt);
@@ -191,7 +192,7 @@ __global__ void __launch_bounds__(kScanBlock, 1)
             if (c >= kRevStages) {
                 bool got = true;
                 if (lane == 0)
-                    got = mbar_wait_bounded(&sm.empty[s], ((c / kRevStages) - 1) & 1, kWaitPolls);
+                    got = mbar_wait_sleep_bounded(&sm.empty[s], ((c / kRevStages) - 1) & 1, kSleepPolls, kSleepNs);
                 ok = __shfl_sync(full, got ? 1 : 0, 0) != 0;
                 if (!ok && lane == 0)
                     raise_device_error(1u);
@@ -261,15 +262,33 @@ __global__ void __launch_bounds__(kScanBlock, 1)
             // B / C rows to float32 once the tile has landed, then the stage is ready
             bool got = true;
             if (lane == 0)
-                got = mbar_wait_bounded(&sm.full[s], (c / kRevStages) & 1, kWaitPolls);
+                got = mbar_wait_sleep_bounded(&sm.full[s], (c / kRevStages) & 1, kSleepPolls, kSleepNs);
             got = __shfl_sync(full, got ? 1 : 0, 0) != 0;
             if (!got && lane == 0)
                 raise_device_error(1u);
-            for (int i = lane; i < 2 * KC * 16; i += 32) {
-                const int which = i / (KC * 16);
-                const int rem = i - which * (KC * 16);
-                const IO *src = which ? &sm.craw[s].v[0][rem] : &sm.braw[s].v[0][rem];
-                (&sm.bc[s][0][0][0])[(rem / 16) * 32 + which * 16 + (rem % 16)] = got ? tr::to_f(*src) : 0.0f;
+            {
+                // each step fills one 512-byte group of bc (4 tokens x B|C x 16
+                // states), lane l its bytes [16 l, 16 l + 16): token l / 8 of the
+                // group, B or C by bit 2, states 4 (l & 3) .. +3
+                const int which = (lane >> 2) & 1;
+                const int n4 = (lane & 3) * 4;
+                const int tl = lane >> 3;
+                const IO *src = (which ? &sm.craw[s].v[0][0] : &sm.braw[s].v[0][0]) + tl * 16 + n4;
+                float *dst = &sm.bc[s][tl][which][n4];
+#pragma unroll
+                for (int i = 0; i < KC / 4; ++i) {
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (got) {
+                        if constexpr (sizeof(IO) == 2) {
+                            const uint2 r = *reinterpret_cast<const uint2 *>(src + i * 64);
+                            v = make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u),
+                                            __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
+                        } else {
+                            v = *reinterpret_cast<const float4 *>(src + i * 64);
+                        }
+                    }
+                    *reinterpret_cast<float4 *>(dst + i * 128) = v;
+                }
             }
             __syncwarp();
             if (lane == 0)

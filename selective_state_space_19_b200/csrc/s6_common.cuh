@@ -249,6 +249,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread may sleep up to `ns`
+// nanoseconds (or until the phase completes) instead of returning at once, so a
+// warp that waits long issues few instructions.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait with suspend hints; at most `limit` polls of at most `ns` each.
+__device__ __forceinline__ bool mbar_wait_sleep_bounded(uint64_t *bar, uint32_t parity, uint32_t limit, uint32_t ns) {
+    for (uint32_t i = 0; i < limit; ++i)
+        if (mbar_try_wait_sleep(bar, parity, ns))
+            return true;
+    return false;
+}
+
 // Bounded wait on an mbarrier phase.  Returns false after `limit` polls (each
 // try_wait may itself suspend the thread for a short, hardware-chosen time).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint32_t limit) {

@@ -191,13 +191,20 @@ __device__ __forceinline__ UnitPos unit_pos(int u, const ScanArgs &a) {
 }
 
 constexpr uint32_t kWaitPolls = 1u << 24;
+// sleeping waits: at most kSleepPolls polls of at most kSleepNs each (about 2 s)
+constexpr uint32_t kSleepPolls = 1u << 21;
+constexpr uint32_t kSleepNs = 1000u;
 
 // EXT: 0 the plain scan; 1 the extended scan, which may start from a given
 // state (h_init, conv_hist) and may take the associative split; 2 the
 // extended scan in checkpoint mode for the backward (N = 16 only).  Separate
 // instantiations, so that each one carries only its own code.
+//
+// Registers: two CTAs of kScanBlock threads per SM allow 200 per thread; a
+// cap of 168 measured 0.8 % faster on the long-sequence workload than the
+// allocator's own choice under that bound (165), and leaves the same two CTAs.
 template <typename IO, int NS, int TPC, int T, int STAGES, bool CONV, int MODE, int EXT>
-__global__ void __launch_bounds__(kScanBlock, 2)
+__global__ void __maxnreg__(168)
     s6_scan_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                    const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
                    const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -235,6 +242,9 @@ __global__ void __launch_bounds__(kScanBlock, 2)
 
     if (warp == kConsumerWarps) {
         // =========================================================== producer
+        // Its waits sleep between polls (kSleepNs): this warp shares an SM
+        // sub-partition with consumer warps, and a spinning wait would take
+        // their issue slots.
         if (lane == 0) {
             prefetch_tensormap(&tm_x);
             if (!CONSTD)
@@ -255,7 +265,7 @@ __global__ void __launch_bounds__(kScanBlock, 2)
             __syncwarp();  // lane 0's metadata write is visible to the warp
             bool got = true;
             if (lane == 0)
-                got = mbar_wait_bounded(&sm.full[sp], (cc / STAGES) & 1, kWaitPolls);
+                got = mbar_wait_sleep_bounded(&sm.full[sp], (cc / STAGES) & 1, kSleepPolls, kSleepNs);
             got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
             if (!got) {
                 if (lane == 0)
@@ -279,6 +289,44 @@ __global__ void __launch_bounds__(kScanBlock, 2)
                 fence_proxy_async_smem();  // before the stage is refilled by the tensor unit
             }
             constexpr int kSlots = 2 * T * NS;
+            if constexpr (NS == 16 && T % 4 == 0) {
+                if (got && a.bc_tma && a.N == NS) {
+                    // Whole rows.  This warp shares an SM sub-partition with
+                    // consumer warps, so the copy is kept to a few instructions a
+                    // value: each step fills one 512-byte group of bc (4 tokens x
+                    // B|C x 16 states), lane l its bytes [16 l, 16 l + 16) -- token
+                    // l / 8 of the group, B or C by bit 2, states 4 (l & 3) .. +3 --
+                    // with every address a per-lane base plus a constant.
+                    const int which = (lane >> 2) & 1;
+                    const int n4 = (lane & 3) * 4;
+                    const int tl = lane >> 3;
+                    const IO *src = (which ? &sm.craw[sp].v[0][0] : &sm.braw[sp].v[0][0]) + tl * NS + n4;
+                    float *dst = &sm.bc[sp][tl][which][n4];
+                    auto row4 = [&](int i) {
+                        if constexpr (sizeof(IO) == 2) {
+                            const uint2 r = *reinterpret_cast<const uint2 *>(src + i * 4 * NS);
+                            return make_float4(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u),
+                                               __uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
+                        } else {
+                            return *reinterpret_cast<const float4 *>(src + i * 4 * NS);
+                        }
+                    };
+                    if (m.z == T) {
+#pragma unroll
+                        for (int i = 0; i < T / 4; ++i)
+                            *reinterpret_cast<float4 *>(dst + i * 4 * 2 * NS) = row4(i);
+                    } else {
+                        // a partial chunk: rows past its tokens are zeroed
+                        for (int i = 0; i < T / 4; ++i)
+                            *reinterpret_cast<float4 *>(dst + i * 4 * 2 * NS) =
+                                (4 * i + tl < m.z) ? row4(i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&sm.ready[sp]);
+                    return;
+                }
+            }
             if (got && a.bc_tma && a.N == NS) {
                 // whole rows: four values per lane step
                 for (int j = lane; j < kSlots / 4; j += 32) {
@@ -336,7 +384,7 @@ __global__ void __launch_bounds__(kScanBlock, 2)
             if (c >= STAGES) {
                 bool got = true;
                 if (lane == 0)
-                    got = mbar_wait_bounded(&sm.empty[s], ((c / STAGES) - 1) & 1, kWaitPolls);
+                    got = mbar_wait_sleep_bounded(&sm.empty[s], ((c / STAGES) - 1) & 1, kSleepPolls, kSleepNs);
                 got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
                 if (!got) {
                     if (lane == 0)
@@ -506,14 +554,14 @@ __global__ void __launch_bounds__(kScanBlock, 2)
     // MUFU pipe is fed while the state arithmetic proceeds.
     f2_t ab[NP];
     auto decays = [&](float delta) {
-        if constexpr (CONSTD)
-            return;  // the decays are the constants in A2p
-        const f2_t dd = f2_pack(delta, delta);
+        if constexpr (!CONSTD) {  // the constant cell's decays are the constants in A2p
+            const f2_t dd = f2_pack(delta, delta);
 #pragma unroll
-        for (int q = 0; q < NP; ++q) {
-            float d0, d1;
-            f2_unpack(f2_mul(dd, A2p[q]), d0, d1);
-            ab[q] = f2_pack(ex2_approx(d0), ex2_approx(d1));
+            for (int q = 0; q < NP; ++q) {
+                float d0, d1;
+                f2_unpack(f2_mul(dd, A2p[q]), d0, d1);
+                ab[q] = f2_pack(ex2_approx(d0), ex2_approx(d1));
+            }
         }
     };
     auto update_pipe = [&](const float(*bcrow)[NS], float u, float delta, float delta_next, auto next_tag) -> float {
