@@ -1179,18 +1179,24 @@ int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x
     float *g = dbc + static_cast<size_t>(Bt) * l_dbc;
     const int64_t sms = device_sm_count();
     const unsigned mt = static_cast<unsigned>((Bt + s6::kGemmBM - 1) / s6::kGemmBM);
-    // a product Y = X W^T over the whole batch; the reduction is split across
-    // blocks (atomic adds into Y) until there are about two blocks per SM
-    // (accumulate: Y += the product, Y already holding what it should be added to)
+    // a product over the whole batch, Y = X W^T (add: Y += X W^T).  The
+    // reduction is split across blocks (atomic adds; a Y that is overwritten is
+    // zeroed first) until there are about four blocks per SM: the products are
+    // short, and more blocks hide more of their load latency.
     auto gemm = [&](const float *X, int ldx, int64_t n_out, int64_t k, const int8_t *wq, const float *ws, float *Y,
                     int ldy, bool add) -> int {
         const int64_t tiles = ((n_out + s6::kGemmBN - 1) / s6::kGemmBN) * mt;
-        int64_t sp = add ? (4 * sms + tiles - 1) / tiles : 1;
+        int64_t sp = (4 * sms + tiles - 1) / tiles;
         const int64_t max_sp = (k + s6::kGemmBK - 1) / s6::kGemmBK;
         if (sp > max_sp)
             sp = max_sp;
         if (sp < 1)
             sp = 1;
+        if (sp > 1 && !add) {
+            if (cudaMemset2DAsync(Y, sizeof(float) * ldy, 0, sizeof(float) * n_out, Bt, s) != cudaSuccess)
+                return S6_ERR_CUDA;
+            add = true;
+        }
         const int64_t ks = round_up(static_cast<size_t>((k + sp - 1) / sp), s6::kGemmBK);
         s6::Q8GemmArgs ga;
         ga.M = static_cast<int>(Bt);
@@ -1211,6 +1217,18 @@ int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x
         int dev = 0;
         if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
             return S6_ERR_CUDA;
+        if (vec && k % 16 == 0 && aligned16(wq)) {
+            // the tensor-core form (16-byte weight rows)
+            static int opted_tc[64] = {};
+            if (!opted_tc[dev]) {
+                if (cudaFuncSetAttribute(s6::q8_tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(s6::kTcSmem)) != cudaSuccess)
+                    return S6_ERR_CUDA;
+                opted_tc[dev] = 1;
+            }
+            s6::q8_tc_gemm_kernel<<<grid, s6::kTcThreads, s6::kTcSmem, s>>>(ga);
+            return cudaGetLastError() == cudaSuccess ? S6_OK : S6_ERR_CUDA;
+        }
         if (!opted[dev][vec]) {
             const cudaError_t e =
                 vec ? cudaFuncSetAttribute(s6::q8_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1232,11 +1250,7 @@ int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x
         x, w->ln_w, w->ln_b, hn, static_cast<int>(Bt), static_cast<int>(dm), dims->eps);
     if (cudaGetLastError() != cudaSuccess)
         return S6_ERR_CUDA;
-    // in_proj also splits its reduction (atomic adds into a zeroed xz): its 2 di x Bt
-    // outputs alone give too few blocks to hide the load latency
-    if (cudaMemsetAsync(xz, 0, sizeof(float) * Bt * l_xz, s) != cudaSuccess)
-        return S6_ERR_CUDA;
-    rc = gemm(hn, static_cast<int>(dm), 2 * di, dm, w->in_q, w->in_s, xz, static_cast<int>(l_xz), true);
+    rc = gemm(hn, static_cast<int>(dm), 2 * di, dm, w->in_q, w->in_s, xz, static_cast<int>(l_xz), false);
     if (rc != S6_OK)
         return rc;
     // 2. conv + SiLU (history shifted) and x_proj -> dt | B | C, a block per sequence

@@ -389,6 +389,172 @@ __global__ void __launch_bounds__(kGemmThreads) q8_gemm_kernel(const Q8GemmArgs 
     }
 }
 
+// ------------------------------------------ int8 products on the tensor cores
+// The same product, Y[m][n] (+)= ws[n] * sum_k wq[n][k] X[m][k], with
+// mma.sync m16n8k8 in TF32.  An int8 weight is exact in TF32; an activation
+// is split as x = hi + lo, both TF32 (hi = x rounded to TF32, lo = the rest
+// rounded again), so hi*w + lo*w carries x*w to about 2^-22 of its size -- the
+// float32 product, from two tensor-core products instead of one.
+//
+// A 64 x 64 output tile per block of four warps, each warp 32 x 32 (2 x 4
+// m16n8 tiles); 32-wide K slices staged in shared memory as (hi, lo, w) rows
+// with a 4-float pad, which puts the eight rows x four columns of a fragment
+// load on 32 distinct banks; the next slice is read into registers while the
+// current one is multiplied.  Needs the VEC layout of q8_gemm_kernel and
+// K % 16 == 0 (16-byte weight loads).
+constexpr int kTcThreads = 128;
+constexpr int kTcLD = kGemmBK + 4;
+constexpr size_t kTcSmem = 2 * 3 * 64 * kTcLD * sizeof(float);
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kTcThreads) q8_tc_gemm_kernel(const Q8GemmArgs a) {
+    constexpr int BK = kGemmBK, LD = kTcLD;
+    extern __shared__ __align__(16) float tc_smem[];
+    // [buf][0: hi, 1: lo, 2: w][row][LD]
+    auto sm = [&](int buf, int part, int row, int col) -> float * {
+        return tc_smem + ((buf * 3 + part) * 64 + row) * LD + col;
+    };
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int wm = (warp >> 1) * 32, wn = (warp & 1) * 32;
+    const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+    const int kb = blockIdx.z * a.k_split;
+    const int ke = min(a.K, kb + a.k_split);
+    // staging: thread -> tile row tid / 2, 16 consecutive k from (tid & 1) * 16
+    const int lr = tid >> 1, lk = (tid & 1) * 16;
+    float4 xr[4];
+    int4 wr;
+    auto fetch = [&](int k0) {
+        const int m = m0 + lr, n = n0 + lr, k = k0 + lk;
+        const bool kin = k + 16 <= ke;  // slices are whole (K, k_split multiples of 16)
+        if (m < a.M && kin) {
+            const float4 *src = reinterpret_cast<const float4 *>(a.x + static_cast<size_t>(m) * a.ldx + k);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                xr[q] = src[q];
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                xr[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        wr = (n < a.N && kin) ? *reinterpret_cast<const int4 *>(a.wq + static_cast<size_t>(n) * a.K + k)
+                              : make_int4(0, 0, 0, 0);
+    };
+    auto stage = [&](int buf) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float v[4] = {xr[q].x, xr[q].y, xr[q].z, xr[q].w};
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                hi[e] = to_tf32(v[e]);
+                lo[e] = to_tf32(v[e] - __uint_as_float(hi[e]));
+            }
+            *reinterpret_cast<uint4 *>(sm(buf, 0, lr, lk + 4 * q)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(sm(buf, 1, lr, lk + 4 * q)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        const int wv[4] = {wr.x, wr.y, wr.z, wr.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<float4 *>(sm(buf, 2, lr, lk + 4 * q)) = i8x4_to_f32x4(wv[q]);
+    };
+
+    float acc[2][4][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[i][j][e] = 0.f;
+
+    int buf = 0;
+    if (kb < ke) {
+        fetch(kb);
+        stage(0);
+    }
+    __syncthreads();
+    for (int k0 = kb; k0 < ke; k0 += BK) {
+        const bool more = k0 + BK < ke;
+        if (more)
+            fetch(k0 + BK);  // in flight while this slice is multiplied
+#pragma unroll
+        for (int kk = 0; kk < BK; kk += 8) {
+            uint32_t ah[2][4], al[2][4], bw[4][2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int r = wm + 16 * i + g;
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    const float *h = sm(buf, p, r, kk + t);
+                    uint32_t(&f)[4] = p ? al[i] : ah[i];
+                    f[0] = __float_as_uint(h[0]);
+                    f[1] = __float_as_uint(h[8 * LD]);
+                    f[2] = __float_as_uint(h[4]);
+                    f[3] = __float_as_uint(h[8 * LD + 4]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float *wp = sm(buf, 2, wn + 8 * j + g, kk + t);
+                bw[j][0] = __float_as_uint(wp[0]);
+                bw[j][1] = __float_as_uint(wp[4]);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    mma_tf32(acc[i][j], al[i], bw[j][0], bw[j][1]);
+                    mma_tf32(acc[i][j], ah[i], bw[j][0], bw[j][1]);
+                }
+        }
+        if (more) {
+            // the other buffer was last read before the previous barrier
+            stage(buf ^ 1);
+            __syncthreads();
+            buf ^= 1;
+        }
+    }
+
+    // accumulator (i, j): rows wm + 16 i + g (+8), columns wn + 8 j + 2 t (+1)
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int n = n0 + wn + 8 * j + 2 * t;
+#pragma unroll
+            for (int hrow = 0; hrow < 2; ++hrow) {
+                const int m = m0 + wm + 16 * i + g + 8 * hrow;
+                if (m >= a.M)
+                    continue;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    if (n + e >= a.N)
+                        continue;
+                    const float out = acc[i][j][2 * hrow + e] * a.ws[n + e];
+                    float *dst = a.y + static_cast<size_t>(m) * a.ldy + n + e;
+                    if (a.accumulate)
+                        atomicAdd(dst, out);
+                    else
+                        *dst = out;
+                }
+            }
+        }
+}
+
 // ------------------------------------------------------------ the recurrence
 struct BlockSsmArgs {
     int Bt, di, N, R;
