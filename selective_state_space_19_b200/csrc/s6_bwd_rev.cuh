@@ -68,7 +68,7 @@ struct RevSmem {
     Tile<IO, 1, kRevChunk * 16> braw[kRevStages];
     Tile<IO, 1, kRevChunk * 16> craw[kRevStages];
     float bc[kRevStages][kRevChunk][2][16];         // B | C rows in float32
-    float4 hbuf[kConsumerWarps][kRevChunk][2][32];  // per warp: each lane's 8 states after token j
+    float4 hbuf[kConsumerWarps][kRevChunk + 1][2][32];  // per warp: each lane's 8 states before token j (slot j)
     float4 tab[kConsumerWarps][kRevChunk][16];      // per warp: (Delta, u, ds, dy SiLU'(z)) of its channels
     float acc[2][kRevChunk][32];                    // dB | dC of the tile's channels, per sub-chunk parity
     int4 meta[kRevStages];                          // {unit, t0, tcount, flags}
@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(kScanBlock, 1)
             float g = 1.0f, gp = 0.0f;
             if (a.has_z) {
                 const float zv = ld(zs, j);
-                const float sz = rcp_newton(1.0f + ex2_approx(fminf(-zv * kLog2e, 120.0f)));  // sigmoid(z)
+                const float sz = rcp_approx(1.0f + ex2_approx(fminf(-zv * kLog2e, 120.0f)));  // sigmoid(z)
                 g = zv * sz;                          // SiLU(z)
                 gp = sz * fmaf(zv, 1.0f - sz, 1.0f);  // SiLU'(z)
             }
@@ -467,6 +467,8 @@ __global__ void __launch_bounds__(kScanBlock, 1)
             const int tc = FULL ? KC : tcount;
             // ---- 2. recompute the sub-chunk forward from the checkpoint; keep every state
             {
+                hb[0][0][lane] = ck0;
+                hb[0][1][lane] = ck1;
                 f2_t h[4] = {f2_pack(ck0.x, ck0.y), f2_pack(ck0.z, ck0.w), f2_pack(ck1.x, ck1.y), f2_pack(ck1.z, ck1.w)};
 #pragma unroll 2
                 for (int j = 0; j < tc; ++j) {
@@ -494,26 +496,22 @@ __global__ void __launch_bounds__(kScanBlock, 1)
                     f2_unpack(h[1], a2, a3);
                     f2_unpack(h[2], a4, a5);
                     f2_unpack(h[3], a6, a7);
-                    hb[j][0][lane] = make_float4(a0, a1, a2, a3);
-                    hb[j][1][lane] = make_float4(a4, a5, a6, a7);
+                    hb[j + 1][0][lane] = make_float4(a0, a1, a2, a3);
+                    hb[j + 1][1][lane] = make_float4(a4, a5, a6, a7);
                 }
             }
             __syncwarp();
 
             // ---- 3. walk the sub-chunk back
             // h_t of the token being walked back; h_{t-1} becomes the next token's h_t
-            float4 h0 = hb[tc - 1][0][lane], h1 = hb[tc - 1][1][lane];
+            float4 h0 = hb[tc][0][lane], h1 = hb[tc][1][lane];
 #pragma unroll 2
             for (int j = tc - 1; j >= 0; --j) {
                 const float4 du = tb[j][cw];
                 const float delta = du.x, u = du.y, ds = du.z, dygp = du.w;
                 // softplus'(v) = sigmoid(v) = 1 - e^-Delta (Delta = softplus(v))
                 const float sig_v = 1.0f - ex2_approx(-delta * kLog2e);
-                float4 p0 = ck0, p1 = ck1;  // h_{t-1}
-                if (j > 0) {
-                    p0 = hb[j - 1][0][lane];
-                    p1 = hb[j - 1][1][lane];
-                }
+                const float4 p0 = hb[j][0][lane], p1 = hb[j][1][lane];  // h_{t-1}
                 const f2_t ht[4] = {f2_pack(h0.x, h0.y), f2_pack(h0.z, h0.w), f2_pack(h1.x, h1.y), f2_pack(h1.z, h1.w)};
                 const f2_t hp[4] = {f2_pack(p0.x, p0.y), f2_pack(p0.z, p0.w), f2_pack(p1.x, p1.y), f2_pack(p1.z, p1.w)};
                 const ulonglong2 B01 = *reinterpret_cast<const ulonglong2 *>(&bc[j][0][n0]);
@@ -599,13 +597,10 @@ __global__ void __launch_bounds__(kScanBlock, 1)
                 }
                 dDa = fmaf(ds, u, dDa);
                 dba += dv;
-                if (live && sub == (j & 1)) {
-                    const size_t o = (static_cast<size_t>(b) * a.L + t0 + j) * a.d + ch;
-                    a.du[o] = dxo;
-                    a.ddt[o] = dv;
-                    if (a.has_z)
-                        a.dz[o] = dygp * s_tot;
-                }
+                // the token's outputs, written out by the warp after the walk (this
+                // tab row is not read again)
+                if (sub == 0)
+                    tb[j][cw] = make_float4(dxo, dv, dygp * s_tot, 0.f);
                 // dB, dC of token t0 + j summed over the warp's channels, then the CTA's
                 const float r = reduce_scatter16(vB, vC, lane);
                 atomicAdd(accp + j * 32 + o_lane, r);
@@ -617,6 +612,23 @@ __global__ void __launch_bounds__(kScanBlock, 1)
             phases(std::true_type{});
         else
             phases(std::false_type{});
+
+        // du, ddt, dz of the sub-chunk from the tab rows: lanes 0-15 one token,
+        // 16-31 the next, each a channel -- 64-byte runs per token and output
+        __syncwarp();
+        {
+            const int wc = tile * 64 + warp * 16 + (lane & 15);
+            if (wc < a.d) {
+                for (int j = lane >> 4; j < tcount; j += 2) {
+                    const float4 v = tb[j][lane & 15];
+                    const size_t o = (static_cast<size_t>(b) * a.L + t0 + j) * a.d + wc;
+                    a.du[o] = v.x;
+                    a.ddt[o] = v.y;
+                    if (a.has_z)
+                        a.dz[o] = v.z;
+                }
+            }
+        }
 
         // release the stage (its tiles are no longer read)
         __syncwarp();
