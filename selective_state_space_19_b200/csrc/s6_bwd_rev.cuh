@@ -441,21 +441,32 @@ __global__ void __launch_bounds__(kScanBlock, 1)
         };
 
         // ---- 1. the per-token scalars of the sub-chunk, once per (token, channel):
-        // each thread of a pair takes half of the tokens
-        for (int j = sub; j < tcount; j += 2) {
-            const float v = ld(dts, j) + bias;
-            const float e = ex2_approx(-fabsf(v) * kLog2e);
-            const float delta = fmaf(e, log1p_over_x_01(e), fmaxf(v, 0.0f));  // softplus(v)
-            const float u = CONV ? silu_fast(pre_at(j)) : ld(xs, j);
-            const float dyv = ld(dys, j);
-            float g = 1.0f, gp = 0.0f;
+        // each thread of a pair takes half of the tokens, two at a time (j and
+        // j + 2) in packed arithmetic -- the forward's own softplus and SiLU
+        for (int j = sub; j < tcount; j += 4) {
+            const int j2 = min(j + 2, KC - 1);  // a partial sub-chunk's spare lane reads a row it does not store
+            const f2_t v2 = f2_add(f2_pack(ld(dts, j), ld(dts, j2)), f2_pack(bias, bias));
+            const f2_t d2 = f2_softplus_fast(v2);
+            const f2_t u2 = CONV ? f2_silu_fast(f2_pack(pre_at(j), pre_at(j2))) : f2_pack(ld(xs, j), ld(xs, j2));
+            const f2_t dy2 = f2_pack(ld(dys, j), ld(dys, j2));
+            f2_t g2 = f2_pack(1.0f, 1.0f), gp2 = f2_pack(0.0f, 0.0f);
             if (a.has_z) {
-                const float zv = ld(zs, j);
-                const float sz = rcp_approx(1.0f + ex2_approx(fminf(-zv * kLog2e, 120.0f)));  // sigmoid(z)
-                g = zv * sz;                          // SiLU(z)
-                gp = sz * fmaf(zv, 1.0f - sz, 1.0f);  // SiLU'(z)
+                const float za = ld(zs, j), zb = ld(zs, j2);
+                // sigmoid(z), SiLU(z) = z sigmoid(z), SiLU'(z) = sigmoid(z) (1 + z (1 - sigmoid(z)))
+                const f2_t sz = f2_pack(rcp_approx(1.0f + ex2_approx(fminf(-za * kLog2e, 120.0f))),
+                                        rcp_approx(1.0f + ex2_approx(fminf(-zb * kLog2e, 120.0f))));
+                const f2_t z2 = f2_pack(za, zb);
+                g2 = f2_mul(z2, sz);
+                gp2 = f2_mul(sz, f2_fma(z2, f2_sub(f2_pack(1.0f, 1.0f), sz), f2_pack(1.0f, 1.0f)));
             }
-            tb[j][cw] = make_float4(delta, u, dyv * g, dyv * gp);
+            float da, db, ua, ub, ga, gb, pa, pb;
+            f2_unpack(d2, da, db);
+            f2_unpack(u2, ua, ub);
+            f2_unpack(f2_mul(dy2, g2), ga, gb);
+            f2_unpack(f2_mul(dy2, gp2), pa, pb);
+            tb[j][cw] = make_float4(da, ua, ga, pa);
+            if (j + 2 < tcount)
+                tb[j + 2][cw] = make_float4(db, ub, gb, pb);
         }
         __syncwarp();
 
