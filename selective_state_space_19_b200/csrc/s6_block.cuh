@@ -12,12 +12,15 @@
 //     x      += out_proj(y SiLU(z))              di -> dm
 //
 // Kernels: LayerNorm (a warp per row); the in_proj product; the conv + SiLU
-// with the history shifted in place; the x_proj product; dt_proj fused with the
-// recurrence and the gate (a thread per (sequence, channel)); the out_proj
-// product added into x.  The products (q8_gemm_kernel) are float32 on the CUDA
-// cores: int8 weight rows converted exactly when staged in shared memory, the
-// row scale applied to the finished sum, the reduction split across blocks
-// with atomic adds where the output tile count alone would not fill the GPU.
+// with the history shifted in place, and the x_proj product (a block per
+// sequence); dt_proj fused with the recurrence and the gate (a thread per
+// (sequence, channel)); the out_proj product added into x.  The in_proj and
+// out_proj products run on the tensor cores (q8_tc_gemm_kernel: TF32 with the
+// activations split into two terms, float32-accurate) and otherwise on the
+// CUDA cores (q8_gemm_kernel); both convert the int8 weight rows exactly when
+// staging them in shared memory, apply the row scale to the finished sum and
+// split the reduction across blocks with atomic adds when the output tiles
+// alone would not fill the GPU.
 #pragma once
 
 #include "s6_common.cuh"
