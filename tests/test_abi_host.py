@@ -146,6 +146,45 @@ def test_from_state_and_backward_host_checks(lib):
     assert cbwd(conv_w=P(2)) == S.S6_ERR_ALIGNMENT
 
 
+def test_diag_and_block_host_checks(lib):
+    """The constant-decay cell and the decode block reject bad arguments before
+    any device call."""
+    import selective_state_space_19_b200 as S
+    P = ctypes.c_void_p
+    ok = P(16)
+
+    def diag(src=S.S6_DECAY_CONST, dims=None, w=ok):
+        return lib.s6_diag_recurrence_fwd(ctypes.byref(dims or _dims()), src, ok, None, None, None, w, ok, ok, ok,
+                                          None, None, ok, None, None)
+    assert diag(src=5) == S.S6_ERR_INVALID_ARG
+    assert diag(w=None) == S.S6_ERR_INVALID_ARG                       # the decays are required
+    assert diag(dims=_dims(d_state=17)) == S.S6_ERR_UNSUPPORTED
+    assert diag(w=P(2)) == S.S6_ERR_ALIGNMENT                         # float32 decays
+    assert diag(dims=_dims(batch=0)) == S.S6_OK
+
+    def block(**over):
+        dims = dict(batch=4, d_model=64, d_inner=128, d_state=16, dt_rank=8, conv_width=4, eps=1e-5)
+        ptrs = {k: 16 for k in S.BLOCK_WEIGHT_KEYS}
+        ptrs["conv_b"] = None
+        x = over.pop("x", 16)
+        for k in list(over):
+            if k in ptrs:
+                ptrs[k] = over.pop(k)
+        dims.update(over)
+        w = S.BlockWeights(**{k: v for k, v in ptrs.items()})
+        return lib.s6_block_step(ctypes.byref(S.BlockDims(**dims)), ctypes.byref(w), P(x), ok, ok, None)
+    assert lib.s6_block_step(None, None, ok, ok, ok, None) == S.S6_ERR_INVALID_ARG
+    assert block(d_state=17) == S.S6_ERR_UNSUPPORTED
+    assert block(conv_width=5) == S.S6_ERR_UNSUPPORTED
+    assert block(dt_rank=0) == S.S6_ERR_INVALID_ARG
+    assert block(eps=float("nan")) == S.S6_ERR_INVALID_ARG
+    assert block(in_q=None) == S.S6_ERR_INVALID_ARG                   # every weight but conv_b is required
+    assert block(x=None) == S.S6_ERR_INVALID_ARG
+    assert block(A_log=20) == S.S6_ERR_ALIGNMENT                      # N = 16 rows move as 16-byte vectors
+    assert block(ln_w=2) == S.S6_ERR_ALIGNMENT
+    assert block(batch=0) == S.S6_OK                                  # nothing to do, nothing touched
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     import selective_state_space_19_b200 as S
