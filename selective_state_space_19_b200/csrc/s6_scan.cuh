@@ -830,17 +830,21 @@ __global__ void __maxnreg__(168)
                             sdel += c1s.w;
                     }
                     // each thread finishes its own tokens: own partial + the partner's
-                    const float ra = __shfl_xor_sync(0xffffffffu, half ? acc0 : acc1, 1);
-                    const float rb = __shfl_xor_sync(0xffffffffu, half ? acc2 : acc3, 1);
-                    float ua, ub, ga, gb;
-                    f2_unpack(u2c, ua, ub);
-                    f2_unpack(g2c, ga, gb);
-                    const float ya = fmaf(Dd, ua, (half ? acc1 : acc0) + ra) * ga;
-                    const float yb = fmaf(Dd, ub, (half ? acc3 : acc2) + rb) * gb;
-                    if (FULL || p + half < tc)
-                        yw[p + half][cw] = tr::from_f(ya);
-                    if (FULL || p + 2 + half < tc)
-                        yw[p + 2 + half][cw] = tr::from_f(yb);
+                    // (checkpoint mode writes no y, so the readout, the gate and z
+                    // are not computed at all there)
+                    if constexpr (!CKPT) {
+                        const float ra = __shfl_xor_sync(0xffffffffu, half ? acc0 : acc1, 1);
+                        const float rb = __shfl_xor_sync(0xffffffffu, half ? acc2 : acc3, 1);
+                        float ua, ub, ga, gb;
+                        f2_unpack(u2c, ua, ub);
+                        f2_unpack(g2c, ga, gb);
+                        const float ya = fmaf(Dd, ua, (half ? acc1 : acc0) + ra) * ga;
+                        const float yb = fmaf(Dd, ub, (half ? acc3 : acc2) + rb) * gb;
+                        if (FULL || p + half < tc)
+                            yw[p + half][cw] = tr::from_f(ya);
+                        if (FULL || p + 2 + half < tc)
+                            yw[p + 2 + half][cw] = tr::from_f(yb);
+                    }
                     if (!LAST)
                         exchange((q + 1) & 1, u2n, d2n, c0s, c1s);
                     u2c = u2n;
