@@ -812,12 +812,13 @@ def run_ours(args):
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
                 "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16 I/O, f32 math and state",
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded numpy, long_seq recipe: x,z,B,C ~ N(0,1), dt_raw ~ 0.5 N(0,1), "
                         "dt_bias = softplus^-1(U[0.001,0.1]), A_log = log(n+1), D ~ U[0.5,1.5])",
                 "config": {"workload": f"{WORKLOAD}: Bt16 L8192 d1536 N16 K4, bf16 I/O, fp32 state, simplified "
                                        "dt*B write, fused conv4+SiLU + SiLU(z) gate, h_final",
                            "global_batch": Bt * world, "seq_len": L, "d_inner": d, "d_state": N,
+                           "io_dtype": "bf16", "state_dtype": "f32",
                            "parallelism": f"dp{world} (independent batches per GPU)",
                            "l2": "inputs larger than L2 (1.2 GB read per step), no flush"},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
