@@ -56,6 +56,15 @@ def test_block_ragged_dims():
     _run(Bt=70, dm=96, di=200, N=8, R=5, K=3, blocks=2, steps=3, seed=12)
 
 
+def test_block_single_sequence_and_tile_edges():
+    """One sequence (a single, mostly empty row tile of the products), then 65
+    sequences (one row past a tile); d_model 48 and d_inner 80 leave the
+    tensor-core products' K (48, 80) a multiple of 16 with N (160, 48) not a
+    multiple of the 64-wide output tile."""
+    _run(Bt=1, dm=48, di=80, N=16, R=4, K=4, blocks=2, steps=3, seed=15)
+    _run(Bt=65, dm=48, di=80, N=16, R=4, K=2, blocks=2, steps=2, seed=16)
+
+
 def test_block_mamba_mini_dims():
     """The Mamba-mini block (d_model 384, d_inner 1536, N 16, dt rank 24, conv 4)
     through all 6 blocks for 6 tokens, on a 16-sequence batch."""
