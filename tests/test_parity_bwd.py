@@ -16,7 +16,7 @@ import pytest
 
 from oracle import s6_oracle as O
 import s6_inputs as SI
-from s6_testutil import as_f64, dev_inputs, from_dev, note, rel_err, to_dev
+from s6_testutil import dev_inputs, note, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
