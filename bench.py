@@ -458,6 +458,51 @@ def row_scan(device, stream, pk, name, zoh=None, over=None, iters=20, label=None
     return row
 
 
+def row_random_A(device, stream, pk, inp_dev, cfg, iters=20):
+    """The headline scan with A_log drawn at random (log U[0.5, 16] per (channel,
+    state), so that no decay is a power of another) against the workload's
+    A_log = log(n + 1), alternating launches of the two on the same inputs: the
+    kernel must take the same time for both (16 live exponentials per element
+    either way)."""
+    import selective_state_space_19_b200 as S
+    import torch
+    Bt, L, d, N = cfg["Bt"], cfg["L"], cfg["d"], cfg["N"]
+    t = inp_dev
+    rng = np.random.default_rng(17)
+    a_rand = torch.from_numpy(np.log(rng.uniform(0.5, 16.0, size=(d, N))).astype(np.float32)).to(device)
+    y = torch.empty_like(t["x"])
+    h = torch.empty(Bt, d, N, device=device)
+
+    def launch(A_log):
+        S.s6_conv_scan_fwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], A_log, t["B"], t["C"], t["D"], z=t["z"],
+                           dt_bias=t["dt_bias"], zoh_mode=int(bool(cfg["zoh"])), y=y, h_final=h, stream=stream)
+
+    ms = {"default": [], "random": []}
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            launch(t["A_log"])
+            launch(a_rand)
+        for _ in range(iters):
+            for key, A_log in (("default", t["A_log"]), ("random", a_rand)):
+                s0 = torch.cuda.Event(enable_timing=True)
+                s1 = torch.cuda.Event(enable_timing=True)
+                s0.record(stream)
+                launch(A_log)
+                s1.record(stream)
+                s1.synchronize()
+                ms[key].append(s0.elapsed_time(s1))
+    assert S.s6_device_status(stream=stream, device=device) == 0
+    elems = Bt * L * d
+    md, mr = statistics.median(ms["default"]), statistics.median(ms["random"])
+    peak_ex2 = SMS * MUFU_PER_SM_CLK * pk["sm_max_mhz"] * 1e6
+    return {"workload": f"{WORKLOAD} scan with A_log ~ log U[0.5, 16] (alternating with the default A_log = "
+                        f"log(n+1) on the same inputs)",
+            "value": elems / (mr * 1e-3) / 1e9, "unit": "Gelem/s", "ms_per_launch": mr,
+            "default_A_log_ms_per_launch": md, "time_ratio_random_over_default": mr / md,
+            "roofline": {"bound": "alu", "achieved": elems * N / (mr * 1e-3) / 1e12, "peak": peak_ex2 / 1e12,
+                         "unit": "Tex2/s", "frac": elems * N / (mr * 1e-3) / peak_ex2}}
+
+
 def row_diag(device, stream, pk, inp_dev, cfg, iters=20):
     """The constant-decay cell (s6_diag_recurrence_fwd, decay 2^w per channel and
     state, write B*u, gate) on the long-sequence workload's u, z, B, C.  No
@@ -806,6 +851,7 @@ def run_ours(args):
                                                label="one long prompt, Bt1 L65536 (associative split)")
         rows["s6_step"] = row_decode(device, stream, pk)
         rows["s6_block_step"] = row_block(device, stream, pk)
+        rows["long_seq_random_A_log"] = row_random_A(device, stream, pk, t, cfg)
         rows["s6_diag_recurrence_fwd_const"] = row_diag(device, stream, pk, t, cfg)
         rows["causal_conv1d_silu_fwd"] = row_conv(device, stream, pk, t, cfg)
         rows["s6_conv_scan_fwd_from_state"] = row_prefill(device, stream, pk, t, cfg)
