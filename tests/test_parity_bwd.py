@@ -156,3 +156,38 @@ def test_bwd_unaligned_rows_take_the_simple_kernel():
     for k in ("du", "ddt", "dz", "dB", "dC", "dA_log", "dD", "ddt_bias"):
         err = rel_err(got[k].cpu().numpy().astype(np.float64), ref[k])
         assert err <= GTOL, f"{k}: {err:.3e}"
+
+
+def test_bwd_full_long_seq_workload():
+    """The backward at the long-sequence workload's full size (Bt16 L8192 d1536
+    N16, bf16 inputs, gate, simplified write), in one launch sequence as the
+    bench times it, against the oracle sequence by sequence: every element of
+    du, ddt, dz, dB and dC, and the sums over all sequences dA_log, dD and
+    ddt_bias."""
+    import torch
+    import selective_state_space_19_b200 as S
+    cfg = SI.CONFIGS["long_seq"]
+    inp = SI.scan_inputs("long_seq")
+    Bt, L, d = cfg["Bt"], cfg["L"], cfg["d"]
+    dy = SI.to_storage(np.random.default_rng(41).standard_normal((Bt, L, d)).astype(np.float32), "bf16")
+    t = dev_inputs(inp)
+    got = S.s6_scan_bwd(t["x"], t["dt"], t["A_log"], t["B"], t["C"], t["D"], to_dev(dy), z=t["z"],
+                        dt_bias=t["dt_bias"])
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    sums = {k: 0.0 for k in ("dA_log", "dD", "ddt_bias")}
+    worst = {}
+    for b in range(Bt):
+        sl = slice(b, b + 1)
+        ref = O.scan_bwd(inp["x"][sl], inp["dt"][sl], inp["A_log"], inp["B"][sl], inp["C"][sl], inp["D"], dy[sl],
+                         z=inp["z"][sl], dt_bias=inp["dt_bias"])
+        for k in ("du", "ddt", "dz", "dB", "dC"):
+            err = rel_err(got[k][b].cpu().numpy().astype(np.float64), ref[k][0])
+            worst[k] = max(worst.get(k, 0.0), err)
+        for k in sums:
+            sums[k] = sums[k] + ref[k]
+    for k in sums:
+        worst[k] = rel_err(got[k].cpu().numpy().astype(np.float64), sums[k])
+    for k, err in worst.items():
+        note(f"grad full long-seq {k} (bf16)", err)
+        assert err <= GTOL, f"{k}: max|g-ref|/(1+|ref|) = {err:.3e}"
