@@ -191,3 +191,37 @@ def test_bwd_full_long_seq_workload():
     for k, err in worst.items():
         note(f"grad full long-seq {k} (bf16)", err)
         assert err <= GTOL, f"{k}: max|g-ref|/(1+|ref|) = {err:.3e}"
+
+
+def test_conv_bwd_full_long_seq_workload():
+    """The fused backward (conv + SiLU + scan) at the long-sequence workload's
+    full size, against the oracle sequence by sequence: every element of dx,
+    ddt, dz, dB and dC, and the sums over all sequences dconv_w, dconv_b,
+    dA_log, dD and ddt_bias."""
+    import torch
+    import selective_state_space_19_b200 as S
+    cfg = SI.CONFIGS["long_seq"]
+    inp = SI.scan_inputs("long_seq")
+    Bt, L, d = cfg["Bt"], cfg["L"], cfg["d"]
+    dy = SI.to_storage(np.random.default_rng(43).standard_normal((Bt, L, d)).astype(np.float32), "bf16")
+    t = dev_inputs(inp)
+    got = S.s6_conv_scan_bwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"],
+                             to_dev(dy), z=t["z"], dt_bias=t["dt_bias"])
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    sums = {k: 0.0 for k in ("dconv_w", "dconv_b", "dA_log", "dD", "ddt_bias")}
+    worst = {}
+    for b in range(Bt):
+        sl = slice(b, b + 1)
+        ref = O.conv_scan_bwd(inp["x"][sl], inp["conv_w"], inp["conv_b"], inp["dt"][sl], inp["A_log"], inp["B"][sl],
+                              inp["C"][sl], inp["D"], dy[sl], z=inp["z"][sl], dt_bias=inp["dt_bias"])
+        for k in ("dx", "ddt", "dz", "dB", "dC"):
+            err = rel_err(got[k][b].cpu().numpy().astype(np.float64), ref[k][0])
+            worst[k] = max(worst.get(k, 0.0), err)
+        for k in sums:
+            sums[k] = sums[k] + ref[k]
+    for k in sums:
+        worst[k] = rel_err(got[k].cpu().numpy().astype(np.float64), sums[k])
+    for k, err in worst.items():
+        note(f"grad fused full long-seq {k} (bf16)", err)
+        assert err <= GTOL, f"{k}: max|g-ref|/(1+|ref|) = {err:.3e}"
