@@ -39,6 +39,22 @@ def test_conv_silu_no_bias_full_long_seq_rows():
     assert_close(as_f64(from_dev(out)), ref, "bf16", "xc")
 
 
+def test_conv_silu_full_long_seq_workload():
+    """The standalone conv at the bench row's configuration: the long-sequence
+    workload's x in full (Bt16 L8192 d1536 bf16, K=4, with bias), every
+    element, the oracle sequence by sequence."""
+    import selective_state_space_19_b200 as S
+    import torch
+    inp = SI.scan_inputs("long_seq")
+    t = dev_inputs(inp)
+    out = S.causal_conv1d_silu_fwd(t["x"], t["conv_w"], t["conv_b"])
+    torch.cuda.synchronize()
+    got = from_dev(out)
+    for b in range(inp["Bt"]):
+        ref = O.conv_silu(inp["x"][b:b + 1], inp["conv_w"], inp["conv_b"])
+        assert_close(as_f64(got[b:b + 1]), ref, "bf16", "xc full long-seq")
+
+
 # ------------------------------------------------------------ streaming step
 def _step_gpu(S, t, tok, h, cs, zoh):
     return S.s6_step(tok["x"], tok["dt"], tok["B"], tok["C"], t["A_log"], t["D"], t["conv_w"], h, cs, z_t=tok["z"],

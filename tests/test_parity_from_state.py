@@ -96,6 +96,37 @@ def test_chunked_prefill_equals_one_scan(io, Bt, d, cuts):
     assert_close(h.cpu().numpy(), rh, io, "h_final")
 
 
+def test_chunked_prefill_full_long_seq_workload():
+    """The bench's chunked-prefill row: the long-sequence workload in full
+    (Bt16 L8192 d1536 bf16) in four 2048-token parts, each from the previous
+    part's state and conv history, against one oracle scan per sequence: every
+    element of y and the final state."""
+    import selective_state_space_19_b200 as S
+    import torch
+    inp = SI.scan_inputs("long_seq")
+    Bt, L, K = inp["Bt"], inp["L"], inp["K"]
+    t = dev_inputs(inp)
+    h, hist, ys = None, None, []
+    cuts = [L * i // 4 for i in range(5)]
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        part = {k: t[k][:, lo:hi].contiguous() for k in ("x", "dt", "z", "B", "C")}
+        y, h = S.s6_conv_scan_fwd_from_state(part["x"], t["conv_w"], t["conv_b"], part["dt"], t["A_log"],
+                                             part["B"], part["C"], t["D"], z=part["z"], dt_bias=t["dt_bias"],
+                                             h_init=h, conv_hist=hist)
+        hist = t["x"][:, hi - (K - 1):hi].transpose(1, 2).contiguous()
+        ys.append(from_dev(y))
+    torch.cuda.synchronize()
+    assert S.s6_device_status() == 0
+    hg = h.cpu().numpy()
+    for b in range(Bt):
+        sl = slice(b, b + 1)
+        ry, rh = O.scan(inp["x"][sl], inp["dt"][sl], inp["A_log"], inp["B"][sl], inp["C"][sl], inp["D"],
+                        z=inp["z"][sl], dt_bias=inp["dt_bias"], conv_w=inp["conv_w"], conv_b=inp["conv_b"])
+        yb = np.concatenate([as_f64(v[b:b + 1]) for v in ys], axis=1)
+        assert_close(yb, ry, "bf16", "prefill full long-seq y")
+        assert_close(hg[b:b + 1], rh, "bf16", "prefill full long-seq h_final")
+
+
 def test_empty_sequence_returns_the_start_state():
     import selective_state_space_19_b200 as S
     import torch
