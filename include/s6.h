@@ -350,8 +350,11 @@ S6_API int s6_step(const s6_dims *dims, const float *A_log, const float *D, cons
  * N = 16).  Uses a library-owned scratch buffer for the intermediate rows
  * (xin|z, the x_proj rows, the gated readout): allocated on the first call on
  * a device, grown on demand; make that call before capturing a stream.
- * out_proj and x_proj add their partial sums with float atomics, so the last
- * bits of x can vary between runs.
+ * in_proj and out_proj split their reductions across blocks and add the
+ * partial sums with float atomics, so the last bits of x can vary between
+ * runs.  Their products keep float32 accuracy: the int8 weights are exact, and
+ * where d_model and d_inner are multiples of 16 they run on the tensor cores
+ * with each float32 activation split into two TF32 terms.
  */
 typedef struct {
     int64_t batch;      /* Bt >= 0 */
