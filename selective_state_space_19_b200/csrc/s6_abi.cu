@@ -1253,29 +1253,9 @@ int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x
     rc = gemm(hn, static_cast<int>(dm), 2 * di, dm, w->in_q, w->in_s, xz, static_cast<int>(l_xz), false);
     if (rc != S6_OK)
         return rc;
-    // 2. conv + SiLU (history shifted) and x_proj -> dt | B | C, a block per sequence
-    {
-        const size_t smem = sizeof(float) * di;
-        if (smem > 48 * 1024) {
-            static int opted[64] = {};
-            int dev = 0;
-            if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-                return S6_ERR_CUDA;
-            if (opted[dev] < static_cast<int>(smem)) {
-                if (smem > 227 * 1024 || cudaFuncSetAttribute(s6::block_conv_xproj_kernel,
-                                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                              static_cast<int>(smem)) != cudaSuccess)
-                    return S6_ERR_UNSUPPORTED;
-                opted[dev] = static_cast<int>(smem);
-            }
-        }
-        s6::block_conv_xproj_kernel<<<static_cast<unsigned>(Bt), s6::kConvXThreads, smem, s>>>(
-            xz, static_cast<int>(l_xz), w->conv_w, w->conv_b, conv_state, xc, static_cast<int>(l_xc), w->xp_q,
-            w->xp_s, dbc, static_cast<int>(l_dbc), static_cast<int>(di), static_cast<int>(K), static_cast<int>(row));
-        if (cudaGetLastError() != cudaSuccess)
-            return S6_ERR_CUDA;
-    }
-    // 3. dt_proj + the recurrence + readout + gate
+    // 2. conv + SiLU (history shifted) and x_proj -> dt | B | C, a block per
+    // sequence; 3. dt_proj + the recurrence + readout + gate -- at N = 16 in the
+    // same block (xc and the x_proj row stay in shared memory)
     s6::BlockSsmArgs a3;
     a3.Bt = static_cast<int>(Bt);
     a3.di = static_cast<int>(di);
@@ -1295,11 +1275,43 @@ int s6_block_step(const s6_block_dims *dims, const s6_block_weights *w, float *x
     a3.D = w->D;
     a3.h = h_ssm;
     a3.g = g;
-    s6::block_ssm_kernel<16><<<dim3(static_cast<unsigned>((di + s6::kSsmThreads - 1) / s6::kSsmThreads),
-                                    static_cast<unsigned>(Bt)),
-                               s6::kSsmThreads, sizeof(float) * row, s>>>(a3);
-    if (cudaGetLastError() != cudaSuccess)
-        return S6_ERR_CUDA;
+    const bool fused = N == 16 && aligned16(h_ssm) && aligned16(w->A_log);
+    {
+        const size_t smem = sizeof(float) * (round_up(static_cast<size_t>(di), 4) + (fused ? row : 0));
+        if (smem > 48 * 1024) {
+            static int opted[64][2] = {};
+            int dev = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+                return S6_ERR_CUDA;
+            if (opted[dev][fused] < static_cast<int>(smem)) {
+                if (smem > 227 * 1024 ||
+                    cudaFuncSetAttribute(fused ? s6::block_conv_xproj_kernel<true> : s6::block_conv_xproj_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem)) != cudaSuccess)
+                    return S6_ERR_UNSUPPORTED;
+                opted[dev][fused] = static_cast<int>(smem);
+            }
+        }
+        if (fused)
+            s6::block_conv_xproj_kernel<true><<<static_cast<unsigned>(Bt), s6::kConvXThreads, smem, s>>>(
+                xz, static_cast<int>(l_xz), w->conv_w, w->conv_b, conv_state, xc, static_cast<int>(l_xc), w->xp_q,
+                w->xp_s, dbc, static_cast<int>(l_dbc), static_cast<int>(di), static_cast<int>(K), static_cast<int>(row),
+                a3);
+        else
+            s6::block_conv_xproj_kernel<false><<<static_cast<unsigned>(Bt), s6::kConvXThreads, smem, s>>>(
+                xz, static_cast<int>(l_xz), w->conv_w, w->conv_b, conv_state, xc, static_cast<int>(l_xc), w->xp_q,
+                w->xp_s, dbc, static_cast<int>(l_dbc), static_cast<int>(di), static_cast<int>(K), static_cast<int>(row),
+                a3);
+        if (cudaGetLastError() != cudaSuccess)
+            return S6_ERR_CUDA;
+    }
+    if (!fused) {
+        s6::block_ssm_kernel<16><<<dim3(static_cast<unsigned>((di + s6::kSsmThreads - 1) / s6::kSsmThreads),
+                                        static_cast<unsigned>(Bt)),
+                                   s6::kSsmThreads, sizeof(float) * row, s>>>(a3);
+        if (cudaGetLastError() != cudaSuccess)
+            return S6_ERR_CUDA;
+    }
     // 4. out_proj, added into the residual stream
     return gemm(g, static_cast<int>(l_xc), dm, di, w->out_q, w->out_s, x, static_cast<int>(dm), true);
 }

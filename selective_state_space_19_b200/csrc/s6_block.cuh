@@ -113,6 +113,20 @@ __global__ void __launch_bounds__(kLnThreads) block_layernorm_kernel(const float
 }
 
 // ------------------------------------------------------------ conv + x_proj
+struct BlockSsmArgs {
+    int Bt, di, N, R;
+    const float *xz;   // [Bt][xz_ld]: xin | z
+    const float *xc;   // [Bt][xc_ld]: SiLU(conv(xin))
+    int xz_ld, xc_ld, g_ld;
+    const float *dbc;  // [Bt][dbc_ld]: dt | B | C (the x_proj rows, R + 2N used)
+    int dbc_ld;
+    const int8_t *dt_q;
+    const float *dt_s, *dt_bias;  // [di][R], [di], [di]
+    const float *A_log, *D;       // [di][N], [di]
+    float *h;  // [Bt][di][N] state, updated in place
+    float *g;  // [Bt][g_ld] gated readout y * SiLU(z)
+};
+
 constexpr int kConvXThreads = 256;
 
 // One block per sequence m: xc[c] = SiLU(conv_b + sum_{j<K-1} w[j] hist[j] +
@@ -120,11 +134,16 @@ constexpr int kConvXThreads = 256;
 // appends xin), kept in shared memory and written out; then the x_proj rows
 // dbc[m][o] = xp_s[o] * sum_c xp_q[o][c] xc[c], each row split over four
 // consecutive threads (a quarter of the channels each) and summed by shuffles.
+// SSM: the recurrence of the sequence follows in the same block (N = 16,
+// 16-byte aligned h and A_log rows): xc and the x_proj row stay in shared
+// memory, and xc, dbc are not written out.
+template <bool SSM>
 __global__ void __launch_bounds__(kConvXThreads) block_conv_xproj_kernel(
     const float *__restrict__ xz, int ldxz, const float *__restrict__ conv_w, const float *__restrict__ conv_b,
     float *__restrict__ hist, float *__restrict__ xc, int ldxc, const int8_t *__restrict__ xp_q,
-    const float *__restrict__ xp_s, float *__restrict__ dbc, int ld_dbc, int di, int Kc, int n_out) {
-    extern __shared__ __align__(16) float xcs[];  // di floats
+    const float *__restrict__ xp_s, float *__restrict__ dbc, int ld_dbc, int di, int Kc, int n_out,
+    const BlockSsmArgs sa) {
+    extern __shared__ __align__(16) float xcs[];  // di floats, rounded up to 4 (+ the x_proj row with SSM)
     const int m = blockIdx.x;
     // conv: a thread's channels in groups of 4, every load of a group issued first
     for (int c0 = threadIdx.x; c0 < di; c0 += 4 * kConvXThreads) {
@@ -179,7 +198,8 @@ __global__ void __launch_bounds__(kConvXThreads) block_conv_xproj_kernel(
             hs[Kc - 2] = xin[g];
             const float v = silu_exact(pre);
             xcs[c] = v;
-            xc[static_cast<size_t>(m) * ldxc + c] = v;
+            if (!SSM)
+                xc[static_cast<size_t>(m) * ldxc + c] = v;
         }
     }
     __syncthreads();
@@ -211,8 +231,81 @@ __global__ void __launch_bounds__(kConvXThreads) block_conv_xproj_kernel(
 #pragma unroll
         for (int off = 16; off; off >>= 1)
             sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane == 0)
-            dbc[static_cast<size_t>(m) * ld_dbc + o] = sum * xp_s[o];
+        if (lane == 0) {
+            if (SSM)
+                xcs[((di + 3) & ~3) + o] = sum * xp_s[o];
+            else
+                dbc[static_cast<size_t>(m) * ld_dbc + o] = sum * xp_s[o];
+        }
+    }
+    if constexpr (SSM) {
+        // the recurrence of this sequence, two channels per step with all of
+        // their loads issued first: dt_proj (R int8 weights on the dt part of
+        // the x_proj row), softplus, the 16 state updates, readout and gate
+        __syncthreads();
+        const float *srow = xcs + ((di + 3) & ~3);
+        const float *Bm = srow + sa.R, *Cm = srow + sa.R + 16;
+        const bool vec_dt = (sa.R % 4) == 0 && (reinterpret_cast<uintptr_t>(sa.dt_q) & 3) == 0;
+        for (int c0 = threadIdx.x; c0 < di; c0 += 2 * kConvXThreads) {
+            float4 h4[2][4], a4[2][4];
+            float zv[2];
+            int cc[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int c = c0 + k * kConvXThreads;
+                cc[k] = c < di ? c : di - 1;  // a spare lane repeats a channel it does not store
+                const float4 *hp = reinterpret_cast<const float4 *>(sa.h + (static_cast<size_t>(m) * di + cc[k]) * 16);
+                const float4 *ap = reinterpret_cast<const float4 *>(sa.A_log + static_cast<size_t>(cc[k]) * 16);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    h4[k][q4] = hp[q4];
+                    a4[k][q4] = ap[q4];
+                }
+                zv[k] = sa.xz[static_cast<size_t>(m) * sa.xz_ld + di + cc[k]];
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int c = c0 + k * kConvXThreads;
+                const int8_t *q = sa.dt_q + static_cast<size_t>(cc[k]) * sa.R;
+                float dtv = 0.f;
+                if (vec_dt) {
+                    const int *qw = reinterpret_cast<const int *>(q);
+                    for (int r4 = 0; r4 < sa.R / 4; ++r4) {
+                        const float4 w = i8x4_to_f32x4(qw[r4]);
+                        dtv = fmaf(w.x, srow[4 * r4], dtv);
+                        dtv = fmaf(w.y, srow[4 * r4 + 1], dtv);
+                        dtv = fmaf(w.z, srow[4 * r4 + 2], dtv);
+                        dtv = fmaf(w.w, srow[4 * r4 + 3], dtv);
+                    }
+                } else {
+                    for (int r = 0; r < sa.R; ++r)
+                        dtv = fmaf(static_cast<float>(q[r]), srow[r], dtv);
+                }
+                const float v = fmaf(dtv, sa.dt_s[cc[k]], sa.dt_bias[cc[k]]);
+                const float delta = fmaxf(v, 0.f) + log1pf(__expf(-fabsf(v)));  // softplus
+                const float x_c = xcs[cc[k]];
+                const float du = delta * x_c;
+                const float dl2 = -delta * kLog2e;
+                float acc = 0.f;
+                float4 *hp = reinterpret_cast<float4 *>(sa.h + (static_cast<size_t>(m) * di + cc[k]) * 16);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float hh[4] = {h4[k][q4].x, h4[k][q4].y, h4[k][q4].z, h4[k][q4].w};
+                    const float aa[4] = {a4[k][q4].x, a4[k][q4].y, a4[k][q4].z, a4[k][q4].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int n = 4 * q4 + e;
+                        const float ab = ex2_approx(dl2 * __expf(aa[e]));  // exp(Delta A), A = -exp(A_log)
+                        hh[e] = fmaf(ab, hh[e], du * Bm[n]);
+                        acc = fmaf(hh[e], Cm[n], acc);
+                    }
+                    if (c < di)
+                        hp[q4] = make_float4(hh[0], hh[1], hh[2], hh[3]);
+                }
+                if (c < di)
+                    sa.g[static_cast<size_t>(m) * sa.g_ld + c] = fmaf(sa.D[c], x_c, acc) * silu_exact(zv[k]);
+            }
+        }
     }
 }
 
@@ -557,21 +650,6 @@ __global__ void __launch_bounds__(kTcThreads) q8_tc_gemm_kernel(const Q8GemmArgs
             }
         }
 }
-
-// ------------------------------------------------------------ the recurrence
-struct BlockSsmArgs {
-    int Bt, di, N, R;
-    const float *xz;   // [Bt][xz_ld]: xin | z
-    const float *xc;   // [Bt][xc_ld]: SiLU(conv(xin))
-    int xz_ld, xc_ld, g_ld;
-    const float *dbc;  // [Bt][dbc_ld]: dt | B | C (the x_proj rows, R + 2N used)
-    int dbc_ld;
-    const int8_t *dt_q;
-    const float *dt_s, *dt_bias;  // [di][R], [di], [di]
-    const float *A_log, *D;       // [di][N], [di]
-    float *h;  // [Bt][di][N] state, updated in place
-    float *g;  // [Bt][g_ld] gated readout y * SiLU(z)
-};
 
 constexpr int kSsmThreads = 256;
 
