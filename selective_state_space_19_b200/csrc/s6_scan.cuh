@@ -29,6 +29,9 @@
 // the [T x N] rows of B and C into a STAGES-deep shared-memory ring, fetches a
 // unit's start state from the carry buffer once its flags are published, and
 // converts each chunk's B/C rows to float32 before marking the stage ready.
+// It shares an SM sub-partition with consumer warps, so it keeps its own
+// instruction count low: the B/C copy moves whole 512-byte groups with
+// constant per-lane addresses, and its waits sleep between polls.
 // The 3 halo rows give the conv its K-1 earlier inputs; rows before token 0
 // are zero-filled by the TMA unit (the conv's zero left padding).  Warps 0-3
 // are consumers: each waits for a ready stage, runs its 32/TPC channels over
@@ -50,9 +53,11 @@
 // rows they read (conv window, z, dt) fetched one quad ahead.  State
 // arithmetic runs on packed float32 pairs (f32x2).
 //
-// The INIT instantiations also start a chain from a given state (h_init, and
-// for the fused form the conv history before token 0); they are separate so
-// that the plain scan's code is untouched by that support.
+// The extended instantiations (EXT = 1) also start a chain from a given state
+// (h_init, and for the fused form the conv history before token 0) and take
+// the associative split of few long chains; the checkpoint instantiation
+// (EXT = 2) stores the backward's state checkpoints and computes no output.
+// They are separate so that the plain scan's code is untouched by that support.
 //
 // No tensor cores: the recurrence is diagonal (an elementwise product with a
 // data-dependent decay), not a contraction.
