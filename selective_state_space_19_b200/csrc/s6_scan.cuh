@@ -31,7 +31,10 @@
 // converts each chunk's B/C rows to float32 before marking the stage ready.
 // It shares an SM sub-partition with consumer warps, so it keeps its own
 // instruction count low: the B/C copy moves whole 512-byte groups with
-// constant per-lane addresses, and its waits sleep between polls.
+// constant per-lane addresses, and its waits sleep between polls.  It is the
+// CTA's fifth warp, so that the four consumer warps (warps 0-3) fall on the
+// SM's four sub-partitions: moving the producer to another warp index put two
+// consumers on one sub-partition and cost a quarter of the throughput.
 // The 3 halo rows give the conv its K-1 earlier inputs; rows before token 0
 // are zero-filled by the TMA unit (the conv's zero left padding).  Warps 0-3
 // are consumers: each waits for a ready stage, runs its 32/TPC channels over
