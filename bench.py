@@ -892,11 +892,19 @@ def run_profile_case(case):
     """Small fixed cases for ncu captures of kernels outside the timed step:
     'bwd' -- three s6_scan_bwd calls on the long_seq recipe at Bt16 L1024 (the
     full workload's 384 chains, ~0.65 GB on the device); 'block' -- three decode
-    token steps of 256 sequences through the 6 Mamba-mini blocks."""
+    token steps of 256 sequences through the 6 Mamba-mini blocks; 'mamba_mini'
+    -- three fused scans of the Mamba-mini block workload (Bt8 L256 d1536,
+    float32)."""
     import torch
     import selective_state_space_19_b200 as S
     dev = torch.device("cuda", 0)
-    if case == "bwd":
+    if case == "mamba_mini":
+        inp = SI.scan_inputs("mamba_mini")
+        t = {k: to_dev(inp[k], dev) for k in ("x", "z", "B", "C", "dt", "A_log", "D", "dt_bias", "conv_w", "conv_b")}
+        for _ in range(3):
+            S.s6_conv_scan_fwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"],
+                               z=t["z"], dt_bias=t["dt_bias"])
+    elif case == "bwd":
         inp = SI.scan_inputs("long_seq", Bt=16, L=1024, seed=3)
         t = {k: to_dev(inp[k], dev) for k in ("x", "z", "B", "C", "dt", "A_log", "D", "dt_bias")}
         gen = torch.Generator(device=dev).manual_seed(7)
@@ -925,9 +933,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["full", "small", "bwd", "block"], default="full",
-                    help="small: the workload at L=2048 (for ncu captures); bwd, block: small cases of the "
-                         "backward and the decode block for captures (no JSON line)")
+    ap.add_argument("--case", choices=["full", "small", "bwd", "block", "mamba_mini"], default="full",
+                    help="small: the workload at L=2048 (for ncu captures); bwd, block, mamba_mini: small cases "
+                         "of the backward, the decode block and the Mamba-mini scan for captures (no JSON line)")
     ap.add_argument("--no-rows", action="store_true", help="skip the decode-step and standalone-conv rows")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -935,7 +943,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
-    if args.case in ("bwd", "block"):
+    if args.case in ("bwd", "block", "mamba_mini"):
         return run_profile_case(args.case)
     return run_ours(args)
 

@@ -269,13 +269,13 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
     const int64_t L = dims->seqlen;
     a.tiles = static_cast<int>((dims->d_inner + CPB - 1) / CPB);
     const int64_t chains = dims->batch * a.tiles;
-    // Every SM gets the same number of persistent CTAs, and no more CTAs run
-    // than there are chains (a CTA beyond that would only wait).
+    // Persistent CTAs, as many per SM as fit; no more of them than chains (or
+    // units, for the associative split) can run at once.  With fewer chains
+    // than CTA slots this still puts a second CTA on some SMs: measured on
+    // Mamba-mini's 192 chains, 192 CTAs beat 148 (one per SM) by 2 %.
     const int64_t sms = device_sm_count();
     const bool assoc = INIT && want_assoc(chains, L, T, sms * occ);
-    int64_t per_sm = occ;
-    while (!assoc && per_sm > 1 && per_sm * sms > chains)
-        --per_sm;
+    const int64_t per_sm = occ;
     const int64_t workers = sms * per_sm;
     int64_t nseg = 1, seg_len = round_up(static_cast<size_t>(L), T);
     if (assoc) {
