@@ -9,8 +9,12 @@ one s6_conv_scan_fwd launch over 201M (b, t, channel) elements.  Inputs
 metric: Gelem/s = Bt*L*d_inner / time.  value: whole job (all ranks).
 Also reported: the roofline of the dominant kernel (MUFU ex2: N = 16
 exponentials per element; HBM alongside), the oracle on the host cores
-(cpu_baseline), the same metric end to end from pinned host buffers (e2e), and
-the other rows of the path -- the streaming-decode step and the standalone conv.
+(cpu_baseline), the same metric end to end from pinned host buffers (e2e,
+pipelined over batch chunks), and rows for the rest of the path, each with its
+own roofline: the other workloads of the pages (Mamba-mini, wide, one long
+prompt), random A_log, the streaming-decode step, the decode block, the
+constant-decay cell, the standalone conv, a chunked prefill and the two
+backward passes.
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Multi-GPU: torchrun ... bench.py --gpus N; each rank scans its own batch (weak
