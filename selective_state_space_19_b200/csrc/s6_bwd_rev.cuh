@@ -27,7 +27,8 @@
 // channels' 32 values per token across its lanes (15 shuffles a thread), the
 // four warps add theirs in shared memory, and one row per (tile, token) is
 // written to a partial buffer that s6_bwd_bc_reduce_kernel sums over the
-// tiles -- no global atomics, and the same sums on every run.  A chain is cut
+// tiles -- no global atomics (the order of the four warps' shared-memory adds
+// is not fixed, so runs agree to float32 rounding).  A chain is cut
 // into segments pulled last-first from a global counter; a segment's unit
 // starts from dLoss/dh (and the conv's dpre window) published by the unit of
 // the segment after it, which was pulled earlier, so every (bounded) wait ends.
