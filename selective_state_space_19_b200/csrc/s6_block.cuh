@@ -128,6 +128,13 @@ struct BlockSsmArgs {
 };
 
 constexpr int kConvXThreads = 256;
+constexpr int kXprojIt = 12;  // x_proj weight words a lane holds per row (rows of up to 12 x 128 channels)
+
+// Asks the L2 to fetch [p, p + bytes) ahead of use: p 16-byte aligned, bytes a
+// multiple of 16, the range inside one allocation.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 // One block per sequence m: xc[c] = SiLU(conv_b + sum_{j<K-1} w[j] hist[j] +
 // w[K-1] xin[c]) for every channel (the history drops its oldest input and
@@ -136,15 +143,27 @@ constexpr int kConvXThreads = 256;
 // consecutive threads (a quarter of the channels each) and summed by shuffles.
 // SSM: the recurrence of the sequence follows in the same block (N = 16,
 // 16-byte aligned h and A_log rows): xc and the x_proj row stay in shared
-// memory, and xc, dbc are not written out.
+// memory, and xc, dbc are not written out; the sequence's state row is sent
+// to the L2 when the block starts, so the recurrence does not wait on HBM.
+// With rows of up to 12 x 128 channels (a multiple of 4), a lane holds a
+// row's weight words in registers and fetches the next row's while it sums
+// this one.
 template <bool SSM>
-__global__ void __launch_bounds__(kConvXThreads) block_conv_xproj_kernel(
+__global__ void __launch_bounds__(kConvXThreads, 2) block_conv_xproj_kernel(
     const float *__restrict__ xz, int ldxz, const float *__restrict__ conv_w, const float *__restrict__ conv_b,
     float *__restrict__ hist, float *__restrict__ xc, int ldxc, const int8_t *__restrict__ xp_q,
     const float *__restrict__ xp_s, float *__restrict__ dbc, int ld_dbc, int di, int Kc, int n_out,
     const BlockSsmArgs sa) {
     extern __shared__ __align__(16) float xcs[];  // di floats, rounded up to 4 (+ the x_proj row with SSM)
     const int m = blockIdx.x;
+    if constexpr (SSM) {
+        // the state row h[m] (di x 16 floats), in pieces of at most 16 KB
+        constexpr uint32_t kPiece = 16384;
+        const uint32_t bytes = static_cast<uint32_t>(di) * 16u * sizeof(float);
+        const char *row = reinterpret_cast<const char *>(sa.h + static_cast<size_t>(m) * di * 16);
+        for (uint32_t off = threadIdx.x * kPiece; off < bytes; off += kConvXThreads * kPiece)
+            bulk_prefetch_l2(row + off, min(kPiece, bytes - off));
+    }
     // conv: a thread's channels in groups of 4, every load of a group issued first
     for (int c0 = threadIdx.x; c0 < di; c0 += 4 * kConvXThreads) {
         float xin[4], hv[4][3], wv[4][4], bv[4];
@@ -207,7 +226,53 @@ __global__ void __launch_bounds__(kConvXThreads) block_conv_xproj_kernel(
     // weight rows, consecutive float4 of xc)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool vec = (di % 4) == 0 && (reinterpret_cast<uintptr_t>(xp_q) & 3) == 0;
-    for (int o = warp; o < n_out; o += kConvXThreads / 32) {
+    const int n4 = di / 4;
+    if (vec && n4 <= 32 * kXprojIt) {
+        // a row's words in registers; the next row's loads go out before this row's sums
+        const float4 *x4 = reinterpret_cast<const float4 *>(xcs);
+        int wq[kXprojIt], wn[kXprojIt];
+        auto fetch = [&](int o, int (&w)[kXprojIt]) {
+            const int *qw = reinterpret_cast<const int *>(xp_q + static_cast<size_t>(o) * di);
+#pragma unroll
+            for (int k = 0; k < kXprojIt; ++k) {
+                const int c4 = lane + 32 * k;
+                w[k] = c4 < n4 ? __ldg(qw + c4) : 0;
+            }
+        };
+        if (warp < n_out)
+            fetch(warp, wq);
+        for (int o = warp; o < n_out; o += kConvXThreads / 32) {
+            if (o + kConvXThreads / 32 < n_out)
+                fetch(o + kConvXThreads / 32, wn);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < kXprojIt; ++k) {
+                const int c4 = lane + 32 * k;
+                if (c4 < n4) {
+                    const float4 wv = i8x4_to_f32x4(wq[k]);
+                    const float4 xv = x4[c4];
+                    acc[0] = fmaf(wv.x, xv.x, acc[0]);
+                    acc[1] = fmaf(wv.y, xv.y, acc[1]);
+                    acc[2] = fmaf(wv.z, xv.z, acc[2]);
+                    acc[3] = fmaf(wv.w, xv.w, acc[3]);
+                }
+            }
+            float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+#pragma unroll
+            for (int off = 16; off; off >>= 1)
+                sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            if (lane == 0) {
+                if (SSM)
+                    xcs[((di + 3) & ~3) + o] = sum * xp_s[o];
+                else
+                    dbc[static_cast<size_t>(m) * ld_dbc + o] = sum * xp_s[o];
+            }
+#pragma unroll
+            for (int k = 0; k < kXprojIt; ++k)
+                wq[k] = wn[k];
+        }
+    }
+    for (int o = warp; !(vec && n4 <= 32 * kXprojIt) && o < n_out; o += kConvXThreads / 32) {
         const int8_t *q = xp_q + static_cast<size_t>(o) * di;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         if (vec) {
