@@ -65,6 +65,14 @@ def test_block_single_sequence_and_tile_edges():
     _run(Bt=65, dm=48, di=80, N=16, R=4, K=2, blocks=2, steps=2, seed=16)
 
 
+def test_block_xproj_row_paths():
+    """d_inner 1600 (x_proj rows longer than the 12 x 128 channels a lane
+    holds in registers) and 90 (rows not a multiple of 4 channels): the x_proj
+    loops that stream a row from the L2, in front of the fused recurrence."""
+    _run(Bt=3, dm=40, di=1600, N=16, R=6, K=4, blocks=1, steps=2, seed=17)
+    _run(Bt=3, dm=40, di=90, N=16, R=6, K=4, blocks=1, steps=2, seed=18)
+
+
 def test_block_mamba_mini_dims():
     """The Mamba-mini block (d_model 384, d_inner 1536, N 16, dt rank 24, conv 4)
     through all 6 blocks for 6 tokens, on a 16-sequence batch."""
