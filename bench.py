@@ -13,8 +13,9 @@ exponentials per element; HBM alongside), the oracle on the host cores
 pipelined over batch chunks), and rows for the rest of the path, each with its
 own roofline: the other workloads of the pages (Mamba-mini, wide, one long
 prompt), random A_log, the streaming-decode step, the decode block, the
-constant-decay cell, the standalone conv, a chunked prefill and the two
-backward passes.
+constant-decay cell, the standalone conv, a chunked prefill, the two
+backward passes and a training step (forward keeping checkpoints, backward
+from them).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Multi-GPU: torchrun ... bench.py --gpus N; each rank scans its own batch (weak
@@ -394,6 +395,66 @@ def row_bwd(device, stream, pk, inp_dev, cfg, iters=3, fused=False):
                          "frac": ex2_per_s / peak_ex2,
                          "note": "16 ex2 per element credited (the forward's); the kernel issues 48 "
                                  "(forward to checkpoints, chunk recompute, reverse)"}}
+
+
+def row_train(device, stream, pk, inp_dev, cfg, iters=3):
+    """A training step of the fused path on the long_seq inputs: the forward that
+    also keeps the state before every 16th token (s6_conv_scan_fwd_ckpt), then the
+    backward from those states (s6_conv_scan_bwd with ckpt), which runs no forward
+    of its own.  Beside it, the same step with the backward that recomputes its
+    checkpoints (s6_conv_scan_fwd, then s6_conv_scan_bwd)."""
+    import selective_state_space_19_b200 as S
+    import torch
+    Bt, L, d, N = cfg["Bt"], cfg["L"], cfg["d"], cfg["N"]
+    t = inp_dev
+    gen = torch.Generator(device=device).manual_seed(7)
+    dy = torch.randn(Bt, L, d, device=device, generator=gen).to(t["x"].dtype)
+    zoh = int(bool(cfg["zoh"]))
+    y = torch.empty_like(t["x"])
+    h = torch.empty(Bt, d, N, device=device)
+    ck = torch.empty(Bt, (L + S.CKPT_EVERY - 1) // S.CKPT_EVERY, d, N, device=device)
+    args = (t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"])
+
+    def fwd_ckpt():
+        S.s6_conv_scan_fwd_ckpt(*args, z=t["z"], dt_bias=t["dt_bias"], zoh_mode=zoh, y=y, h_final=h, ckpt=ck,
+                                stream=stream)
+
+    def bwd_ckpt():
+        S.s6_conv_scan_bwd(*args, dy, z=t["z"], dt_bias=t["dt_bias"], zoh_mode=zoh, ckpt=ck, stream=stream)
+
+    def step():
+        fwd_ckpt()
+        bwd_ckpt()
+
+    def step_recompute():
+        S.s6_conv_scan_fwd(*args, z=t["z"], dt_bias=t["dt_bias"], zoh_mode=zoh, y=y, h_final=h, stream=stream)
+        S.s6_conv_scan_bwd(*args, dy, z=t["z"], dt_bias=t["dt_bias"], zoh_mode=zoh, stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()
+        step_recompute()
+        torch.cuda.synchronize(device)
+        ms = time_events(step, iters, stream)
+        ms_re = time_events(step_recompute, iters, stream)
+        ms_f = time_events(fwd_ckpt, iters, stream)
+        ms_b = time_events(bwd_ckpt, iters, stream)
+    assert S.s6_device_status(stream=stream, device=device) == 0
+    elems = Bt * L * d
+    ex2_per_s = elems * 2 * N / (ms * 1e-3)
+    peak_ex2 = SMS * MUFU_PER_SM_CLK * pk["sm_max_mhz"] * 1e6
+    return {"workload": "training step of the fused path on long_seq (Bt16 L8192 d1536 N16, bf16 in, float32 "
+                        "gradients, gate, simplified write): s6_conv_scan_fwd_ckpt (y, h_final and the state every "
+                        "16 tokens), then s6_conv_scan_bwd from those states",
+            "value": elems / (ms * 1e-3) / 1e9, "unit": "Gelem/s (forward + backward)", "ms_per_step": ms,
+            "forward_ckpt_ms": ms_f, "backward_from_ckpt_ms": ms_b,
+            "backward_from_ckpt_value": elems / (ms_b * 1e-3) / 1e9,
+            "recomputing_step": {"ms_per_step": ms_re, "value": elems / (ms_re * 1e-3) / 1e9,
+                                 "what": "s6_conv_scan_fwd, then s6_conv_scan_bwd running its own "
+                                         "checkpointing forward"},
+            "roofline": {"bound": "alu", "achieved": ex2_per_s / 1e12, "peak": peak_ex2 / 1e12, "unit": "Tex2/s",
+                         "frac": ex2_per_s / peak_ex2,
+                         "note": "16 ex2 per element credited to each of the forward and the backward; the "
+                                 "kernels issue 48 (forward, chunk recompute, reverse)"}}
 
 
 def row_scan(device, stream, pk, name, zoh=None, over=None, iters=20, label=None):
@@ -866,6 +927,7 @@ def run_ours(args):
         rows["s6_conv_scan_fwd_from_state"] = row_prefill(device, stream, pk, t, cfg)
         rows["s6_scan_bwd"] = row_bwd(device, stream, pk, t, cfg)
         rows["s6_conv_scan_bwd"] = row_bwd(device, stream, pk, t, cfg, fused=True)
+        rows["train_step_conv_scan"] = row_train(device, stream, pk, t, cfg)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -256,9 +256,12 @@ S6_API int s6_diag_recurrence_fwd(const s6_dims *dims, int decay_source, const v
  *  dh_init   [Bt,d,N]      with respect to h_init (NULL = not wanted)
  * dB, dC, dA_log, dD and ddt_bias are zeroed by the call, then accumulated
  * with atomics, so their last bits depend on the order of the additions.  The
- * call uses the library-owned scratch buffer (state checkpoints every 64
- * tokens plus one chunk of states: (ceil(L/64) + 64) * Bt * d * 16 floats at
- * N = 16).  Pointers need only element alignment.
+ * call uses the library-owned scratch buffer.  At N = 16 with 16-byte aligned
+ * u, dt, z, dy, B, C and d * sizeof(io) a multiple of 16 (the pipelined
+ * backward) it holds the state before every 16th token (ceil(L/16) * Bt * d *
+ * 16 floats) and per-tile dB / dC rows (ceil(d/64) * Bt * L * 32 floats);
+ * otherwise the state every 64 tokens plus one chunk of states ((ceil(L/64) +
+ * 64) * Bt * d * N floats).  Pointers need only element alignment.
  */
 S6_API int s6_scan_bwd(const s6_dims *dims, const void *u, const void *dt, const float *A_log,
                        const void *B, const void *C, const float *D, const void *z,
@@ -284,6 +287,54 @@ S6_API int s6_conv_scan_bwd(const s6_dims *dims, const void *x, const float *con
                             const void *dy, float *dx, float *dconv_w, float *dconv_b,
                             float *ddt, float *dz, float *dB, float *dC, float *dA_log,
                             float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream);
+
+/*
+ * s6_scan_fwd_ckpt, s6_conv_scan_fwd_ckpt -- the forward of a training step:
+ * s6_scan_fwd_from_state / s6_conv_scan_fwd (zero conv history) that also
+ * keeps what the backward would otherwise recompute, so that the backward
+ * does not run the forward again ("Carry context through a selective state":
+ * the recurrence is what makes training slow).  Arguments as those calls
+ * (h_init [Bt,d,N] f32, NULL = zeros), plus
+ *
+ *  ckpt  [Bt][ceil(L/16)][d][16] f32  written: ckpt[b][k] is the state before
+ *        token 16 k (h_init, or zeros, at k = 0); 16-byte aligned
+ *
+ * N = 16 only (S6_ERR_UNSUPPORTED otherwise).  The SiLUs are evaluated as the
+ * backward evaluates them (the exponential form), so with bfloat16 I/O y may
+ * differ from s6_conv_scan_fwd's in its last bit.  The checkpoints stay valid
+ * for the inputs they were computed from.
+ */
+S6_API int s6_scan_fwd_ckpt(const s6_dims *dims, const void *u, const void *dt, const float *A_log,
+                            const void *B, const void *C, const float *D, const void *z,
+                            const float *dt_bias, int zoh_mode, const float *h_init, void *y,
+                            float *h_final, float *ckpt, s6_stream_t stream);
+S6_API int s6_conv_scan_fwd_ckpt(const s6_dims *dims, const void *x, const float *conv_w,
+                                 const float *conv_b, const void *dt, const float *A_log,
+                                 const void *B, const void *C, const float *D, const void *z,
+                                 const float *dt_bias, int zoh_mode, const float *h_init, void *y,
+                                 float *h_final, float *ckpt, s6_stream_t stream);
+
+/*
+ * s6_scan_bwd_ckpt, s6_conv_scan_bwd_ckpt -- s6_scan_bwd / s6_conv_scan_bwd
+ * given the checkpoints that the matching _ckpt forward wrote for the same
+ * inputs: the arguments of those calls with ckpt (read only) in place of
+ * h_init, which the checkpoints already hold.  Only the pipelined backward
+ * takes checkpoints: N = 16 (S6_ERR_UNSUPPORTED otherwise), and u / x, dt, z,
+ * dy, B, C and ckpt 16-byte aligned with d * sizeof(io) a multiple of 16
+ * (S6_ERR_ALIGNMENT otherwise).  The scratch holds only the dB / dC rows.
+ */
+S6_API int s6_scan_bwd_ckpt(const s6_dims *dims, const void *u, const void *dt, const float *A_log,
+                            const void *B, const void *C, const float *D, const void *z,
+                            const float *dt_bias, int zoh_mode, const float *ckpt, const void *dy,
+                            float *du, float *ddt, float *dz, float *dB, float *dC, float *dA_log,
+                            float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream);
+S6_API int s6_conv_scan_bwd_ckpt(const s6_dims *dims, const void *x, const float *conv_w,
+                                 const float *conv_b, const void *dt, const float *A_log,
+                                 const void *B, const void *C, const float *D, const void *z,
+                                 const float *dt_bias, int zoh_mode, const float *ckpt,
+                                 const void *dy, float *dx, float *dconv_w, float *dconv_b,
+                                 float *ddt, float *dz, float *dB, float *dC, float *dA_log,
+                                 float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream);
 
 /*
  * causal_conv1d_silu_fwd -- the conv + SiLU alone ("mamba, live":

@@ -19,7 +19,9 @@ import os
 
 __all__ = [
     "S6Error", "lib", "s6_scan_fwd", "s6_conv_scan_fwd", "s6_conv_scan_fwd_noalloc", "s6_scan_fwd_from_state",
-    "s6_conv_scan_fwd_from_state", "s6_diag_recurrence_fwd", "S6_DECAY_LIVE", "S6_DECAY_CONST", "s6_scan_bwd", "s6_conv_scan_bwd", "causal_conv1d_silu_fwd", "s6_step",
+    "s6_conv_scan_fwd_from_state", "s6_scan_fwd_ckpt", "s6_conv_scan_fwd_ckpt", "CKPT_EVERY",
+    "s6_diag_recurrence_fwd", "S6_DECAY_LIVE", "S6_DECAY_CONST", "s6_scan_bwd", "s6_conv_scan_bwd",
+    "causal_conv1d_silu_fwd", "s6_step",
     "s6_block_step", "BlockDims", "BlockWeights", "BLOCK_WEIGHT_KEYS",
     "s6_device_status", "s6_status_string", "s6_version", "s6_debug_carry_fault", "S6_F32", "S6_BF16", "Dims",
 ]
@@ -31,6 +33,7 @@ S6_F32, S6_BF16 = 0, 1
 S6_OK, S6_ERR_INVALID_ARG, S6_ERR_UNSUPPORTED, S6_ERR_ALIGNMENT, S6_ERR_CUDA, S6_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 S6_ERR_SCRATCH_LIMIT = -6
 S6_DECAY_LIVE, S6_DECAY_CONST = 0, 1
+CKPT_EVERY = 16  # tokens between the states a training forward keeps for the backward
 
 
 class Dims(ctypes.Structure):
@@ -84,6 +87,10 @@ def lib() -> ctypes.CDLL:
         L.s6_diag_recurrence_fwd.argtypes = [DP, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.s6_scan_bwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P] + [_P] * 9 + [_P]
         L.s6_conv_scan_bwd.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P] + [_P] * 11 + [_P]
+        L.s6_scan_fwd_ckpt.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]
+        L.s6_conv_scan_fwd_ckpt.argtypes = [DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]
+        L.s6_scan_bwd_ckpt.argtypes = L.s6_scan_bwd.argtypes
+        L.s6_conv_scan_bwd_ckpt.argtypes = L.s6_conv_scan_bwd.argtypes
         L.causal_conv1d_silu_fwd.argtypes = [DP, _P, _P, _P, _P, _P]
         L.s6_step.argtypes = [DP, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.s6_device_status.argtypes = [_P]
@@ -156,7 +163,7 @@ def _check(status, where):
 
 
 def _scan(fn, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w, conv_b, want_h, stream,
-          from_state=False, h_init=None, conv_hist=None):
+          from_state=False, h_init=None, conv_hist=None, ckpt_mode=False, ckpt=None):
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x/u must be [batch, seqlen, d_inner]")
@@ -182,12 +189,19 @@ def _scan(fn, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w, c
              _ptr(B, "B", x.dtype, (Bt, L, N), dev), _ptr(C, "C", x.dtype, (Bt, L, N), dev),
              _ptr(D, "D", f32, (d,), dev), _ptr(z, "z", x.dtype, seq, dev),
              _ptr(dt_bias, "dt_bias", f32, (d,), dev), int(zoh_mode)]
-    if from_state:
+    if from_state or ckpt_mode:
         args += [_ptr(h_init, "h_init", f32, (Bt, d, N), dev)]
-        if conv_w is not None:
+        if conv_w is not None and not ckpt_mode:
             args += [_ptr(conv_hist, "conv_hist", x.dtype, (Bt, d, K - 1), dev)]
-    args += [_ptr(y, "y", x.dtype, seq, dev), _ptr(h_final, "h_final", f32, (Bt, d, N), dev), _stream(stream, dev)]
+    args += [_ptr(y, "y", x.dtype, seq, dev), _ptr(h_final, "h_final", f32, (Bt, d, N), dev)]
+    if ckpt_mode:
+        if ckpt is None:
+            ckpt = torch.empty((Bt, (L + CKPT_EVERY - 1) // CKPT_EVERY, d, N), dtype=f32, device=dev)
+        args += [_ptr(ckpt, "ckpt", f32, (Bt, (L + CKPT_EVERY - 1) // CKPT_EVERY, d, N), dev)]
+    args += [_stream(stream, dev)]
     _check(fn(*args), fn.__name__)
+    if ckpt_mode:
+        return y, h_final, ckpt
     return y, h_final
 
 
@@ -230,6 +244,24 @@ def s6_conv_scan_fwd_from_state(x, conv_w, conv_b, dt, A_log, B, C, D, z=None, d
                  conv_b, want_h_final, stream, from_state=True, h_init=h_init, conv_hist=conv_hist)
 
 
+def s6_scan_fwd_ckpt(u, dt, A_log, B, C, D, z=None, dt_bias=None, zoh_mode=0, h_init=None, y=None, h_final=None,
+                     ckpt=None, want_h_final=True, stream=None):
+    """The forward of a training step: s6_scan_fwd_from_state that also keeps the
+    state before every 16th token, ckpt [Bt, ceil(L/16), d, 16] float32, for
+    s6_scan_bwd(..., ckpt=ckpt).  N = 16.  Returns (y, h_final, ckpt)."""
+    return _scan(lib().s6_scan_fwd_ckpt, u, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, None, None,
+                 want_h_final, stream, h_init=h_init, ckpt_mode=True, ckpt=ckpt)
+
+
+def s6_conv_scan_fwd_ckpt(x, conv_w, conv_b, dt, A_log, B, C, D, z=None, dt_bias=None, zoh_mode=0, h_init=None,
+                          y=None, h_final=None, ckpt=None, want_h_final=True, stream=None):
+    """The forward of a training step on the fused path (zero conv history): also
+    keeps the state before every 16th token for s6_conv_scan_bwd(..., ckpt=ckpt).
+    N = 16.  Returns (y, h_final, ckpt)."""
+    return _scan(lib().s6_conv_scan_fwd_ckpt, x, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, conv_w,
+                 conv_b, want_h_final, stream, h_init=h_init, ckpt_mode=True, ckpt=ckpt)
+
+
 def s6_diag_recurrence_fwd(u, B, C, D, decay_source=S6_DECAY_CONST, log2_decay=None, dt=None, A_log=None,
                            dt_bias=None, z=None, h_init=None, y=None, h_final=None, want_h_final=True, stream=None):
     """The diagonal recurrence with the decay source as a parameter: constant
@@ -264,11 +296,23 @@ def s6_diag_recurrence_fwd(u, B, C, D, decay_source=S6_DECAY_CONST, log2_decay=N
     return y, h_final
 
 
+def _bwd_start(fn, fn_ckpt, h_init, ckpt, Bt, L, d, N, dev):
+    """The backward entry point and its start argument: h_init, or the checkpoints
+    of a training forward (which hold the start state)."""
+    if ckpt is None:
+        return fn, _ptr(h_init, "h_init", _torch().float32, (Bt, d, N), dev)
+    if h_init is not None:
+        raise ValueError("with ckpt, the start state is in the checkpoints: pass h_init to the forward")
+    return fn_ckpt, _ptr(ckpt, "ckpt", _torch().float32, (Bt, (L + CKPT_EVERY - 1) // CKPT_EVERY, d, N), dev)
+
+
 def s6_scan_bwd(u, dt, A_log, B, C, D, dy, z=None, dt_bias=None, zoh_mode=0, h_init=None, want_dh_init=False,
-                stream=None):
+                stream=None, ckpt=None):
     """Gradients of s6_scan_fwd for the loss sum(dy * y).  Returns a dict of float32
     tensors: du, ddt, dz (None without z) [Bt, L, d]; dB, dC [Bt, L, N]; dA_log [d, N];
-    dD, ddt_bias (None without dt_bias) [d]; dh_init [Bt, d, N] (None unless wanted)."""
+    dD, ddt_bias (None without dt_bias) [d]; dh_init [Bt, d, N] (None unless wanted).
+    ckpt: the checkpoints of s6_scan_fwd_ckpt on the same inputs (its h_init is
+    in them, so h_init must then be None); the backward then skips its own forward."""
     torch = _torch()
     if u.dim() != 3:
         raise ValueError("u must be [batch, seqlen, d_inner]")
@@ -285,23 +329,25 @@ def s6_scan_bwd(u, dt, A_log, B, C, D, dy, z=None, dt_bias=None, zoh_mode=0, h_i
          "dh_init": torch.empty((Bt, d, N), dtype=f32, device=dev) if want_dh_init else None}
     dims = Dims(Bt, L, d, N, 0, _io_code(u))
     io = u.dtype
-    st = lib().s6_scan_bwd(ctypes.byref(dims), _ptr(u, "u", io, seq, dev), _ptr(dt, "dt", io, seq, dev),
+    fn, start = _bwd_start(lib().s6_scan_bwd, lib().s6_scan_bwd_ckpt, h_init, ckpt, Bt, L, d, N, dev)
+    st = fn(ctypes.byref(dims), _ptr(u, "u", io, seq, dev), _ptr(dt, "dt", io, seq, dev),
                            _ptr(A_log, "A_log", f32, (d, N), dev), _ptr(B, "B", io, (Bt, L, N), dev),
                            _ptr(C, "C", io, (Bt, L, N), dev), _ptr(D, "D", f32, (d,), dev),
                            _ptr(z, "z", io, seq, dev), _ptr(dt_bias, "dt_bias", f32, (d,), dev), int(zoh_mode),
-                           _ptr(h_init, "h_init", f32, (Bt, d, N), dev), _ptr(dy, "dy", io, seq, dev),
+                           start, _ptr(dy, "dy", io, seq, dev),
                            *[_ptr(g[k], k) for k in ("du", "ddt", "dz", "dB", "dC", "dA_log", "dD", "ddt_bias",
                                                      "dh_init")],
                            _stream(stream, dev))
-    _check(st, "s6_scan_bwd")
+    _check(st, fn.__name__)
     return g
 
 
 def s6_conv_scan_bwd(x, conv_w, conv_b, dt, A_log, B, C, D, dy, z=None, dt_bias=None, zoh_mode=0, h_init=None,
-                     want_dh_init=False, stream=None):
+                     want_dh_init=False, stream=None, ckpt=None):
     """Gradients of s6_conv_scan_fwd for the loss sum(dy * y).  Returns the dict of
     s6_scan_bwd with dx [Bt, L, d] in place of du, plus dconv_w [d, K] and dconv_b
-    [d] (None without conv_b)."""
+    [d] (None without conv_b).  ckpt: the checkpoints of s6_conv_scan_fwd_ckpt on
+    the same inputs (h_init must then be None)."""
     torch = _torch()
     if x.dim() != 3:
         raise ValueError("x must be [batch, seqlen, d_inner]")
@@ -322,16 +368,17 @@ def s6_conv_scan_bwd(x, conv_w, conv_b, dt, A_log, B, C, D, dy, z=None, dt_bias=
          "dh_init": torch.empty((Bt, d, N), dtype=f32, device=dev) if want_dh_init else None}
     dims = Dims(Bt, L, d, N, K, _io_code(x))
     io = x.dtype
-    st = lib().s6_conv_scan_bwd(ctypes.byref(dims), _ptr(x, "x", io, seq, dev), _ptr(conv_w, "conv_w", f32, (d, K), dev),
+    fn, start = _bwd_start(lib().s6_conv_scan_bwd, lib().s6_conv_scan_bwd_ckpt, h_init, ckpt, Bt, L, d, N, dev)
+    st = fn(ctypes.byref(dims), _ptr(x, "x", io, seq, dev), _ptr(conv_w, "conv_w", f32, (d, K), dev),
                                 _ptr(conv_b, "conv_b", f32, (d,), dev), _ptr(dt, "dt", io, seq, dev),
                                 _ptr(A_log, "A_log", f32, (d, N), dev), _ptr(B, "B", io, (Bt, L, N), dev),
                                 _ptr(C, "C", io, (Bt, L, N), dev), _ptr(D, "D", f32, (d,), dev),
                                 _ptr(z, "z", io, seq, dev), _ptr(dt_bias, "dt_bias", f32, (d,), dev), int(zoh_mode),
-                                _ptr(h_init, "h_init", f32, (Bt, d, N), dev), _ptr(dy, "dy", io, seq, dev),
+                                start, _ptr(dy, "dy", io, seq, dev),
                                 *[_ptr(g[k], k) for k in ("dx", "dconv_w", "dconv_b", "ddt", "dz", "dB", "dC",
                                                           "dA_log", "dD", "ddt_bias", "dh_init")],
                                 _stream(stream, dev))
-    _check(st, "s6_conv_scan_bwd")
+    _check(st, fn.__name__)
     return g
 
 

@@ -350,8 +350,8 @@ int launch_scan_t(const s6_dims *dims, const void *x, const void *dt, const void
 template <typename IO, bool CONV, int MODE, int EXT>
 int launch_scan_n(const s6_dims *dims, const void *x, const void *dt, const void *z, void *y, const ScanArgs &a,
                   cudaStream_t st, const FixedScratch *fixed = nullptr) {
-    if constexpr (EXT == 2) {  // checkpoints: N = 16 only (checked by the caller)
-        return launch_scan_t<IO, 16, 2, CONV, MODE, 2>(dims, x, dt, z, y, a, st, fixed);
+    if constexpr (EXT >= 2) {  // checkpoints: N = 16 only (checked by the caller)
+        return launch_scan_t<IO, 16, 2, CONV, MODE, EXT>(dims, x, dt, z, y, a, st, fixed);
     } else {
         if (dims->d_state <= 4)
             return launch_scan_t<IO, 4, 1, CONV, MODE, EXT>(dims, x, dt, z, y, a, st, fixed);
@@ -373,7 +373,8 @@ bool few_chains(const s6_dims *dims) {
 
 template <typename IO>
 int launch_scan_io(const s6_dims *dims, bool conv, int mode, const void *x, const void *dt, const void *z, void *y,
-                   const ScanArgs &a, cudaStream_t st, const FixedScratch *fixed = nullptr) {
+                   const ScanArgs &a, cudaStream_t st, const FixedScratch *fixed = nullptr,
+                   bool ckpt_outputs = false) {
     using s6::kModeConst;
     using s6::kModeSimplified;
     using s6::kModeZOH;
@@ -381,7 +382,14 @@ int launch_scan_io(const s6_dims *dims, bool conv, int mode, const void *x, cons
         return (a.h_init || few_chains<IO>(dims)) ? launch_scan_n<IO, false, kModeConst, 1>(dims, x, dt, z, y, a, st, fixed)
                                                   : launch_scan_n<IO, false, kModeConst, 0>(dims, x, dt, z, y, a, st, fixed);
     const bool zoh = mode == kModeZOH;
-    if (a.ckpt) {  // the backward's checkpointing forward
+    if (a.ckpt && ckpt_outputs) {  // a training forward: outputs and checkpoints
+        if (conv)
+            return zoh ? launch_scan_n<IO, true, kModeZOH, 3>(dims, x, dt, z, y, a, st, fixed)
+                       : launch_scan_n<IO, true, kModeSimplified, 3>(dims, x, dt, z, y, a, st, fixed);
+        return zoh ? launch_scan_n<IO, false, kModeZOH, 3>(dims, x, dt, z, y, a, st, fixed)
+                   : launch_scan_n<IO, false, kModeSimplified, 3>(dims, x, dt, z, y, a, st, fixed);
+    }
+    if (a.ckpt) {  // the backward's checkpointing forward (no outputs)
         if (conv)
             return zoh ? launch_scan_n<IO, true, kModeZOH, 2>(dims, x, dt, z, y, a, st, fixed)
                        : launch_scan_n<IO, true, kModeSimplified, 2>(dims, x, dt, z, y, a, st, fixed);
@@ -410,7 +418,7 @@ int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv
                 const void *dt, const float *A_log, const void *B, const void *C, const float *D, const void *z,
                 const float *dt_bias, int mode, void *y, float *h_final, s6_stream_t stream,
                 const FixedScratch *fixed = nullptr, const float *h_init = nullptr,
-                const void *conv_hist = nullptr, float *ckpt = nullptr) {
+                const void *conv_hist = nullptr, float *ckpt = nullptr, bool ckpt_outputs = false) {
     int st = check_dims(dims, true, conv);
     if (st != S6_OK)
         return st;
@@ -475,8 +483,8 @@ int scan_common(const s6_dims *dims, bool conv, const void *x, const float *conv
     if (use_stream_device(s) != S6_OK)
         return S6_ERR_CUDA;
     if (dims->io_dtype == S6_BF16)
-        return launch_scan_io<__nv_bfloat16>(dims, conv, mode, x, dt, z, y, a, s, fixed);
-    return launch_scan_io<float>(dims, conv, mode, x, dt, z, y, a, s, fixed);
+        return launch_scan_io<__nv_bfloat16>(dims, conv, mode, x, dt, z, y, a, s, fixed, ckpt_outputs);
+    return launch_scan_io<float>(dims, conv, mode, x, dt, z, y, a, s, fixed, ckpt_outputs);
 }
 
 // ------------------------------------------------------------ step dispatch
@@ -776,23 +784,26 @@ int bwd_rev(const s6_dims *dims, bool conv, const void *x, const float *conv_w, 
             const float *A_log, const void *B, const void *C, const float *D, const void *z, const float *dt_bias,
             int zoh_mode, const float *h_init, const void *dy, float *dx, float *dconv_w, float *dconv_b, float *ddt,
             float *dz, float *dB, float *dC, float *dA_log, float *dD, float *ddt_bias, float *dh_init,
-            cudaStream_t s) {
+            cudaStream_t s, const float *ckpt_in = nullptr) {
     const int64_t Bt = dims->batch, L = dims->seqlen, d = dims->d_inner;
     const int64_t nck = (L + s6::kRevChunk - 1) / s6::kRevChunk;
     const int64_t tiles = (d + 63) / 64;
-    void *ck = nullptr, *pt = nullptr;
-    int rc = get_scratch(sizeof(float) * Bt * nck * d * 16, s, &ck, kScratchCkpt);
+    void *ck = const_cast<float *>(ckpt_in), *pt = nullptr;
+    int rc = ckpt_in ? S6_OK : get_scratch(sizeof(float) * Bt * nck * d * 16, s, &ck, kScratchCkpt);
     if (rc == S6_OK)
         rc = get_scratch(sizeof(float) * tiles * Bt * L * 32, s, &pt, kScratchPart);
     if (rc != S6_OK)
         return rc;
-    // 1. the forward with checkpoints (no outputs)
-    const s6_dims fd = *dims;
-    rc = scan_common(&fd, conv, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode,
-                     const_cast<void *>(x), nullptr, reinterpret_cast<s6_stream_t>(s), nullptr, h_init, nullptr,
-                     static_cast<float *>(ck));
-    if (rc != S6_OK)
-        return rc;
+    // 1. the forward with checkpoints (no outputs), unless the caller's training
+    // forward left them
+    if (!ckpt_in) {
+        const s6_dims fd = *dims;
+        rc = scan_common(&fd, conv, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode,
+                         const_cast<void *>(x), nullptr, reinterpret_cast<s6_stream_t>(s), nullptr, h_init, nullptr,
+                         static_cast<float *>(ck));
+        if (rc != S6_OK)
+            return rc;
+    }
     // 2. the reverse walk
     s6::RevArgs r;
     std::memset(&r, 0, sizeof(r));
@@ -851,12 +862,22 @@ int bwd_common(const s6_dims *dims, bool conv, const void *x, const float *conv_
                const void *dt, const float *A_log, const void *B, const void *C, const float *D, const void *z,
                const float *dt_bias, int zoh_mode, const float *h_init, const void *dy, float *dx,
                float *dconv_w, float *dconv_b, float *ddt, float *dz, float *dB, float *dC, float *dA_log, float *dD,
-               float *ddt_bias, float *dh_init, s6_stream_t stream) {
+               float *ddt_bias, float *dh_init, s6_stream_t stream, const float *ckpt_in = nullptr,
+               bool from_ckpt = false) {
     int st = check_dims(dims, true, conv);
     if (st != S6_OK)
         return st;
     if (zoh_mode != 0 && zoh_mode != 1)
         return S6_ERR_INVALID_ARG;
+    if (from_ckpt) {
+        // the checkpoints of a training forward: the pipelined backward only
+        if (!ckpt_in && dims->batch > 0 && dims->seqlen > 0)
+            return S6_ERR_INVALID_ARG;
+        if (dims->d_state != 16)
+            return S6_ERR_UNSUPPORTED;
+        if ((ckpt_in && !aligned16(ckpt_in)) || !bwd_rev_ok(dims, x, dt, z, dy, B, C))
+            return S6_ERR_ALIGNMENT;
+    }
     if (dims->batch == 0)
         return S6_OK;
     if (!x || !dt || !A_log || !B || !C || !D || !dy || !dx || !ddt || !dB || !dC || !dA_log || !dD || (z && !dz) ||
@@ -894,7 +915,7 @@ int bwd_common(const s6_dims *dims, bool conv, const void *x, const float *conv_
     }
     if (bwd_rev_ok(dims, x, dt, z, dy, B, C))
         return bwd_rev(dims, conv, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, h_init, dy, dx,
-                       dconv_w, dconv_b, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, s);
+                       dconv_w, dconv_b, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, s, ckpt_in);
     s6::BwdArgs a;
     std::memset(&a, 0, sizeof(a));
     a.Bt = static_cast<int>(Bt);
@@ -930,6 +951,29 @@ int bwd_common(const s6_dims *dims, bool conv, const void *x, const float *conv_
     if (dims->io_dtype == S6_BF16)
         return launch_bwd_io<__nv_bfloat16>(a, zoh_mode == 1, conv, s);
     return launch_bwd_io<float>(a, zoh_mode == 1, conv, s);
+}
+
+// The training forwards: the scan with its outputs, also storing the state
+// before every kCkptEvery-th token for a later s6_*_bwd_ckpt call.
+int fwd_ckpt_common(const s6_dims *dims, bool conv, const void *x, const float *conv_w, const float *conv_b,
+                    const void *dt, const float *A_log, const void *B, const void *C, const float *D, const void *z,
+                    const float *dt_bias, int zoh_mode, const float *h_init, void *y, float *h_final, float *ckpt,
+                    s6_stream_t stream) {
+    int st = check_dims(dims, true, conv);
+    if (st != S6_OK)
+        return st;
+    if (zoh_mode != 0 && zoh_mode != 1)
+        return S6_ERR_INVALID_ARG;
+    if (dims->d_state != 16)
+        return S6_ERR_UNSUPPORTED;
+    if (dims->batch > 0 && dims->seqlen > 0) {
+        if (!ckpt)
+            return S6_ERR_INVALID_ARG;
+        if (!aligned16(ckpt))
+            return S6_ERR_ALIGNMENT;
+    }
+    return scan_common(dims, conv, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, y, h_final, stream,
+                       nullptr, h_init, nullptr, ckpt, true);
 }
 
 extern "C" {
@@ -1037,6 +1081,42 @@ int s6_conv_scan_bwd(const s6_dims *dims, const void *x, const float *conv_w, co
     DeviceRestore restore_device;
     return bwd_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, h_init, dy, dx,
                       dconv_w, dconv_b, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, stream);
+}
+
+int s6_scan_fwd_ckpt(const s6_dims *dims, const void *u, const void *dt, const float *A_log, const void *B,
+                     const void *C, const float *D, const void *z, const float *dt_bias, int zoh_mode,
+                     const float *h_init, void *y, float *h_final, float *ckpt, s6_stream_t stream) {
+    DeviceRestore restore_device;
+    return fwd_ckpt_common(dims, false, u, nullptr, nullptr, dt, A_log, B, C, D, z, dt_bias, zoh_mode, h_init, y,
+                           h_final, ckpt, stream);
+}
+
+int s6_conv_scan_fwd_ckpt(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b,
+                          const void *dt, const float *A_log, const void *B, const void *C, const float *D,
+                          const void *z, const float *dt_bias, int zoh_mode, const float *h_init, void *y,
+                          float *h_final, float *ckpt, s6_stream_t stream) {
+    DeviceRestore restore_device;
+    return fwd_ckpt_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, h_init, y,
+                           h_final, ckpt, stream);
+}
+
+int s6_scan_bwd_ckpt(const s6_dims *dims, const void *u, const void *dt, const float *A_log, const void *B,
+                     const void *C, const float *D, const void *z, const float *dt_bias, int zoh_mode,
+                     const float *ckpt, const void *dy, float *du, float *ddt, float *dz, float *dB, float *dC,
+                     float *dA_log, float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream) {
+    DeviceRestore restore_device;
+    return bwd_common(dims, false, u, nullptr, nullptr, dt, A_log, B, C, D, z, dt_bias, zoh_mode, nullptr, dy, du,
+                      nullptr, nullptr, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, stream, ckpt, true);
+}
+
+int s6_conv_scan_bwd_ckpt(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b,
+                          const void *dt, const float *A_log, const void *B, const void *C, const float *D,
+                          const void *z, const float *dt_bias, int zoh_mode, const float *ckpt, const void *dy,
+                          float *dx, float *dconv_w, float *dconv_b, float *ddt, float *dz, float *dB, float *dC,
+                          float *dA_log, float *dD, float *ddt_bias, float *dh_init, s6_stream_t stream) {
+    DeviceRestore restore_device;
+    return bwd_common(dims, true, x, conv_w, conv_b, dt, A_log, B, C, D, z, dt_bias, zoh_mode, nullptr, dy, dx,
+                      dconv_w, dconv_b, ddt, dz, dB, dC, dA_log, dD, ddt_bias, dh_init, stream, ckpt, true);
 }
 
 int causal_conv1d_silu_fwd(const s6_dims *dims, const void *x, const float *conv_w, const float *conv_b, void *out,

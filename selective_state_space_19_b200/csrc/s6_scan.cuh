@@ -205,8 +205,10 @@ constexpr uint32_t kSleepNs = 1000u;
 
 // EXT: 0 the plain scan; 1 the extended scan, which may start from a given
 // state (h_init, conv_hist) and may take the associative split; 2 the
-// extended scan in checkpoint mode for the backward (N = 16 only).  Separate
-// instantiations, so that each one carries only its own code.
+// extended scan in checkpoint mode for the backward (N = 16 only, no
+// outputs); 3 the same with its outputs, a training forward whose checkpoints
+// the backward then reuses.  Separate instantiations, so that each one carries
+// only its own code.
 //
 // Registers: two CTAs of kScanBlock threads per SM allow 200 per thread; a
 // cap of 168 measured 0.8 % faster on the long-sequence workload than the
@@ -223,7 +225,8 @@ __global__ void __maxnreg__(168)
     constexpr bool ZOH = MODE == kModeZOH;
     constexpr bool CONSTD = MODE == kModeConst;  // decay from a constant, no step size
     constexpr bool INIT = EXT >= 1;  // given start state, associative split
-    constexpr bool CKPT = EXT == 2;  // checkpoints for the backward, no outputs
+    constexpr bool CKPT = EXT >= 2;   // the state before every kCkptEvery-th token
+    constexpr bool NOOUT = EXT == 2;  // the backward's own forward: no y, no readout
     static_assert(!CKPT || (NS == 16 && TPC == 2), "checkpoints are kept at N = 16 only");
     constexpr int NH = Sh::NH;
     constexpr int NP = NH / 2;  // state pairs per thread
@@ -713,8 +716,9 @@ __global__ void __maxnreg__(168)
             }
             const f2_t BIAS = f2_pack(bias, bias);
             auto silu2 = [&](f2_t v) {
-                // bfloat16 outputs take the tanh form; float32 outputs, and the
-                // backward's checkpoints, the exponential one
+                // bfloat16 outputs take the tanh form; float32 outputs, and any
+                // scan that keeps checkpoints (the backward recomputes from them
+                // with this form), the exponential one
                 if constexpr (sizeof(IO) == 2) {
                     if constexpr (CKPT)
                         return f2_silu_fast(v);
@@ -838,9 +842,9 @@ __global__ void __maxnreg__(168)
                             sdel += c1s.w;
                     }
                     // each thread finishes its own tokens: own partial + the partner's
-                    // (checkpoint mode writes no y, so the readout, the gate and z
-                    // are not computed at all there)
-                    if constexpr (!CKPT) {
+                    // (the backward's own forward writes no y, so the readout, the
+                    // gate and z are not computed at all there)
+                    if constexpr (!NOOUT) {
                         const float ra = __shfl_xor_sync(0xffffffffu, half ? acc0 : acc1, 1);
                         const float rb = __shfl_xor_sync(0xffffffffu, half ? acc2 : acc3, 1);
                         float ua, ub, ga, gb;
@@ -1053,7 +1057,7 @@ __global__ void __maxnreg__(168)
         __syncwarp();
         if (lane == 0) {
             mbar_arrive(&sm.empty[s]);
-            if (!CKPT && !(INIT && (m.w & kMetaNoY))) {
+            if (!NOOUT && !(INIT && (m.w & kMetaNoY))) {
                 if (c0 + warp * CPW < a.d) {  // a tile's last warps may lie past d
                     tma_store_3d(&tm_y, &sm.y[warp][c % kYBuf].v[0][0], c0 + warp * CPW, m.y, bseq);
                     bulk_commit_group();

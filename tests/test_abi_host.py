@@ -146,6 +146,46 @@ def test_from_state_and_backward_host_checks(lib):
     assert cbwd(conv_w=P(2)) == S.S6_ERR_ALIGNMENT
 
 
+def test_training_forward_and_backward_host_checks(lib):
+    """The checkpoint calls: N = 16 only, a checkpoint buffer that must be given
+    and 16-byte aligned, and the pipelined backward's row alignment -- all
+    refused before anything reaches the device."""
+    import selective_state_space_19_b200 as S
+    P = ctypes.c_void_p
+    ok = P(16)
+
+    def fwd(dims=None, zoh=0, ckpt=ok):  # s6_scan_fwd_ckpt
+        dd = ctypes.byref(dims or _dims())
+        return lib.s6_scan_fwd_ckpt(dd, ok, ok, ok, ok, ok, ok, None, None, zoh, None, ok, None, ckpt, None)
+    assert fwd(zoh=3) == S.S6_ERR_INVALID_ARG
+    assert fwd(dims=_dims(d_state=8)) == S.S6_ERR_UNSUPPORTED
+    assert fwd(ckpt=None) == S.S6_ERR_INVALID_ARG
+    assert fwd(ckpt=P(8)) == S.S6_ERR_ALIGNMENT
+    assert fwd(dims=_dims(batch=0), ckpt=None) == S.S6_OK  # nothing to do, nothing touched
+
+    def cfwd(ckpt=ok, conv_w=ok):  # s6_conv_scan_fwd_ckpt
+        return lib.s6_conv_scan_fwd_ckpt(ctypes.byref(_dims()), ok, conv_w, None, ok, ok, ok, ok, ok, None, None,
+                                         0, None, ok, None, ckpt, None)
+    assert cfwd(ckpt=P(4)) == S.S6_ERR_ALIGNMENT
+    assert cfwd(conv_w=None) == S.S6_ERR_INVALID_ARG
+
+    def bwd(dims=None, ckpt=ok, u=ok):  # s6_scan_bwd_ckpt
+        dd = ctypes.byref(dims or _dims())
+        return lib.s6_scan_bwd_ckpt(dd, u, ok, ok, ok, ok, ok, None, None, 0, ckpt, ok, ok, ok, None, ok, ok, ok,
+                                    ok, None, None, None)
+    assert bwd(ckpt=None) == S.S6_ERR_INVALID_ARG
+    assert bwd(dims=_dims(d_state=8)) == S.S6_ERR_UNSUPPORTED
+    assert bwd(ckpt=P(8)) == S.S6_ERR_ALIGNMENT
+    assert bwd(u=P(4)) == S.S6_ERR_ALIGNMENT               # rows the tensor unit moves
+    assert bwd(dims=_dims(d_inner=66)) == S.S6_ERR_ALIGNMENT  # 66 float32 is not a whole number of 16 bytes
+
+    def cbwd(ckpt=ok):  # s6_conv_scan_bwd_ckpt
+        return lib.s6_conv_scan_bwd_ckpt(ctypes.byref(_dims()), ok, ok, None, ok, ok, ok, ok, ok, None, None, 0,
+                                         ckpt, ok, ok, ok, None, ok, None, ok, ok, ok, ok, None, None, None)
+    assert cbwd(ckpt=None) == S.S6_ERR_INVALID_ARG
+    assert cbwd(ckpt=P(24)) == S.S6_ERR_ALIGNMENT
+
+
 def test_diag_and_block_host_checks(lib):
     """The constant-decay cell and the decode block reject bad arguments before
     any device call."""
