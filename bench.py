@@ -965,7 +965,8 @@ def run_profile_case(case):
     full workload's 384 chains, ~0.65 GB on the device); 'block' -- three decode
     token steps of 256 sequences through the 6 Mamba-mini blocks; 'mamba_mini'
     -- three fused scans of the Mamba-mini block workload (Bt8 L256 d1536,
-    float32)."""
+    float32); 'diag' -- three constant-decay cells on the long_seq recipe at
+    L = 2048 (50M elements; u, z, y 300 MB, larger than L2)."""
     import torch
     import selective_state_space_19_b200 as S
     dev = torch.device("cuda", 0)
@@ -975,6 +976,13 @@ def run_profile_case(case):
         for _ in range(3):
             S.s6_conv_scan_fwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"],
                                z=t["z"], dt_bias=t["dt_bias"])
+    elif case == "diag":
+        inp = SI.scan_inputs("long_seq", L=2048)
+        t = {k: to_dev(inp[k], dev) for k in ("x", "z", "B", "C", "D")}
+        w = to_dev(SI.diag_log2_decay(inp["x"].shape[2], 16), dev)
+        for _ in range(3):
+            S.s6_diag_recurrence_fwd(t["x"], t["B"], t["C"], t["D"], decay_source=S.S6_DECAY_CONST, log2_decay=w,
+                                     z=t["z"])
     elif case == "bwd":
         inp = SI.scan_inputs("long_seq", Bt=16, L=1024, seed=3)
         t = {k: to_dev(inp[k], dev) for k in ("x", "z", "B", "C", "dt", "A_log", "D", "dt_bias")}
@@ -1004,9 +1012,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["full", "small", "bwd", "block", "mamba_mini"], default="full",
-                    help="small: the workload at L=2048 (for ncu captures); bwd, block, mamba_mini: small cases "
-                         "of the backward, the decode block and the Mamba-mini scan for captures (no JSON line)")
+    ap.add_argument("--case", choices=["full", "small", "bwd", "block", "mamba_mini", "diag"], default="full",
+                    help="small: the workload at L=2048 (for ncu captures); bwd, block, mamba_mini, diag: small "
+                         "cases of the backward, the decode block, the Mamba-mini scan and the constant-decay cell "
+                         "for captures (no JSON line)")
     ap.add_argument("--no-rows", action="store_true", help="skip the decode-step and standalone-conv rows")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1014,7 +1023,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
-    if args.case in ("bwd", "block", "mamba_mini"):
+    if args.case in ("bwd", "block", "mamba_mini", "diag"):
         return run_profile_case(args.case)
     return run_ours(args)
 
