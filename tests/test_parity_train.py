@@ -80,17 +80,12 @@ def _check_grads(io, got, ref, keys, what):
         assert err <= GTOL, f"{what} {k}: max|g-ref|/(1+|ref|) = {err:.3e}"
 
 
-@pytest.mark.parametrize("io", ["f32", "bf16"])
-@pytest.mark.parametrize("zoh", [False, True])
-@pytest.mark.parametrize("conv", [False, True])
-def test_train_step_matches_oracle(io, zoh, conv):
+def _train_case(io, zoh, conv, Bt, L, d, seed):
     """Forward with checkpoints, then the backward from them: y, h_final, every
-    kept state, and every gradient (Bt 2, L 150: the last group holds 6 tokens;
-    a start state)."""
+    kept state and every gradient against the oracle (with a start state)."""
     import torch
     import selective_state_space_19_b200 as S
-    Bt, L, d = 2, 150, 64
-    inp, dy, h0 = _inputs(io, Bt, L, d, seed=170 + 2 * int(zoh) + int(conv))
+    inp, dy, h0 = _inputs(io, Bt, L, d, seed=seed)
     t = dev_inputs(inp)
     y, h, ck = _train_fwd(S, t, conv, zoh, to_dev(h0))
     torch.cuda.synchronize()
@@ -110,7 +105,36 @@ def test_train_step_matches_oracle(io, zoh, conv):
         keys = ("du", "ddt", "dz", "dB", "dC", "dA_log", "dD", "ddt_bias", "dh_init")
     torch.cuda.synchronize()
     assert S.s6_device_status() == 0
-    _check_grads(io, got, ref, keys, f"io={io} zoh={zoh} conv={conv}")
+    _check_grads(io, got, ref, keys, f"io={io} zoh={zoh} conv={conv} Bt={Bt} L={L} d={d}")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("zoh", [False, True])
+@pytest.mark.parametrize("conv", [False, True])
+def test_train_step_matches_oracle(io, zoh, conv):
+    """Bt 2, L 150 (the last group of 16 tokens holds 6), 64 channels."""
+    _train_case(io, zoh, conv, Bt=2, L=150, d=64, seed=170 + 2 * int(zoh) + int(conv))
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [dict(Bt=3, L=17, d=40, zoh=True, conv=True),     # a tile of 40 channels
+                                   dict(Bt=1, L=1, d=72, zoh=False, conv=False),     # one token, a ragged tile
+                                   dict(Bt=2, L=16, d=136, zoh=False, conv=True)])   # exactly one group
+def test_train_step_ragged_shapes(io, shape):
+    sh = dict(shape)
+    _train_case(io, sh.pop("zoh"), sh.pop("conv"), seed=200 + sh["L"] + sh["d"], **sh)
+
+
+def test_train_forward_empty_sequence():
+    """L = 0: no checkpoints, h_final is the start state."""
+    import torch
+    import selective_state_space_19_b200 as S
+    inp, _, h0 = _inputs("f32", 2, 0, 64, seed=5)
+    t = dev_inputs(inp)
+    y, h, ck = _train_fwd(S, t, True, False, to_dev(h0))
+    torch.cuda.synchronize()
+    assert tuple(ck.shape) == (2, 0, 64, 16) and y.numel() == 0
+    assert np.array_equal(h.cpu().numpy(), h0)
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
