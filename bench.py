@@ -388,8 +388,9 @@ def row_bwd(device, stream, pk, inp_dev, cfg, iters=3, fused=False):
     ex2_per_s = elems * N / (ms * 1e-3)
     peak_ex2 = SMS * MUFU_PER_SM_CLK * pk["sm_max_mhz"] * 1e6
     name = "s6_conv_scan_bwd (conv4 + SiLU + scan)" if fused else "s6_scan_bwd"
+    write = "exact ZOH write" if zoh else "simplified write"
     return {"workload": f"{name} on long_seq (Bt16 L8192 d1536 N16, bf16 in, float32 gradients, gate, "
-                        "simplified write): all gradients of sum(dy * y)",
+                        f"{write}): all gradients of sum(dy * y)",
             "value": elems / (ms * 1e-3) / 1e9, "unit": "Gelem/s", "ms_per_launch": ms,
             "roofline": {"bound": "alu", "achieved": ex2_per_s / 1e12, "peak": peak_ex2 / 1e12, "unit": "Tex2/s",
                          "frac": ex2_per_s / peak_ex2,
@@ -927,6 +928,7 @@ def run_ours(args):
         rows["s6_conv_scan_fwd_from_state"] = row_prefill(device, stream, pk, t, cfg)
         rows["s6_scan_bwd"] = row_bwd(device, stream, pk, t, cfg)
         rows["s6_conv_scan_bwd"] = row_bwd(device, stream, pk, t, cfg, fused=True)
+        rows["s6_conv_scan_bwd_zoh"] = row_bwd(device, stream, pk, t, dict(cfg, zoh=True), fused=True)
         rows["train_step_conv_scan"] = row_train(device, stream, pk, t, cfg)
 
     cpu = None

@@ -142,8 +142,12 @@ __device__ __forceinline__ float zoh_dgain_dA_rev(float x, float a, float delta,
 }
 
 
+// Registers: the register file is allotted per SM sub-partition (16,384
+// each), and two CTAs of five warps put two warps of a CTA on one of them, so
+// 168 a thread is the most that keeps two CTAs per SM (the exact-ZOH fused
+// instantiation would otherwise take 181 and run one CTA per SM).
 template <typename IO, bool ZOH, bool CONV>
-__global__ void __launch_bounds__(kScanBlock, 1)
+__global__ void __maxnreg__(168)
     s6_scan_bwd_rev_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_dt,
                            const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_dy,
                            const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
@@ -517,6 +521,14 @@ __global__ void __launch_bounds__(kScanBlock, 1)
             // ---- 3. walk the sub-chunk back
             // h_t of the token being walked back; h_{t-1} becomes the next token's h_t
             float4 h0 = hb[tc][0][lane], h1 = hb[tc][1][lane];
+            // the conv window: x rows j+1 .. j+3 of token j kept from the token
+            // after it, so that each token reads one new row (row j)
+            float xr1 = 0.f, xr2 = 0.f, xr3 = 0.f;
+            if (CONV) {
+                xr1 = ld(xs, tc);
+                xr2 = ld(xs, tc + 1);
+                xr3 = ld(xs, tc + 2);
+            }
 #pragma unroll 2
             for (int j = tc - 1; j >= 0; --j) {
                 const float4 du = tb[j][cw];
@@ -594,14 +606,18 @@ __global__ void __launch_bounds__(kScanBlock, 1)
                 const float dv = ddel * sig_v;
                 float dxo = dut;
                 if (CONV) {
-                    const float pre = pre_at(j);
+                    const float xr0 = ld(xs, j);
+                    const float pre = fmaf(w3, xr3, fmaf(w2, xr2, fmaf(w1, xr1, fmaf(w0, xr0, cbv))));
                     const float sp_ = rcp_approx(1.0f + ex2_approx(fminf(-pre * kLog2e, 120.0f)));
                     const float dpre = dut * sp_ * fmaf(pre, 1.0f - sp_, 1.0f);  // SiLU'(pre)
                     dxo = fmaf(w3, dpre, fmaf(w2, dp1, fmaf(w1, dp2, w0 * dp3)));
-                    dW0 = fmaf(dpre, ld(xs, j), dW0);
-                    dW1 = fmaf(dpre, ld(xs, j + 1), dW1);
-                    dW2 = fmaf(dpre, ld(xs, j + 2), dW2);
-                    dW3 = fmaf(dpre, ld(xs, j + 3), dW3);
+                    dW0 = fmaf(dpre, xr0, dW0);
+                    dW1 = fmaf(dpre, xr1, dW1);
+                    dW2 = fmaf(dpre, xr2, dW2);
+                    dW3 = fmaf(dpre, xr3, dW3);
+                    xr3 = xr2;
+                    xr2 = xr1;
+                    xr1 = xr0;
                     dcb += dpre;
                     dp3 = dp2;
                     dp2 = dp1;
