@@ -133,11 +133,13 @@ __device__ __forceinline__ int reduce_scatter16_index(int lane) {
 // d gain / dA at fixed Delta for the exact ZOH write, gain = (e^x - 1)/A with
 // x = Delta A: (x e^x - (e^x - 1))/A^2 = Delta^2 (1/2 + x/3 + x^2/8 + x^3/30 +
 // x^4/144 + ...); the series for |x| < 1/4 (truncation below 3e-6 relative),
-// where the closed form cancels in float32.  e^x is the decay a.
-__device__ __forceinline__ float zoh_dgain_dA_rev(float x, float a, float delta, float A) {
+// where the closed form cancels in float32.  e^x is the decay a; 1/A^2 is
+// taken as nrA^2 with nrA = -1/A, which the walk holds per state, instead of a
+// division per state and token.
+__device__ __forceinline__ float zoh_dgain_dA_rev(float x, float a, float delta, float nrA) {
     const float p = fmaf(fmaf(fmaf(fmaf(x, 1.0f / 144.0f, 1.0f / 30.0f), x, 0.125f), x, 1.0f / 3.0f), x, 0.5f);
     const float series = delta * delta * p;
-    const float closed = (x * a - (a - 1.0f)) / (A * A);
+    const float closed = (x * a - (a - 1.0f)) * (nrA * nrA);
     return fabsf(x) < 0.25f ? series : closed;
 }
 
@@ -573,12 +575,13 @@ __global__ void __maxnreg__(168)
                     acc_q = f2_fma(qv, Ap[q], acc_q);
                     dAacc[q] = f2_fma(qv, dd, dAacc[q]);
                     if (ZOH) {
-                        float g0, g1, A0, A1, ab0, ab1, dhb0, dhb1;
+                        float g0, g1, A0, A1, nr0, nr1, ab0, ab1, dhb0, dhb1;
                         f2_unpack(Ap[q], A0, A1);
+                        f2_unpack(nrAp[q], nr0, nr1);
                         f2_unpack(ab, ab0, ab1);
                         f2_unpack(f2_mul(f2_mul(dh, Bq[q]), uu), dhb0, dhb1);
-                        g0 = dhb0 * zoh_dgain_dA_rev(delta * A0, ab0, delta, A0);
-                        g1 = dhb1 * zoh_dgain_dA_rev(delta * A1, ab1, delta, A1);
+                        g0 = dhb0 * zoh_dgain_dA_rev(delta * A0, ab0, delta, nr0);
+                        g1 = dhb1 * zoh_dgain_dA_rev(delta * A1, ab1, delta, nr1);
                         dAacc[q] = f2_add(dAacc[q], f2_pack(g0, g1));
                     }
                     gcar[q] = f2_mul(dh, ab);
