@@ -690,7 +690,12 @@ __global__ void __launch_bounds__(kTcThreads) q8_tc_gemm_kernel(const Q8GemmArgs
         }
     }
 
-    // accumulator (i, j): rows wm + 16 i + g (+8), columns wn + 8 j + 2 t (+1)
+    // accumulator (i, j): rows wm + 16 i + g (+8), columns wn + 8 j + 2 t (+1);
+    // a split reduction adds a thread's two adjacent columns with one 8-byte
+    // atomic when the output rows allow it (half the atomic operations; 16-byte
+    // atomics after a lane-pair exchange measured slower)
+    const bool pairs =
+        a.accumulate && ((reinterpret_cast<uintptr_t>(a.y) | static_cast<uintptr_t>(a.ldy) * 4u) & 7u) == 0;
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
@@ -701,6 +706,11 @@ __global__ void __launch_bounds__(kTcThreads) q8_tc_gemm_kernel(const Q8GemmArgs
                 const int m = m0 + wm + 16 * i + g + 8 * hrow;
                 if (m >= a.M)
                     continue;
+                if (pairs && n + 1 < a.N) {
+                    float2 *dst = reinterpret_cast<float2 *>(a.y + static_cast<size_t>(m) * a.ldy + n);
+                    atomicAdd(dst, make_float2(acc[i][j][2 * hrow] * a.ws[n], acc[i][j][2 * hrow + 1] * a.ws[n + 1]));
+                    continue;
+                }
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     if (n + e >= a.N)

@@ -73,6 +73,15 @@ def test_block_xproj_row_paths():
     _run(Bt=3, dm=40, di=90, N=16, R=6, K=4, blocks=1, steps=2, seed=18)
 
 
+def test_block_product_epilogue_paths():
+    """The tensor-core product's split-reduction adds: 8-byte atomics on rows
+    of an even length (every test above), and single floats where d_model 45
+    makes out_proj's rows (the residual stream, K = d_inner 96 on the tensor
+    cores) only 4-byte aligned."""
+    _run(Bt=5, dm=45, di=96, N=16, R=4, K=4, blocks=2, steps=2, seed=19)
+    _run(Bt=70, dm=40, di=128, N=16, R=8, K=4, blocks=1, steps=2, seed=20)
+
+
 def test_block_mamba_mini_dims():
     """The Mamba-mini block (d_model 384, d_inner 1536, N 16, dt rank 24, conv 4)
     through all 6 blocks for 6 tokens, on a 16-sequence batch."""
