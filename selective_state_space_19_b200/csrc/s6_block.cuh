@@ -46,10 +46,12 @@ __device__ __forceinline__ float4 i8x4_to_f32x4(int w) {
 constexpr int kLnThreads = 256;  // 8 rows per block, a warp per row
 
 constexpr int kLnPerLane = 32;   // rows up to 1024 values are held in registers
+constexpr int kLnVec = 4;        // float4 per lane of the vector path (rows up to 512 values)
 
 // out[m] = (x[m] - mean) / sqrt(var + eps) * w + b (biased variance).  The
 // row is read once into registers (two-pass statistics from them); longer
-// rows are read again for each pass.
+// rows are read again for each pass.  Rows of up to 512 values in whole
+// 16-byte units move as float4, with the weights and biases loaded alongside.
 __global__ void __launch_bounds__(kLnThreads) block_layernorm_kernel(const float *x, const float *w, const float *b,
                                                                      float *out, int M, int K, float eps) {
     const int m = blockIdx.x * (kLnThreads / 32) + (threadIdx.x >> 5);
@@ -58,6 +60,54 @@ __global__ void __launch_bounds__(kLnThreads) block_layernorm_kernel(const float
         return;
     const float *xr = x + static_cast<size_t>(m) * K;
     float *orow = out + static_cast<size_t>(m) * K;
+    if (K % 4 == 0 && K <= 32 * 4 * kLnVec &&
+        ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(b) |
+          reinterpret_cast<uintptr_t>(out)) & 15u) == 0) {
+        // the row, the weights and the biases as float4, all loads issued first
+        const int K4 = K / 4;
+        const float4 *x4 = reinterpret_cast<const float4 *>(xr);
+        float4 v[kLnVec], wv[kLnVec], bv[kLnVec];
+        const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < kLnVec; ++i) {
+            const int k4 = lane + 32 * i;
+            const bool in = k4 < K4;
+            v[i] = in ? x4[k4] : zero;
+            wv[i] = in ? reinterpret_cast<const float4 *>(w)[k4] : zero;
+            bv[i] = in ? reinterpret_cast<const float4 *>(b)[k4] : zero;
+        }
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < kLnVec; ++i)
+            s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+#pragma unroll
+        for (int o = 16; o; o >>= 1)
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+        const float mean = s / K;
+        float q = 0.f;
+#pragma unroll
+        for (int i = 0; i < kLnVec; ++i) {
+            if (lane + 32 * i < K4) {
+                const float d0 = v[i].x - mean, d1 = v[i].y - mean, d2 = v[i].z - mean, d3 = v[i].w - mean;
+                q = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, q))));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1)
+            q += __shfl_xor_sync(0xffffffffu, q, o);
+        const float r = rsqrtf(q / K + eps);
+        float4 *o4 = reinterpret_cast<float4 *>(orow);
+#pragma unroll
+        for (int i = 0; i < kLnVec; ++i) {
+            const int k4 = lane + 32 * i;
+            if (k4 < K4)
+                o4[k4] = make_float4(fmaf((v[i].x - mean) * r, wv[i].x, bv[i].x),
+                                     fmaf((v[i].y - mean) * r, wv[i].y, bv[i].y),
+                                     fmaf((v[i].z - mean) * r, wv[i].z, bv[i].z),
+                                     fmaf((v[i].w - mean) * r, wv[i].w, bv[i].w));
+        }
+        return;
+    }
     if (K <= 32 * kLnPerLane) {
         float v[kLnPerLane];
 #pragma unroll
