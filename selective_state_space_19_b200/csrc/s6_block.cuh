@@ -27,7 +27,9 @@
 
 namespace s6 {
 
-__device__ __forceinline__ float silu_exact(float v) { return v / (1.0f + __expf(-v)); }
+// SiLU(v) = v / (1 + e^-v), with the fast division (about 2 ulp; 0 for v
+// below about -88, where e^-v overflows and SiLU is 0 to float precision)
+__device__ __forceinline__ float silu_exact(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
 
 // Four int8 values (bytes of w, lowest first) as floats without the
 // conversion unit: each byte, biased to unsigned (b + 128), is placed under the
@@ -361,6 +363,7 @@ __global__ void __launch_bounds__(kConvXThreads, 2) block_conv_xproj_kernel(
         const float *srow = xcs + ((di + 3) & ~3);
         const float *Bm = srow + sa.R, *Cm = srow + sa.R + 16;
         const bool vec_dt = (sa.R % 4) == 0 && (reinterpret_cast<uintptr_t>(sa.dt_q) & 3) == 0;
+        const bool vec_bc = (sa.R % 4) == 0;  // the x_proj row in shared memory starts 16-byte aligned
         for (int c0 = threadIdx.x; c0 < di; c0 += 2 * kConvXThreads) {
             float4 h4[2][4], a4[2][4];
             float zv[2];
@@ -407,12 +410,24 @@ __global__ void __launch_bounds__(kConvXThreads, 2) block_conv_xproj_kernel(
                 for (int q4 = 0; q4 < 4; ++q4) {
                     float hh[4] = {h4[k][q4].x, h4[k][q4].y, h4[k][q4].z, h4[k][q4].w};
                     const float aa[4] = {a4[k][q4].x, a4[k][q4].y, a4[k][q4].z, a4[k][q4].w};
+                    float bq[4], cq[4];
+                    if (vec_bc) {  // B and C rows as 16-byte reads (R a multiple of 4)
+                        const float4 b4 = reinterpret_cast<const float4 *>(Bm)[q4];
+                        const float4 c4 = reinterpret_cast<const float4 *>(Cm)[q4];
+                        bq[0] = b4.x, bq[1] = b4.y, bq[2] = b4.z, bq[3] = b4.w;
+                        cq[0] = c4.x, cq[1] = c4.y, cq[2] = c4.z, cq[3] = c4.w;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            bq[e] = Bm[4 * q4 + e];
+                            cq[e] = Cm[4 * q4 + e];
+                        }
+                    }
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int n = 4 * q4 + e;
                         const float ab = ex2_approx(dl2 * __expf(aa[e]));  // exp(Delta A), A = -exp(A_log)
-                        hh[e] = fmaf(ab, hh[e], du * Bm[n]);
-                        acc = fmaf(hh[e], Cm[n], acc);
+                        hh[e] = fmaf(ab, hh[e], du * bq[e]);
+                        acc = fmaf(hh[e], cq[e], acc);
                     }
                     if (c < di)
                         hp[q4] = make_float4(hh[0], hh[1], hh[2], hh[3]);
