@@ -296,20 +296,22 @@ __global__ void __launch_bounds__(kConvXThreads, 2) block_conv_xproj_kernel(
         for (int o = warp; o < n_out; o += kConvXThreads / 32) {
             if (o + kConvXThreads / 32 < n_out)
                 fetch(o + kConvXThreads / 32, wn);
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            // the four column accumulators as two packed pairs
+            f2_t acc01 = f2_pack(0.f, 0.f), acc23 = acc01;
 #pragma unroll
             for (int k = 0; k < kXprojIt; ++k) {
                 const int c4 = lane + 32 * k;
                 if (c4 < n4) {
                     const float4 wv = i8x4_to_f32x4(wq[k]);
                     const float4 xv = x4[c4];
-                    acc[0] = fmaf(wv.x, xv.x, acc[0]);
-                    acc[1] = fmaf(wv.y, xv.y, acc[1]);
-                    acc[2] = fmaf(wv.z, xv.z, acc[2]);
-                    acc[3] = fmaf(wv.w, xv.w, acc[3]);
+                    acc01 = f2_fma(f2_pack(wv.x, wv.y), f2_pack(xv.x, xv.y), acc01);
+                    acc23 = f2_fma(f2_pack(wv.z, wv.w), f2_pack(xv.z, xv.w), acc23);
                 }
             }
-            float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            float a0, a1, a2, a3;
+            f2_unpack(acc01, a0, a1);
+            f2_unpack(acc23, a2, a3);
+            float sum = (a0 + a1) + (a2 + a3);
 #pragma unroll
             for (int off = 16; off; off >>= 1)
                 sum += __shfl_xor_sync(0xffffffffu, sum, off);
@@ -404,7 +406,8 @@ __global__ void __launch_bounds__(kConvXThreads, 2) block_conv_xproj_kernel(
                 const float x_c = xcs[cc[k]];
                 const float du = delta * x_c;
                 const float dl2 = -delta * kLog2e;
-                float acc = 0.f;
+                const f2_t l2e2 = f2_pack(kLog2e, kLog2e), dl22 = f2_pack(dl2, dl2), du2 = f2_pack(du, du);
+                f2_t acc2 = f2_pack(0.f, 0.f);
                 float4 *hp = reinterpret_cast<float4 *>(sa.h + (static_cast<size_t>(m) * di + cc[k]) * 16);
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
@@ -423,17 +426,25 @@ __global__ void __launch_bounds__(kConvXThreads, 2) block_conv_xproj_kernel(
                             cq[e] = Cm[4 * q4 + e];
                         }
                     }
+                    // two states at a time: exp(A_log) = 2^(A_log log2 e) = -A, then
+                    // exp(Delta A) = 2^(-Delta log2 e exp(A_log)); update and readout
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float ab = ex2_approx(dl2 * __expf(aa[e]));  // exp(Delta A), A = -exp(A_log)
-                        hh[e] = fmaf(ab, hh[e], du * bq[e]);
-                        acc = fmaf(hh[e], cq[e], acc);
+                    for (int e = 0; e < 4; e += 2) {
+                        float t0, t1;
+                        f2_unpack(f2_mul(f2_pack(aa[e], aa[e + 1]), l2e2), t0, t1);
+                        f2_unpack(f2_mul(dl22, f2_pack(ex2_approx(t0), ex2_approx(t1))), t0, t1);
+                        const f2_t ab = f2_pack(ex2_approx(t0), ex2_approx(t1));
+                        const f2_t h2 = f2_fma(ab, f2_pack(hh[e], hh[e + 1]), f2_mul(du2, f2_pack(bq[e], bq[e + 1])));
+                        acc2 = f2_fma(h2, f2_pack(cq[e], cq[e + 1]), acc2);
+                        f2_unpack(h2, hh[e], hh[e + 1]);
                     }
                     if (c < di)
                         hp[q4] = make_float4(hh[0], hh[1], hh[2], hh[3]);
                 }
+                float acc0, acc1;
+                f2_unpack(acc2, acc0, acc1);
                 if (c < di)
-                    sa.g[static_cast<size_t>(m) * sa.g_ld + c] = fmaf(sa.D[c], x_c, acc) * silu_exact(zv[k]);
+                    sa.g[static_cast<size_t>(m) * sa.g_ld + c] = fmaf(sa.D[c], x_c, acc0 + acc1) * silu_exact(zv[k]);
             }
         }
     }
