@@ -968,7 +968,10 @@ def run_profile_case(case):
     token steps of 256 sequences through the 6 Mamba-mini blocks; 'mamba_mini'
     -- three fused scans of the Mamba-mini block workload (Bt8 L256 d1536,
     float32); 'diag' -- three constant-decay cells on the long_seq recipe at
-    L = 2048 (50M elements; u, z, y 300 MB, larger than L2)."""
+    L = 2048 (50M elements; u, z, y 300 MB, larger than L2); 'train' -- three
+    training steps of the fused path (s6_conv_scan_fwd_ckpt, then
+    s6_conv_scan_bwd from its checkpoints) on the long_seq recipe at Bt16
+    L1024."""
     import torch
     import selective_state_space_19_b200 as S
     dev = torch.device("cuda", 0)
@@ -978,6 +981,15 @@ def run_profile_case(case):
         for _ in range(3):
             S.s6_conv_scan_fwd(t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"],
                                z=t["z"], dt_bias=t["dt_bias"])
+    elif case == "train":
+        inp = SI.scan_inputs("long_seq", Bt=16, L=1024, seed=3)
+        t = {k: to_dev(inp[k], dev) for k in ("x", "z", "B", "C", "dt", "A_log", "D", "dt_bias", "conv_w", "conv_b")}
+        gen = torch.Generator(device=dev).manual_seed(7)
+        dy = torch.randn(16, 1024, 1536, device=dev, generator=gen).to(torch.bfloat16)
+        args = (t["x"], t["conv_w"], t["conv_b"], t["dt"], t["A_log"], t["B"], t["C"], t["D"])
+        for _ in range(3):
+            _, _, ck = S.s6_conv_scan_fwd_ckpt(*args, z=t["z"], dt_bias=t["dt_bias"])
+            S.s6_conv_scan_bwd(*args, dy, z=t["z"], dt_bias=t["dt_bias"], ckpt=ck)
     elif case == "diag":
         inp = SI.scan_inputs("long_seq", L=2048)
         t = {k: to_dev(inp[k], dev) for k in ("x", "z", "B", "C", "D")}
@@ -1014,10 +1026,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--case", choices=["full", "small", "bwd", "block", "mamba_mini", "diag"], default="full",
-                    help="small: the workload at L=2048 (for ncu captures); bwd, block, mamba_mini, diag: small "
-                         "cases of the backward, the decode block, the Mamba-mini scan and the constant-decay cell "
-                         "for captures (no JSON line)")
+    ap.add_argument("--case", choices=["full", "small", "bwd", "block", "mamba_mini", "diag", "train"],
+                    default="full",
+                    help="small: the workload at L=2048 (for ncu captures); bwd, block, mamba_mini, diag, train: "
+                         "small cases of the backward, the decode block, the Mamba-mini scan, the constant-decay "
+                         "cell and a training step for captures (no JSON line)")
     ap.add_argument("--no-rows", action="store_true", help="skip the decode-step and standalone-conv rows")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1025,7 +1038,7 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
-    if args.case in ("bwd", "block", "mamba_mini", "diag"):
+    if args.case in ("bwd", "block", "mamba_mini", "diag", "train"):
         return run_profile_case(args.case)
     return run_ours(args)
 
