@@ -859,7 +859,7 @@ def run_ours(args):
         # device copies, the scan, device-to-host copies -- so that the copies of
         # one chunk overlap the scan of another and the two directions overlap
         # each other.  Each chunk is one s6_conv_scan_fwd call on its sequences.
-        nch = 4 if Bt % 4 == 0 else 1
+        nch = max(c for c in (1, 2, 4, 8, 16, 32) if c <= args.e2e_chunks and Bt % c == 0)
         cb = Bt // nch
         s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
         ev_in = [torch.cuda.Event() for _ in range(nch)]
@@ -1035,6 +1035,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-chunks", type=int, default=16,
+                    help="chunks of sequences in the end-to-end pipeline (the largest of 1, 2, 4, ... 32 that is at "
+                         "most this and divides the batch)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
